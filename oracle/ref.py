@@ -1,0 +1,421 @@
+"""Plain float64 CPU oracle of causal attention with RoPE at remapped positions.
+
+TEST INFRASTRUCTURE ONLY: imported by the tests, by ``__graft_entry__.smoke()``
+and by the CPU-baseline leg of ``bench.py``; never by the product path. It
+shares no code, table or constant generator with the CUDA library.
+
+What it computes, and where each step is defined:
+
+* RoPE frequencies theta_i = base^(-2i/d), i = 0..d/2-1, and the
+  block-diagonal 2x2 rotation R_t acting on coordinate pairs (2i, 2i+1):
+  "Periodic RoPE for Infinite Context LLMs", §3.1 Eq. 1-2.
+* Position interpolation divides every position by the factor s ("linearly
+  compresses positions into the pretrained range"): "Jet-Long: Efficient
+  Long-Context Extension with Dynamic Bifocal RoPE", §2.2; used by
+  "EndPrompt: Efficient Long-Context Extension via Terminal Anchoring",
+  abstract and summary ("combined with RoPE interpolation").
+* Periodic position phi(t) = t mod W inside causal sliding-window attention
+  over the W keys {t-W+1 .. t}: Periodic RoPE, §3.2 Eq. 4-5.
+* NoPE causal attention A_ts = q.k / sqrt(d_h), s <= t: Periodic RoPE, §3.3
+  Eq. 6 (this also fixes the softmax scale 1/sqrt(d) for every kind).
+* EndPrompt two-segment positions: an intact first segment at 0..n1-1, then
+  a terminal segment whose positions start near the target length
+  (EndPrompt, abstract).
+* Bifocal score: RoPE at (q, k) when q - k <= w0, else RoPE at (f(q), f(k)),
+  with G = max(1, ceil(L / w_pretrained)) and f(x) = floor(x / G): Jet-Long,
+  §3 Eq. 1, §3.1 Eq. 2-3.
+* Decode with an untouched cache k_cache[k] = RoPE(x_k, k) and the correction
+  rotation by Delta = f(x) - x on the query and on each cached key: Jet-Long,
+  §3.2 Eq. 4-6.
+* The literal three-call inclusion-exclusion merge: Jet-Long, §3.3 Eq. 7
+  (kept as a self-check; the routed softmax is the definition it reaches).
+
+Readings where the pages leave a step open (each listed in the design notes):
+adjacent pairing (2i, 2i+1); natural-log LSE of the scaled scores; the local
+set of the bifocal score is 0 <= q-k <= w0 inclusive; for prefill L = S; for
+decode L = n, the cache length including the current token at n-1.
+
+Floating point: everything is float64. ``stage_bf16=True`` rounds the rotated
+q and k to bfloat16 (round to nearest even) before the dot products, because
+the tensor-core prefill multiplies bf16 operands; this is a modelled input
+rounding, not a change of the method.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+STANDARD, ENDPROMPT, PERIODIC, NOPE, BIFOCAL = 0, 1, 2, 3, 4
+
+__all__ = [
+    "STANDARD", "ENDPROMPT", "PERIODIC", "NOPE", "BIFOCAL",
+    "round_bf16", "rope_frequencies", "rotation_matrix", "rotate",
+    "periodic_position", "endprompt_position", "group_size", "remote_position",
+    "position_maps", "softmax_scale", "prefill", "prefill_three_call",
+    "decode", "brute_prefill", "brute_decode", "to_f64",
+]
+
+
+# ----------------------------------------------------------------------------
+# helpers
+# ----------------------------------------------------------------------------
+def to_f64(x) -> np.ndarray:
+    """torch tensor (any dtype, any device) or array -> float64 numpy."""
+    if hasattr(x, "detach"):
+        return x.detach().to("cpu").double().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to the nearest bfloat16 (8 significant bits), ties
+    to even. Written out with frexp so no library conversion is involved.
+    Valid for normal-range values (|x| >= 2^-126 or x == 0), which is all the
+    oracle ever rounds."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)                   # x = m * 2^e, 0.5 <= |m| < 1
+    r = np.round(m * 256.0)              # 8 significant bits; np.round is half-to-even
+    return np.ldexp(r, e - 8)
+
+
+def softmax_scale(D: int, params) -> float:
+    """Periodic RoPE, §3.3 Eq. 6: scores are divided by sqrt(d_h)."""
+    s = float(getattr(params, "softmax_scale", 0.0) or 0.0)
+    return s if s > 0.0 else 1.0 / math.sqrt(D)
+
+
+# ----------------------------------------------------------------------------
+# RoPE (Periodic RoPE §3.1 Eq. 1-2; interpolation: Jet-Long §2.2)
+# ----------------------------------------------------------------------------
+def rope_frequencies(D: int, base: float, interp: float = 1.0) -> np.ndarray:
+    """theta_i = 1 / base^(2i/D) for i = 0..D/2-1, divided by the
+    interpolation factor s (angle = (p / s) * theta_i)."""
+    i = np.arange(D // 2, dtype=np.float64)
+    return (1.0 / np.power(float(base), 2.0 * i / D)) / float(interp)
+
+
+def rotation_matrix(p: float, freqs: np.ndarray) -> np.ndarray:
+    """The D x D block-diagonal R_p of Eq. 2: block i is
+    [[cos(p th_i), -sin(p th_i)], [sin(p th_i), cos(p th_i)]] on rows/cols
+    (2i, 2i+1)."""
+    D = 2 * len(freqs)
+    R = np.zeros((D, D), dtype=np.float64)
+    for i, th in enumerate(freqs):
+        c, s = math.cos(p * th), math.sin(p * th)
+        R[2 * i, 2 * i] = c
+        R[2 * i, 2 * i + 1] = -s
+        R[2 * i + 1, 2 * i] = s
+        R[2 * i + 1, 2 * i + 1] = c
+    return R
+
+
+def rotate(x: np.ndarray, pos: np.ndarray, freqs: np.ndarray) -> np.ndarray:
+    """Apply R_{pos[n]} to x[..., n, :] (the action of Eq. 2 without forming
+    the matrix). x: [..., N, D]; pos: [N] (integer-valued)."""
+    x = np.asarray(x, dtype=np.float64)
+    ang = np.asarray(pos, dtype=np.float64)[:, None] * freqs[None, :]   # [N, D/2]
+    c, s = np.cos(ang), np.sin(ang)
+    x0, x1 = x[..., 0::2], x[..., 1::2]
+    out = np.empty_like(x)
+    out[..., 0::2] = x0 * c - x1 * s
+    out[..., 1::2] = x0 * s + x1 * c
+    return out
+
+
+# ----------------------------------------------------------------------------
+# position maps
+# ----------------------------------------------------------------------------
+def periodic_position(t, W: int):
+    """Periodic RoPE §3.2 Eq. 4: phi(t) = t mod W."""
+    return np.asarray(t, dtype=np.int64) % int(W)
+
+
+def endprompt_position(t, n1: int, term_start: int):
+    """EndPrompt two-segment positions: the first segment keeps 0..n1-1, the
+    terminal segment continues from ``term_start`` (placed near the target
+    length)."""
+    t = np.asarray(t, dtype=np.int64)
+    return np.where(t < n1, t, term_start + (t - n1))
+
+
+def group_size(L: int, w_pretrained: int) -> int:
+    """Jet-Long §3.1 Eq. 2: G = max(1, ceil(L / w_pretrained))."""
+    return max(1, -(-int(L) // int(w_pretrained)))
+
+
+def remote_position(t, G: int):
+    """Jet-Long §3.1 Eq. 3: f(x) = floor(x / G)."""
+    return np.asarray(t, dtype=np.int64) // int(G)
+
+
+def position_maps(params, L: int):
+    """(pos_local, pos_remote or None, G) for token indices 0..L-1.
+
+    pos_local is the position RoPE uses for the kind (for BIFOCAL the exact
+    position of the local window); pos_remote is f(t) for BIFOCAL only. NOPE
+    returns zeros (unused). G is 1 unless the kind is BIFOCAL."""
+    t = np.arange(int(L), dtype=np.int64)
+    k = int(params.kind)
+    if k == STANDARD:
+        return t, None, 1
+    if k == ENDPROMPT:
+        return endprompt_position(t, params.seg1_len, params.term_start), None, 1
+    if k == PERIODIC:
+        return periodic_position(t, params.window), None, 1
+    if k == NOPE:
+        return np.zeros_like(t), None, 1
+    if k == BIFOCAL:
+        G = group_size(L, params.w_pretrained)
+        return t, remote_position(t, G), G
+    raise ValueError(f"unknown kind {k}")
+
+
+def _freqs(params, D):
+    interp = float(getattr(params, "interp", 1.0) or 1.0) if int(params.kind) == ENDPROMPT else 1.0
+    return rope_frequencies(D, params.rope_base, interp)
+
+
+# ----------------------------------------------------------------------------
+# prefill: the routed softmax, written as its plain definition
+# ----------------------------------------------------------------------------
+def _allowed(params, t: int, s: np.ndarray) -> np.ndarray:
+    """Keys s a query at t attends to: causal s <= t; Periodic RoPE adds the
+    window {t-W+1 .. t} (§3.2)."""
+    ok = s <= t
+    if int(params.kind) == PERIODIC:
+        ok &= s >= t - int(params.window) + 1
+    return ok
+
+
+def _softmax_rows(scores: np.ndarray, ok: np.ndarray, v: np.ndarray):
+    """out = sum softmax(scores) v over the allowed keys; lse = ln sum exp."""
+    sc = np.where(ok, scores, -np.inf)
+    m = sc.max(axis=-1, keepdims=True)
+    e = np.where(ok, np.exp(sc - m), 0.0)
+    l = e.sum(axis=-1, keepdims=True)
+    out = (e @ v) / l
+    lse = (m + np.log(l))[..., 0]
+    return out, lse
+
+
+def prefill(q, k, v, params, rows=None, stage_bf16: bool = True):
+    """Causal attention with RoPE at remapped positions (every kind).
+
+    q [B,S,Hq,D], k/v [B,S,Hkv,D] (torch or numpy). Returns (out, lse):
+    out [B,R,Hq,D], lse [B,Hq,R] for the R = len(rows) query rows (all rows
+    when ``rows`` is None). GQA: q head h reads kv head h // (Hq // Hkv).
+
+    score(t,s) = scale * <R_a q_t, R_b k_s>, with (a, b) the positions the kind
+    assigns; for BIFOCAL (a,b) = (t,s) if t-s <= w0 else (f(t), f(s)) with L = S.
+    """
+    q, k, v = to_f64(q), to_f64(k), to_f64(v)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    grp = Hq // Hkv
+    rows = np.arange(S) if rows is None else np.asarray(rows, dtype=np.int64)
+    scale = softmax_scale(D, params)
+    kind = int(params.kind)
+    freqs = _freqs(params, D)
+    p_loc, p_rem, _G = position_maps(params, S)
+    stage = round_bf16 if stage_bf16 else (lambda a: a)
+
+    out = np.zeros((B, len(rows), Hq, D))
+    lse = np.zeros((B, Hq, len(rows)))
+    keys = np.arange(S)
+    for b in range(B):
+        for hk in range(Hkv):
+            kk = k[b, :, hk, :]
+            kl = kk if kind == NOPE else stage(rotate(kk, p_loc, freqs))
+            kr = stage(rotate(kk, p_rem, freqs)) if kind == BIFOCAL else None
+            for h in range(hk * grp, (hk + 1) * grp):
+                # rows in chunks only to bound memory; each row is independent
+                for c0 in range(0, len(rows), 64):
+                    rr = rows[c0:c0 + 64]
+                    nk = int(rr.max()) + 1            # keys beyond the last row are masked
+                    ok = np.stack([_allowed(params, int(t), keys[:nk]) for t in rr])
+                    qq = q[b, rr, h, :]
+                    ql = qq if kind == NOPE else stage(rotate(qq, p_loc[rr], freqs))
+                    sc = (ql @ kl[:nk].T) * scale                         # [r, nk]
+                    if kind == BIFOCAL:
+                        qr = stage(rotate(qq, p_rem[rr], freqs))
+                        sr = (qr @ kr[:nk].T) * scale
+                        local = (rr[:, None] - keys[None, :nk]) <= int(params.w0)
+                        sc = np.where(local, sc, sr)
+                    o, l = _softmax_rows(sc, ok, v[b, :nk, hk, :])
+                    out[b, c0:c0 + 64, h, :] = o
+                    lse[b, h, c0:c0 + 64] = l
+    return out, lse
+
+
+def prefill_three_call(q, k, v, params, stage_bf16: bool = True):
+    """BIFOCAL prefill by the literal route of Jet-Long §3.3: (A) sliding
+    window w0 with exact positions, (B) full causal with remote positions,
+    (C) sliding window w0 with remote positions, each giving (O_X, l_X), then
+    Eq. 7: O = (W_A O_A + W_B O_B - W_C O_C) / (W_A + W_B - W_C), with
+    M = max(l_A, l_B, l_C) and W_X = exp(l_X - M). The merged LSE is
+    M + ln(W_A + W_B - W_C). Self-check only: ``prefill`` is the definition."""
+    q, k, v = to_f64(q), to_f64(k), to_f64(v)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    grp = Hq // Hkv
+    scale = softmax_scale(D, params)
+    freqs = _freqs(params, D)
+    G = group_size(S, params.w_pretrained)
+    t = np.arange(S)
+    f = remote_position(t, G)
+    stage = round_bf16 if stage_bf16 else (lambda a: a)
+    causal = t[:, None] >= t[None, :]
+    swa = causal & ((t[:, None] - t[None, :]) <= int(params.w0))
+    out = np.zeros((B, S, Hq, D))
+    lse = np.zeros((B, Hq, S))
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // grp
+            qb, qr = stage(rotate(q[b, :, h], t, freqs)), stage(rotate(q[b, :, h], f, freqs))
+            kb, kr = stage(rotate(k[b, :, hk], t, freqs)), stage(rotate(k[b, :, hk], f, freqs))
+            vv = v[b, :, hk]
+            OA, lA = _softmax_rows((qb @ kb.T) * scale, swa, vv)
+            OB, lB = _softmax_rows((qr @ kr.T) * scale, causal, vv)
+            OC, lC = _softmax_rows((qr @ kr.T) * scale, swa, vv)
+            M = np.maximum(np.maximum(lA, lB), lC)
+            WA, WB, WC = np.exp(lA - M), np.exp(lB - M), np.exp(lC - M)
+            den = WA + WB - WC
+            out[b, :, h] = (WA[:, None] * OA + WB[:, None] * OB - WC[:, None] * OC) / den[:, None]
+            lse[b, h] = M + np.log(den)
+    return out, lse
+
+
+# ----------------------------------------------------------------------------
+# decode (Jet-Long §3.2): untouched cache + correction rotation
+# ----------------------------------------------------------------------------
+def decode(q, k_cache, v_cache, params):
+    """One query token at position n-1 against a cache of n keys.
+
+    q [B,Hq,D] unrotated; k_cache [B,n,Hkv,D] holds keys already rotated at
+    their own positions (Eq. 4: k_cache[k] = RoPE(x_k, k)); v_cache likewise.
+    L = n. The query is rotated to its position; for BIFOCAL, keys with
+    (n-1) - k > w0 are read through the correction rotation
+    k_remote = RoPE(k_cache[k], Delta k), Delta k = f(k) - k, and the query
+    through q_remote = RoPE(q_local, Delta q) (Eq. 5-6). Rotations are kept in
+    float64 (no bf16 staging): the decode kernel keeps them in registers.
+    Returns out [B,Hq,D], lse [B,Hq]."""
+    q, kc, vc = to_f64(q), to_f64(k_cache), to_f64(v_cache)
+    B, Hq, D = q.shape
+    n, Hkv = kc.shape[1], kc.shape[2]
+    grp = Hq // Hkv
+    scale = softmax_scale(D, params)
+    kind = int(params.kind)
+    freqs = _freqs(params, D)
+    p_loc, _, G = position_maps(params, n)
+    t = n - 1
+    keys = np.arange(n)
+    ok = _allowed(params, t, keys)[None, :]
+    out = np.zeros((B, Hq, D))
+    lse = np.zeros((B, Hq))
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // grp
+            qq = q[b, h][None, :]
+            ql = qq if kind == NOPE else rotate(qq, np.array([p_loc[t]]), freqs)
+            sc = (ql @ kc[b, :, hk].T) * scale                     # [1, n]
+            if kind == BIFOCAL:
+                dq = int(remote_position(t, G)) - t                # Eq. 5
+                qr = rotate(ql, np.array([dq]), freqs)             # Eq. 6, query
+                dk = remote_position(keys, G) - keys               # Eq. 5
+                kr = rotate(kc[b, :, hk], dk, freqs)               # Eq. 6, keys
+                sr = (qr @ kr.T) * scale
+                local = (t - keys) <= int(params.w0)
+                sc = np.where(local[None, :], sc, sr)
+            o, l = _softmax_rows(sc, ok, vc[b, :, hk])
+            out[b, h] = o[0]
+            lse[b, h] = l[0]
+    return out, lse
+
+
+# ----------------------------------------------------------------------------
+# brute force: explicit matrices and loops, tiny inputs only
+# ----------------------------------------------------------------------------
+def _brute_positions(params, t: int, s: int, L: int, D: int):
+    """(a, b) positions for the pair (t, s), or None for NoPE."""
+    kind = int(params.kind)
+    if kind == NOPE:
+        return None
+    if kind == STANDARD:
+        return t, s
+    if kind == ENDPROMPT:
+        pos = lambda x: x if x < params.seg1_len else params.term_start + x - params.seg1_len
+        return pos(t), pos(s)
+    if kind == PERIODIC:
+        return t % params.window, s % params.window
+    G = max(1, math.ceil(L / params.w_pretrained))
+    if t - s <= params.w0:
+        return t, s
+    return t // G, s // G
+
+
+def brute_prefill(q, k, v, params, stage_bf16: bool = False):
+    """Every score from explicit D x D rotation matrices, every softmax by a
+    Python loop over the allowed keys. For S <= ~64."""
+    q, k, v = to_f64(q), to_f64(k), to_f64(v)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    grp = Hq // Hkv
+    scale = softmax_scale(D, params)
+    freqs = _freqs(params, D)
+    stage = round_bf16 if stage_bf16 else (lambda a: a)
+    out = np.zeros((B, S, Hq, D))
+    lse = np.zeros((B, Hq, S))
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // grp
+            for t in range(S):
+                keys = [s for s in range(S) if s <= t and
+                        (int(params.kind) != PERIODIC or s >= t - params.window + 1)]
+                scores = []
+                for s in keys:
+                    ab = _brute_positions(params, t, s, S, D)
+                    if ab is None:
+                        qa, kb = q[b, t, h], k[b, s, hk]
+                    else:
+                        qa = stage(rotation_matrix(ab[0], freqs) @ q[b, t, h])
+                        kb = stage(rotation_matrix(ab[1], freqs) @ k[b, s, hk])
+                    scores.append(scale * float(qa @ kb))
+                m = max(scores)
+                w = [math.exp(x - m) for x in scores]
+                z = sum(w)
+                out[b, t, h] = sum(wi * v[b, s, hk] for wi, s in zip(w, keys)) / z
+                lse[b, h, t] = m + math.log(z)
+    return out, lse
+
+
+def brute_decode(q, k_raw, v, params):
+    """Decode by its definition on RAW keys: the score of key s is the
+    prefill score of the last row (t = n-1) computed from unrotated k_s, so
+    this pins the cache-plus-correction route of ``decode`` (R_a R_b = R_{a+b})."""
+    q, k_raw, v = to_f64(q), to_f64(k_raw), to_f64(v)
+    B, Hq, D = q.shape
+    n, Hkv = k_raw.shape[1], k_raw.shape[2]
+    grp = Hq // Hkv
+    scale = softmax_scale(D, params)
+    freqs = _freqs(params, D)
+    t = n - 1
+    out = np.zeros((B, Hq, D))
+    lse = np.zeros((B, Hq))
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // grp
+            keys = [s for s in range(n) if int(params.kind) != PERIODIC or s >= t - params.window + 1]
+            scores = []
+            for s in keys:
+                ab = _brute_positions(params, t, s, n, D)
+                if ab is None:
+                    sc = q[b, h] @ k_raw[b, s, hk]
+                else:
+                    sc = (rotation_matrix(ab[0], freqs) @ q[b, h]) @ (rotation_matrix(ab[1], freqs) @ k_raw[b, s, hk])
+                scores.append(scale * float(sc))
+            m = max(scores)
+            w = [math.exp(x - m) for x in scores]
+            z = sum(w)
+            out[b, h] = sum(wi * v[b, s, hk] for wi, s in zip(w, keys)) / z
+            lse[b, h] = m + math.log(z)
+    return out, lse
