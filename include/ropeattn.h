@@ -1,0 +1,169 @@
+/*
+ * ropeattn — causal attention with rotary position embedding (RoPE) applied at
+ * remapped position indices, for NVIDIA B200 (sm_100a).
+ *
+ * Plain C ABI: pointers, sizes and one parameter struct. Every device pointer
+ * must point to memory of the current CUDA device. Streams are passed as
+ * `void*` holding a cudaStream_t (NULL = legacy default stream). All compute
+ * calls are asynchronous and stream-ordered; the host returns after launch.
+ *
+ * What is computed (the passages that define it):
+ *   RoPE frequencies theta_i = base^(-2i/d) and the block-diagonal rotation
+ *   R_p on coordinate pairs (2i, 2i+1): "Periodic RoPE for Infinite Context
+ *   LLMs", §3.1 Eq. 1-2. Position interpolation by a factor s uses angle
+ *   (p/s)*theta_i: "Jet-Long: Efficient Long-Context Extension with Dynamic
+ *   Bifocal RoPE", §2.2. The softmax scale is 1/sqrt(d) (Periodic RoPE §3.3
+ *   Eq. 6) unless softmax_scale > 0 is given.
+ *
+ * Layouts (row-major, contiguous, 16-byte aligned base pointers):
+ *   prefill q [B, S, Hq, D] bf16; k, v [B, S, Hkv, D] bf16 (unrotated);
+ *           out [B, S, Hq, D] fp32; lse [B, Hq, S] fp32 (natural log of the
+ *           sum of exp of the scaled scores).
+ *   decode  q [B, Hq, D] bf16 (unrotated, the token at position n-1);
+ *           k_cache [B, n, Hkv, D] bf16 already rotated at each key's own
+ *           position; v_cache [B, n, Hkv, D] bf16; out [B, Hq, D] fp32;
+ *           lse [B, Hq] fp32.
+ *   GQA: query head h reads key/value head h / (Hq / Hkv).
+ *   Supported: D in {64, 128}; Hq % Hkv == 0; decode also needs
+ *   Hq / Hkv <= 4 for D = 128 and <= 8 for D = 64.
+ *
+ * Errors: every entry point returns ROPEATTN_OK (0) or a negative code and
+ * sets a thread-local message readable with ropeattn_last_error(). Argument
+ * errors are reported before any launch and leave all buffers untouched.
+ */
+#ifndef ROPEATTN_H_
+#define ROPEATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ROPEATTN_OK                      0
+#define ROPEATTN_ERR_INVALID_ARG        -1  /* null/misaligned pointer, bad shape or parameter */
+#define ROPEATTN_ERR_UNSUPPORTED_DEVICE -2  /* current device is not sm_100 */
+#define ROPEATTN_ERR_WORKSPACE          -3  /* workspace missing or smaller than required */
+#define ROPEATTN_ERR_CUDA               -4  /* a CUDA runtime call or launch failed */
+#define ROPEATTN_ERR_TIMEOUT            -5  /* a kernel's bounded wait ran out (see ropeattn_status) */
+
+/* Position-map kinds. */
+typedef enum {
+  /* p(t) = t. Periodic RoPE §3.1. */
+  ROPEATTN_STANDARD  = 0,
+  /* EndPrompt two segments: p(t) = t for t < seg1_len, else
+   * term_start + (t - seg1_len); angles use p / interp (position
+   * interpolation). "EndPrompt: Efficient Long-Context Extension via
+   * Terminal Anchoring", abstract. */
+  ROPEATTN_ENDPROMPT = 1,
+  /* p(t) = t mod window inside causal sliding-window attention over the
+   * `window` keys {t-window+1 .. t}. Periodic RoPE §3.2 Eq. 4-5. */
+  ROPEATTN_PERIODIC  = 2,
+  /* No rotation, full causal attention. Periodic RoPE §3.3 Eq. 6. */
+  ROPEATTN_NOPE      = 3,
+  /* Jet-Long bifocal: keys with t - s <= w0 use RoPE at (t, s); the others
+   * use RoPE at (f(t), f(s)), f(x) = floor(x / G),
+   * G = max(1, ceil(L / w_pretrained)), L = the sequence length (prefill: S;
+   * decode: n). Jet-Long §3 Eq. 1, §3.1 Eq. 2-3. */
+  ROPEATTN_BIFOCAL   = 4
+} ropeattn_kind;
+
+/* Parameters of the position map. Fields a kind does not use are ignored,
+ * except the reserved ones, which must be zero. */
+typedef struct ropeattn_params {
+  int32_t kind;           /* ropeattn_kind */
+  int32_t reserved0;      /* must be 0 */
+  double  rope_base;      /* Theta > 1 (e.g. 1e4, 5e5, 1e6) */
+  double  interp;         /* ENDPROMPT: interpolation factor s >= 1 (others: ignored) */
+  int64_t seg1_len;       /* ENDPROMPT: n1 >= 0, length of the intact first segment */
+  int64_t term_start;     /* ENDPROMPT: first position of the terminal segment, >= 0 */
+  int64_t window;         /* PERIODIC: W >= 1 (window length = period) */
+  int64_t w0;             /* BIFOCAL: local window, >= 0 (0 = the token itself only) */
+  int64_t w_pretrained;   /* BIFOCAL: pretrained context window, >= 1 */
+  float   softmax_scale;  /* > 0 to override; 0 -> 1/sqrt(D) */
+  int32_t reserved[3];    /* must be 0 */
+} ropeattn_params;
+
+/* Position map of a sequence of length L (Periodic RoPE §3.2 Eq. 4; Jet-Long
+ * §3.1 Eq. 2-3; EndPrompt abstract).
+ *   d_pos_local  [L] int32, device: the position RoPE uses for each token
+ *                (BIFOCAL: the exact position t; NOPE: 0).
+ *   d_pos_remote [L] int32, device, may be NULL; required for BIFOCAL:
+ *                f(t) = floor(t / G). Written as t for other kinds when given.
+ *   h_G          host int32, may be NULL: receives G (1 unless BIFOCAL).
+ * Asynchronous on `stream` (h_G is written before return). L == 0 is a no-op.
+ * Errors: INVALID_ARG (L < 0, L >= 2^31, a position >= 2^31, null
+ * d_pos_local with L > 0, null d_pos_remote for BIFOCAL), CUDA. */
+int ropeattn_posmap(const ropeattn_params* params, int64_t L,
+                    int32_t* d_pos_local, int32_t* d_pos_remote, int32_t* h_G,
+                    void* stream);
+
+/* Bytes of device workspace ropeattn_prefill needs for these shapes:
+ * rotated keys (one copy per position map the kind uses) and the query
+ * angle tables. 0 for NOPE. */
+size_t ropeattn_prefill_workspace_size(const ropeattn_params* params, int64_t B,
+                                       int64_t S, int32_t Hq, int32_t Hkv, int32_t D);
+
+/* Causal prefill attention with RoPE at remapped positions, L = S.
+ * One pre-pass rotates the keys into `workspace` (and writes the query angle
+ * tables); the attention kernel rotates each query tile inside its TMA-staged
+ * load, runs QK^T and PV on the tensor cores (tcgen05, TMEM accumulators),
+ * keeps an online softmax per row, and for BIFOCAL merges the local and
+ * remote partials by their log-sum-exp (Jet-Long §3.3 Eq. 7) before writing.
+ * Tensor-core operands are bf16: the rotated q and k are rounded to bf16
+ * (round to nearest even); scores, softmax and outputs are fp32.
+ *   workspace: device, 256-byte aligned, >= ropeattn_prefill_workspace_size
+ *              bytes (may be NULL when that size is 0). Caller-owned; the
+ *              call overwrites it; calls sharing it must be stream-ordered.
+ * S == 0 or B == 0 is a no-op.
+ * Errors: INVALID_ARG, UNSUPPORTED_DEVICE, WORKSPACE, CUDA. */
+int ropeattn_prefill(const void* q, const void* k, const void* v,
+                     float* out, float* lse,
+                     int64_t B, int64_t S, int32_t Hq, int32_t Hkv, int32_t D,
+                     const ropeattn_params* params,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of device workspace ropeattn_decode needs (split-KV partials and
+ * per-head arrival counters). Depends on the current device's SM count. */
+size_t ropeattn_decode_workspace_size(int64_t B, int64_t n, int32_t Hq,
+                                      int32_t Hkv, int32_t D);
+
+/* One decode step: the query token at position n-1 against a cache of n keys
+ * (its own key included, stored last), L = n. Jet-Long §3.2 Eq. 4-6: the
+ * cache is never rewritten; for BIFOCAL the query is rotated to p = n-1 and
+ * corrected by Delta q = f(n-1) - (n-1), and each cached key with
+ * (n-1) - k > w0 is corrected on the fly by Delta k = f(k) - k, in fp32
+ * registers. Other kinds: the query is rotated to its position p(n-1) and
+ * the cache is read as stored (PERIODIC reads only the last `window` keys).
+ * Split-KV: each CTA streams a contiguous key range of one KV head with
+ * 128-bit loads, and the last CTA of each head merges the partials by their
+ * log-sum-exp in a fixed order (deterministic).
+ *   workspace: device, >= ropeattn_decode_workspace_size bytes. The call
+ *              clears its counters with cudaMemsetAsync on `stream` first;
+ *              calls sharing a workspace must be stream-ordered.
+ * n == 0 or B == 0 is a no-op.
+ * Errors: INVALID_ARG, UNSUPPORTED_DEVICE, WORKSPACE, CUDA. */
+int ropeattn_decode(const void* q, const void* k_cache, const void* v_cache,
+                    float* out, float* lse,
+                    int64_t B, int64_t n, int32_t Hq, int32_t Hkv, int32_t D,
+                    const ropeattn_params* params,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* Reads and clears the device status word of the current device (waits for
+ * the device to be idle first). Returns ROPEATTN_OK, or ROPEATTN_ERR_TIMEOUT
+ * if any kernel since the last call gave up on a bounded wait (its outputs
+ * are then invalid), or ROPEATTN_ERR_CUDA. */
+int ropeattn_status(void);
+
+/* Message for the last error on this host thread ("" if none). */
+const char* ropeattn_last_error(void);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int ropeattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif  /* ROPEATTN_H_ */

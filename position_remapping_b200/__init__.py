@@ -1,0 +1,19 @@
+"""ropeattn: causal attention with RoPE at remapped positions on B200 (sm_100a).
+
+The compute path is the C-ABI library ``libropeattn.so`` (include/ropeattn.h);
+``position_remapping_b200.ropeattn`` binds it. Attribute access below loads the
+library lazily so that ``position_remapping_b200.inputs`` stays importable
+without it; any compute call without the library raises ImportError.
+"""
+from .inputs import (BIFOCAL, ENDPROMPT, NOPE, PERIODIC, STANDARD, MapParams,  # noqa: F401
+                     Workload, WORKLOADS, make_qkv)
+
+_API = ("prefill", "decode", "posmap", "status", "version", "prefill_workspace_size",
+        "decode_workspace_size", "RopeAttnError")
+
+
+def __getattr__(name):
+    if name in _API:
+        from . import ropeattn
+        return getattr(ropeattn, name)
+    raise AttributeError(name)

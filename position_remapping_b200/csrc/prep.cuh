@@ -1,0 +1,59 @@
+// Key pre-rotation and query angle tables for prefill.
+//
+// Every key tile is read by all S/128 query tiles of every query head of its
+// group, so the keys are rotated once, here, in one streaming pass (per
+// position map the kind uses), instead of once per tile visit. The same pass
+// writes the (cos, sin) table of each query position that the attention
+// kernel applies to the query tile it stages in shared memory.
+//
+// Angles: theta_i = base^(-2i/D) / s (Periodic RoPE §3.1 Eq. 1; position
+// interpolation, Jet-Long §2.2), phase = p * theta_i in double precision,
+// sincos in double, rounded to fp32. The rotation of a pair (Eq. 2) is done in
+// fp32 and the result rounded to bf16 (nearest even), the tensor-core operand
+// type.
+#pragma once
+
+#include "common.cuh"
+#include "posmap.cuh"
+
+namespace ropeattn {
+
+struct PrepArgs {
+  const uint32_t* k;      // [B, S, Hkv, D] bf16, read as bf16 pairs
+  uint32_t* k_rot0;       // map 0: primary / local positions
+  uint32_t* k_rot1;       // map 1: remote positions (BIFOCAL), else null
+  float2* tab0;           // [S][D/2] (cos, sin) at map-0 positions
+  float2* tab1;           // [S][D/2] at map-1 positions, or null
+  int B, S, Hkv, D;
+  PosMap m;
+  double theta[kMaxPairs];
+};
+
+__global__ void __launch_bounds__(256) rope_prep_kernel(const PrepArgs a) {
+  const int P = a.D >> 1;
+  const int rows = blockDim.x / P;
+  const int t = blockIdx.x * rows + threadIdx.x / P;
+  const int i = threadIdx.x % P;
+  if (t >= a.S) return;
+  const int nmaps = a.k_rot1 ? 2 : 1;
+  for (int mi = 0; mi < nmaps; ++mi) {
+    const int p = mi == 0 ? pos_primary(a.m, t) : pos_remote(a.m, t);
+    double sd, cd;
+    sincos(static_cast<double>(p) * a.theta[i], &sd, &cd);
+    const float c = static_cast<float>(cd), s = static_cast<float>(sd);
+    float2* tab = mi == 0 ? a.tab0 : a.tab1;
+    tab[static_cast<size_t>(t) * P + i] = make_float2(c, s);
+    uint32_t* dst = mi == 0 ? a.k_rot0 : a.k_rot1;
+    for (int b = 0; b < a.B; ++b) {
+      for (int h = 0; h < a.Hkv; ++h) {
+        const size_t w = ((static_cast<size_t>(b) * a.S + t) * a.Hkv + h) * P + i;
+        const uint32_t x = __ldg(a.k + w);
+        float y0, y1;
+        rot_pair(bf16lo(x), bf16hi(x), c, s, y0, y1);
+        dst[w] = pack_bf16x2(y0, y1);
+      }
+    }
+  }
+}
+
+}  // namespace ropeattn

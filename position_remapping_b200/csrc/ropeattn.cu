@@ -1,0 +1,443 @@
+// Host side of the ropeattn C ABI: argument checks, workspace layout, TMA
+// tensor maps and kernel launches. All kernels live in this translation unit.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/ropeattn.h"
+#include "common.cuh"
+#include "decode_sm100.cuh"
+#include "posmap.cuh"
+#include "prefill_sm100.cuh"
+#include "prep.cuh"
+
+using namespace ropeattn;
+
+namespace {
+
+constexpr int kVersion = 10000;  // 1.0.0
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(ROPEATTN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define CUDA_TRY(call, what)                 \
+  do {                                       \
+    cudaError_t _e = (call);                 \
+    if (_e != cudaSuccess) return cuda_fail(_e, what); \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// sm_100 check, cached per device
+int check_device() {
+  static std::mutex mu;
+  static int cached[64];  // 0 unknown, 1 ok, -1 bad
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(ROPEATTN_ERR_UNSUPPORTED_DEVICE, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(mu);
+  if (cached[dev] == 0) {
+    int major = 0, minor = 0;
+    CUDA_TRY(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev), "cudaDeviceGetAttribute");
+    CUDA_TRY(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev), "cudaDeviceGetAttribute");
+    cached[dev] = (major == 10 && minor == 0) ? 1 : -1;
+    if (cached[dev] < 0)
+      return fail(ROPEATTN_ERR_UNSUPPORTED_DEVICE, "device %d is sm_%d%d; this library is built for sm_100a", dev,
+                  major, minor);
+  }
+  if (cached[dev] < 0) return fail(ROPEATTN_ERR_UNSUPPORTED_DEVICE, "device %d is not sm_100", dev);
+  return ROPEATTN_OK;
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 4-D bf16 tensor [d3][d2][d1][d0] (d0 contiguous) with box (b0, 1, b2, 1).
+int make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3,
+             uint32_t b0, uint32_t b2, bool swizzle128) {
+  auto fn = encode_fn();
+  if (!fn) return fail(ROPEATTN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[4] = {d0, d1, d2, d3};
+  cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
+  cuuint32_t box[4] = {b0, 1, b2, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(ROPEATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return ROPEATTN_OK;
+}
+
+constexpr long long kMaxPos = 0x7fffffffLL;
+
+// Validates the parameter struct for a sequence of length L; fills the
+// position map. The kind may be simplified: a bifocal map with G = 1 or with
+// every key inside the local window is exactly the standard map (Jet-Long §3:
+// "reduces to the unmodified base model").
+int check_params(const ropeattn_params* p, long long L, int D, PosMap* m, int* eff_kind) {
+  if (!p) return fail(ROPEATTN_ERR_INVALID_ARG, "params is NULL");
+  if (p->reserved0 != 0 || p->reserved[0] != 0 || p->reserved[1] != 0 || p->reserved[2] != 0)
+    return fail(ROPEATTN_ERR_INVALID_ARG, "reserved fields must be 0");
+  if (p->kind < ROPEATTN_STANDARD || p->kind > ROPEATTN_BIFOCAL)
+    return fail(ROPEATTN_ERR_INVALID_ARG, "unknown kind %d", p->kind);
+  if (p->kind != ROPEATTN_NOPE && !(p->rope_base > 1.0 && std::isfinite(p->rope_base)))
+    return fail(ROPEATTN_ERR_INVALID_ARG, "rope_base must be a finite number > 1");
+  if (!(p->softmax_scale >= 0.0f) || !std::isfinite(p->softmax_scale))
+    return fail(ROPEATTN_ERR_INVALID_ARG, "softmax_scale must be >= 0 and finite");
+  if (L < 0 || L > kMaxPos) return fail(ROPEATTN_ERR_INVALID_ARG, "sequence length %lld out of range", L);
+  *m = PosMap{p->kind, 0, 0, 1, 0, 1};
+  *eff_kind = p->kind;
+  switch (p->kind) {
+    case ROPEATTN_ENDPROMPT:
+      if (!(p->interp >= 1.0 && std::isfinite(p->interp)))
+        return fail(ROPEATTN_ERR_INVALID_ARG, "interp must be >= 1");
+      if (p->seg1_len < 0 || p->term_start < 0 || p->seg1_len > kMaxPos || p->term_start > kMaxPos)
+        return fail(ROPEATTN_ERR_INVALID_ARG, "seg1_len and term_start must be in [0, 2^31)");
+      if (L > p->seg1_len && p->term_start + (L - 1 - p->seg1_len) > kMaxPos)
+        return fail(ROPEATTN_ERR_INVALID_ARG, "terminal positions exceed 2^31-1");
+      m->seg1_len = static_cast<int>(p->seg1_len);
+      m->term_start = static_cast<int>(p->term_start);
+      break;
+    case ROPEATTN_PERIODIC:
+      if (p->window < 1 || p->window > (1LL << 30)) return fail(ROPEATTN_ERR_INVALID_ARG, "window must be in [1, 2^30]");
+      m->window = static_cast<int>(p->window);
+      break;
+    case ROPEATTN_BIFOCAL: {
+      if (p->w0 < 0) return fail(ROPEATTN_ERR_INVALID_ARG, "w0 must be >= 0");
+      if (p->w_pretrained < 1) return fail(ROPEATTN_ERR_INVALID_ARG, "w_pretrained must be >= 1");
+      m->G = group_size(L, p->w_pretrained);
+      m->w0 = static_cast<int>(p->w0 < (1LL << 30) ? p->w0 : (1LL << 30));
+      if (m->G == 1 || p->w0 >= L - 1) *eff_kind = ROPEATTN_STANDARD;
+      break;
+    }
+    default:
+      break;
+  }
+  (void)D;
+  return ROPEATTN_OK;
+}
+
+void fill_theta(const ropeattn_params* p, int D, double* theta) {
+  const double s = p->kind == ROPEATTN_ENDPROMPT ? p->interp : 1.0;
+  for (int i = 0; i < D / 2; ++i) theta[i] = std::pow(p->rope_base, -2.0 * i / D) / s;
+}
+
+float scale_log2(const ropeattn_params* p, int D) {
+  const double sc = p->softmax_scale > 0.0f ? static_cast<double>(p->softmax_scale) : 1.0 / std::sqrt(double(D));
+  return static_cast<float>(sc * 1.4426950408889634074);
+}
+
+int check_shapes(long long B, long long S, int Hq, int Hkv, int D) {
+  if (B < 0 || S < 0) return fail(ROPEATTN_ERR_INVALID_ARG, "B and S must be >= 0");
+  if (D != 64 && D != 128) return fail(ROPEATTN_ERR_INVALID_ARG, "D must be 64 or 128 (got %d)", D);
+  if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0)
+    return fail(ROPEATTN_ERR_INVALID_ARG, "need Hq >= 1, Hkv >= 1 and Hq %% Hkv == 0 (Hq=%d Hkv=%d)", Hq, Hkv);
+  if (S > kMaxPos || B > 65535 || Hq > 65535) return fail(ROPEATTN_ERR_INVALID_ARG, "shape too large");
+  return ROPEATTN_OK;
+}
+
+struct PrefillLayout {
+  int nmaps;
+  size_t krot_bytes, tab_bytes, total;
+  size_t off_krot[2], off_tab[2];
+};
+
+PrefillLayout prefill_layout(int eff_kind, long long B, long long S, int Hkv, int D) {
+  PrefillLayout L{};
+  L.nmaps = eff_kind == ROPEATTN_NOPE ? 0 : (eff_kind == ROPEATTN_BIFOCAL ? 2 : 1);
+  L.krot_bytes = align_up(static_cast<size_t>(B) * S * Hkv * D * 2, 256);
+  L.tab_bytes = align_up(static_cast<size_t>(S) * (D / 2) * sizeof(float2), 256);
+  size_t off = 0;
+  for (int i = 0; i < L.nmaps; ++i) { L.off_krot[i] = off; off += L.krot_bytes; }
+  for (int i = 0; i < L.nmaps; ++i) { L.off_tab[i] = off; off += L.tab_bytes; }
+  L.total = off;
+  return L;
+}
+
+template <int D, int NST>
+int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk0, const CUtensorMap& tk1, const CUtensorMap& tv,
+                   const PrefillParams& pp, int grid, cudaStream_t st) {
+  using L = PrefillSmem<D, NST>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(prefill_kernel<D, NST>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  });
+  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(prefill)");
+  prefill_kernel<D, NST><<<grid, kPrefillThreads, L::kAlloc, st>>>(tq, tk0, tk1, tv, pp);
+  CUDA_TRY(cudaGetLastError(), "prefill launch");
+  return ROPEATTN_OK;
+}
+
+struct DecodeLayout {
+  int nsplit;
+  size_t off_o, off_ml, off_cnt, total;
+};
+
+int decode_nsplit(long long B, long long keys, int Hkv) {
+  long long want = (2LL * sm_count() + Hkv * B - 1) / (Hkv * B);
+  long long cap = (keys + 255) / 256;
+  long long ns = want < cap ? want : cap;
+  return static_cast<int>(ns < 1 ? 1 : ns);
+}
+
+DecodeLayout decode_layout(long long B, long long keys, int Hq, int Hkv, int D) {
+  DecodeLayout L{};
+  L.nsplit = decode_nsplit(B, keys, Hkv);
+  size_t slots = static_cast<size_t>(B) * Hq * L.nsplit;
+  L.off_o = 0;
+  L.off_ml = align_up(slots * D * sizeof(float), 256);
+  L.off_cnt = L.off_ml + align_up(slots * sizeof(float2), 256);
+  L.total = L.off_cnt + align_up(static_cast<size_t>(B) * Hkv * sizeof(int), 256);
+  return L;
+}
+
+template <int D, int GRP>
+int launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& dp, dim3 grid, cudaStream_t st) {
+  using L = DecodeSmem<D>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(decode_kernel<D, GRP>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal);
+  });
+  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(decode)");
+  decode_kernel<D, GRP><<<grid, kDecThreads, L::kTotal, st>>>(tk, tv, dp);
+  CUDA_TRY(cudaGetLastError(), "decode launch");
+  return ROPEATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ropeattn_last_error(void) { return g_last_error.c_str(); }
+
+int ropeattn_version(void) { return kVersion; }
+
+int ropeattn_status(void) {
+  g_last_error.clear();
+  CUDA_TRY(cudaDeviceSynchronize(), "cudaDeviceSynchronize");
+  int v = 0, zero = 0;
+  CUDA_TRY(cudaMemcpyFromSymbol(&v, ropeattn::g_status, sizeof(int)), "read status");
+  CUDA_TRY(cudaMemcpyToSymbol(ropeattn::g_status, &zero, sizeof(int)), "clear status");
+  if (v & kStatusTimeout) return fail(ROPEATTN_ERR_TIMEOUT, "a kernel gave up on a bounded wait");
+  return ROPEATTN_OK;
+}
+
+int ropeattn_posmap(const ropeattn_params* params, int64_t L, int32_t* d_pos_local, int32_t* d_pos_remote,
+                    int32_t* h_G, void* stream) {
+  g_last_error.clear();
+  PosMap m;
+  int eff;
+  int rc = check_params(params, L, 64, &m, &eff);
+  if (rc) return rc;
+  if (L > 0 && !d_pos_local) return fail(ROPEATTN_ERR_INVALID_ARG, "d_pos_local is NULL");
+  if (L > 0 && params->kind == ROPEATTN_BIFOCAL && !d_pos_remote)
+    return fail(ROPEATTN_ERR_INVALID_ARG, "d_pos_remote is required for BIFOCAL");
+  if (h_G) *h_G = m.G;
+  if (L == 0) return ROPEATTN_OK;
+  const int threads = 256;
+  const long long blocks = (L + threads - 1) / threads;
+  posmap_kernel<<<static_cast<unsigned>(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      m, static_cast<int>(L), d_pos_local, d_pos_remote);
+  CUDA_TRY(cudaGetLastError(), "posmap launch");
+  return ROPEATTN_OK;
+}
+
+size_t ropeattn_prefill_workspace_size(const ropeattn_params* params, int64_t B, int64_t S, int32_t Hq,
+                                       int32_t Hkv, int32_t D) {
+  PosMap m;
+  int eff;
+  if (check_params(params, S, D, &m, &eff) || check_shapes(B, S, Hq, Hkv, D)) return 0;
+  return prefill_layout(eff, B, S, Hkv, D).total;
+}
+
+int ropeattn_prefill(const void* q, const void* k, const void* v, float* out, float* lse, int64_t B, int64_t S,
+                     int32_t Hq, int32_t Hkv, int32_t D, const ropeattn_params* params, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  g_last_error.clear();
+  int rc = check_shapes(B, S, Hq, Hkv, D);
+  if (rc) return rc;
+  PosMap m;
+  int eff;
+  rc = check_params(params, S, D, &m, &eff);
+  if (rc) return rc;
+  if (B == 0 || S == 0) return ROPEATTN_OK;
+  if (!q || !k || !v || !out || !lse) return fail(ROPEATTN_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return fail(ROPEATTN_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if ((static_cast<long long>((S + kBM - 1) / kBM)) * Hq * B > 0x7fffffffLL)
+    return fail(ROPEATTN_ERR_INVALID_ARG, "too many query tiles");
+  rc = check_device();
+  if (rc) return rc;
+  const PrefillLayout lay = prefill_layout(eff, B, S, Hkv, D);
+  if (lay.total > 0) {
+    if (!workspace || workspace_bytes < lay.total)
+      return fail(ROPEATTN_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", lay.total,
+                  workspace ? workspace_bytes : size_t(0));
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+      return fail(ROPEATTN_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  m.kind = eff;
+
+  // 1) keys rotated once per map, and the query angle tables
+  const void* kmap0 = k;
+  const void* kmap1 = k;
+  PrefillParams pp{};
+  if (lay.nmaps > 0) {
+    PrepArgs a{};
+    a.k = static_cast<const uint32_t*>(k);
+    a.k_rot0 = reinterpret_cast<uint32_t*>(ws + lay.off_krot[0]);
+    a.k_rot1 = lay.nmaps > 1 ? reinterpret_cast<uint32_t*>(ws + lay.off_krot[1]) : nullptr;
+    a.tab0 = reinterpret_cast<float2*>(ws + lay.off_tab[0]);
+    a.tab1 = lay.nmaps > 1 ? reinterpret_cast<float2*>(ws + lay.off_tab[1]) : nullptr;
+    a.B = static_cast<int>(B);
+    a.S = static_cast<int>(S);
+    a.Hkv = Hkv;
+    a.D = D;
+    a.m = m;
+    fill_theta(params, D, a.theta);
+    const int rows = 256 / (D / 2);
+    rope_prep_kernel<<<static_cast<unsigned>((S + rows - 1) / rows), 256, 0, st>>>(a);
+    CUDA_TRY(cudaGetLastError(), "rope_prep launch");
+    kmap0 = a.k_rot0;
+    kmap1 = lay.nmaps > 1 ? static_cast<const void*>(a.k_rot1) : kmap0;
+    pp.tab0 = a.tab0;
+    pp.tab1 = a.tab1;
+  }
+
+  // 2) attention
+  CUtensorMap tq, tk0, tk1, tv;
+  if ((rc = make_map(&tq, q, D, Hq, S, B, 64, kBM, true))) return rc;
+  if ((rc = make_map(&tk0, kmap0, D, Hkv, S, B, 64, kBN, true))) return rc;
+  if ((rc = make_map(&tk1, kmap1, D, Hkv, S, B, 64, kBN, true))) return rc;
+  if ((rc = make_map(&tv, v, D, Hkv, S, B, 64, kBN, true))) return rc;
+  pp.out = out;
+  pp.lse = lse;
+  pp.B = static_cast<int>(B);
+  pp.S = static_cast<int>(S);
+  pp.Hq = Hq;
+  pp.Hkv = Hkv;
+  pp.nqt = static_cast<int>((S + kBM - 1) / kBM);
+  pp.kind = eff;
+  pp.window = m.window;
+  pp.w0 = m.w0;
+  pp.scale_log2 = scale_log2(params, D);
+  const int grid = pp.nqt * Hq * static_cast<int>(B);
+  if (D == 128) return launch_prefill<128, 2>(tq, tk0, tk1, tv, pp, grid, st);
+  return launch_prefill<64, 4>(tq, tk0, tk1, tv, pp, grid, st);
+}
+
+size_t ropeattn_decode_workspace_size(int64_t B, int64_t n, int32_t Hq, int32_t Hkv, int32_t D) {
+  if (check_shapes(B, n, Hq, Hkv, D) || B == 0 || n == 0) return 0;
+  return decode_layout(B, n, Hq, Hkv, D).total;
+}
+
+int ropeattn_decode(const void* q, const void* k_cache, const void* v_cache, float* out, float* lse, int64_t B,
+                    int64_t n, int32_t Hq, int32_t Hkv, int32_t D, const ropeattn_params* params, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  g_last_error.clear();
+  int rc = check_shapes(B, n, Hq, Hkv, D);
+  if (rc) return rc;
+  PosMap m;
+  int eff;
+  rc = check_params(params, n, D, &m, &eff);
+  if (rc) return rc;
+  if (B == 0 || n == 0) return ROPEATTN_OK;
+  const int grp = Hq / Hkv;
+  if (!((D == 128 && (grp == 1 || grp == 2 || grp == 4)) || (D == 64 && (grp == 1 || grp == 2 || grp == 4 || grp == 8))))
+    return fail(ROPEATTN_ERR_INVALID_ARG, "decode supports Hq/Hkv in {1,2,4} for D=128 and {1,2,4,8} for D=64");
+  if (!q || !k_cache || !v_cache || !out || !lse) return fail(ROPEATTN_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || !aligned16(lse))
+    return fail(ROPEATTN_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  rc = check_device();
+  if (rc) return rc;
+  const long long t = n - 1;
+  const long long k_begin = eff == ROPEATTN_PERIODIC ? (n > m.window ? n - m.window : 0) : 0;
+  const long long keys = n - k_begin;
+  const DecodeLayout lay = decode_layout(B, keys, Hq, Hkv, D);
+  const size_t need = ropeattn_decode_workspace_size(B, n, Hq, Hkv, D);
+  if (!workspace || workspace_bytes < need)
+    return fail(ROPEATTN_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need,
+                workspace ? workspace_bytes : size_t(0));
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+    return fail(ROPEATTN_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+
+  DecodeParams dp{};
+  dp.q = static_cast<const __nv_bfloat16*>(q);
+  dp.out = out;
+  dp.lse = lse;
+  dp.part_o = reinterpret_cast<float*>(ws + lay.off_o);
+  dp.part_ml = reinterpret_cast<float2*>(ws + lay.off_ml);
+  dp.counters = reinterpret_cast<int*>(ws + lay.off_cnt);
+  dp.B = static_cast<int>(B);
+  dp.n = static_cast<int>(n);
+  dp.Hq = Hq;
+  dp.Hkv = Hkv;
+  dp.nsplit = lay.nsplit;
+  dp.keys_per_split = static_cast<int>(align_up(static_cast<size_t>((keys + lay.nsplit - 1) / lay.nsplit), kDecKeys));
+  dp.k_begin = static_cast<int>(k_begin);
+  dp.bifocal = eff == ROPEATTN_BIFOCAL ? 1 : 0;
+  dp.k_local = dp.bifocal ? static_cast<int>(t - m.w0 > 0 ? t - m.w0 : 0) : 0;
+  m.kind = eff;
+  dp.m = m;
+  dp.scale_log2 = scale_log2(params, D);
+  fill_theta(params, D, dp.theta);
+
+  CUtensorMap tk, tv;
+  if ((rc = make_map(&tk, k_cache, D, Hkv, n, B, D, kDecKeys, false))) return rc;
+  if ((rc = make_map(&tv, v_cache, D, Hkv, n, B, D, kDecKeys, false))) return rc;
+  CUDA_TRY(cudaMemsetAsync(dp.counters, 0, static_cast<size_t>(B) * Hkv * sizeof(int), st), "memset counters");
+  dim3 grid(lay.nsplit, Hkv, static_cast<unsigned>(B));
+  if (D == 128) {
+    if (grp == 1) return launch_decode<128, 1>(tk, tv, dp, grid, st);
+    if (grp == 2) return launch_decode<128, 2>(tk, tv, dp, grid, st);
+    return launch_decode<128, 4>(tk, tv, dp, grid, st);
+  }
+  if (grp == 1) return launch_decode<64, 1>(tk, tv, dp, grid, st);
+  if (grp == 2) return launch_decode<64, 2>(tk, tv, dp, grid, st);
+  if (grp == 4) return launch_decode<64, 4>(tk, tv, dp, grid, st);
+  return launch_decode<64, 8>(tk, tv, dp, grid, st);
+}
+
+}  // extern "C"

@@ -1,0 +1,177 @@
+"""Thin Python binding of the ropeattn C ABI (include/ropeattn.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library. PyTorch provides device memory and the current stream. Importing this
+module loads libropeattn.so and raises if it is missing; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+from .inputs import MapParams
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libropeattn.so")
+
+OK = 0
+ERR_INVALID_ARG, ERR_UNSUPPORTED_DEVICE, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = -1, -2, -3, -4, -5
+
+# every symbol include/ropeattn.h declares
+EXPORTS = ("ropeattn_posmap", "ropeattn_prefill_workspace_size", "ropeattn_prefill",
+           "ropeattn_decode_workspace_size", "ropeattn_decode", "ropeattn_status",
+           "ropeattn_last_error", "ropeattn_version")
+
+
+class RopeAttnError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"ropeattn error {code}: {msg}")
+        self.code = code
+
+
+class CParams(ctypes.Structure):
+    """Mirror of ``ropeattn_params``."""
+    _fields_ = [
+        ("kind", ctypes.c_int32),
+        ("reserved0", ctypes.c_int32),
+        ("rope_base", ctypes.c_double),
+        ("interp", ctypes.c_double),
+        ("seg1_len", ctypes.c_int64),
+        ("term_start", ctypes.c_int64),
+        ("window", ctypes.c_int64),
+        ("w0", ctypes.c_int64),
+        ("w_pretrained", ctypes.c_int64),
+        ("softmax_scale", ctypes.c_float),
+        ("reserved", ctypes.c_int32 * 3),
+    ]
+
+
+def to_cparams(p: MapParams) -> CParams:
+    c = CParams()
+    c.kind = int(p.kind)
+    c.rope_base = float(p.rope_base)
+    c.interp = float(p.interp)
+    c.seg1_len = int(p.seg1_len)
+    c.term_start = int(p.term_start)
+    c.window = int(p.window)
+    c.w0 = int(p.w0)
+    c.w_pretrained = int(p.w_pretrained)
+    c.softmax_scale = float(p.softmax_scale)
+    return c
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m position_remapping_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+    P = ctypes.POINTER(CParams)
+    lib.ropeattn_posmap.argtypes = [P, i64, vp, vp, ctypes.POINTER(i32), vp]
+    lib.ropeattn_prefill_workspace_size.argtypes = [P, i64, i64, i32, i32, i32]
+    lib.ropeattn_prefill_workspace_size.restype = sz
+    lib.ropeattn_prefill.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, P, vp, sz, vp]
+    lib.ropeattn_decode_workspace_size.argtypes = [i64, i64, i32, i32, i32]
+    lib.ropeattn_decode_workspace_size.restype = sz
+    lib.ropeattn_decode.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, P, vp, sz, vp]
+    lib.ropeattn_status.argtypes = []
+    lib.ropeattn_last_error.argtypes = []
+    lib.ropeattn_last_error.restype = ctypes.c_char_p
+    lib.ropeattn_version.argtypes = []
+    for name in ("ropeattn_posmap", "ropeattn_prefill", "ropeattn_decode", "ropeattn_status", "ropeattn_version"):
+        getattr(lib, name).restype = ctypes.c_int
+    return lib
+
+
+lib = _load()
+
+
+def _check(rc: int):
+    if rc != OK:
+        raise RopeAttnError(rc, lib.ropeattn_last_error().decode())
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def version() -> int:
+    return lib.ropeattn_version()
+
+
+def status() -> None:
+    """Raises RopeAttnError(ERR_TIMEOUT) if a kernel gave up on a bounded wait."""
+    _check(lib.ropeattn_status())
+
+
+def posmap(params: MapParams, L: int, device="cuda", stream=None) -> Tuple[torch.Tensor, torch.Tensor, int]:
+    cp = to_cparams(params)
+    loc = torch.empty(max(L, 1), dtype=torch.int32, device=device)
+    rem = torch.empty(max(L, 1), dtype=torch.int32, device=device)
+    G = ctypes.c_int32(0)
+    _check(lib.ropeattn_posmap(ctypes.byref(cp), int(L), _ptr(loc), _ptr(rem), ctypes.byref(G), _stream(stream)))
+    return loc[:L], rem[:L], int(G.value)
+
+
+def prefill_workspace_size(params: MapParams, B, S, Hq, Hkv, D) -> int:
+    cp = to_cparams(params)
+    return int(lib.ropeattn_prefill_workspace_size(ctypes.byref(cp), B, S, Hq, Hkv, D))
+
+
+def decode_workspace_size(B, n, Hq, Hkv, D) -> int:
+    return int(lib.ropeattn_decode_workspace_size(B, n, Hq, Hkv, D))
+
+
+def _workspace(nbytes: int, device) -> Optional[torch.Tensor]:
+    if nbytes == 0:
+        return None
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, params: MapParams,
+            out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+            workspace: Optional[torch.Tensor] = None, stream=None):
+    """q [B,S,Hq,D], k/v [B,S,Hkv,D] bf16 contiguous on one CUDA device.
+    Returns (out [B,S,Hq,D] fp32, lse [B,Hq,S] fp32)."""
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if out is None:
+        out = torch.empty((B, S, Hq, D), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
+    need = prefill_workspace_size(params, B, S, Hq, Hkv, D)
+    if workspace is None:
+        workspace = _workspace(need, q.device)
+    cp = to_cparams(params)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.ropeattn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, S, Hq, Hkv, D,
+                                ctypes.byref(cp), _ptr(workspace), ws_bytes, _stream(stream)))
+    return out, lse
+
+
+def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, params: MapParams,
+           out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+           workspace: Optional[torch.Tensor] = None, stream=None):
+    """q [B,Hq,D] (unrotated, position n-1), caches [B,n,Hkv,D] bf16.
+    Returns (out [B,Hq,D] fp32, lse [B,Hq] fp32)."""
+    B, Hq, D = q.shape
+    n, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = _workspace(decode_workspace_size(B, n, Hq, Hkv, D), q.device)
+    cp = to_cparams(params)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.ropeattn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse), B, n, Hq, Hkv, D,
+                               ctypes.byref(cp), _ptr(workspace), ws_bytes, _stream(stream)))
+    return out, lse

@@ -1,0 +1,131 @@
+"""The C-ABI library: it loads without a GPU, exports every symbol the header
+declares, its parameter struct matches the C layout, and host-side argument
+checks reject bad calls before any launch. CPU only."""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ropeattn.h")
+
+
+@pytest.fixture(scope="module")
+def ra():
+    from position_remapping_b200 import build
+    build.build()
+    from position_remapping_b200 import ropeattn
+    return ropeattn
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ropeattn_[a-z_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(ra):
+    names = declared_functions()
+    assert len(names) >= 8
+    lib = ctypes.CDLL(ra.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(ra.EXPORTS)
+    out = subprocess.run(["nm", "-D", "--defined-only", ra.LIB_PATH], capture_output=True, text=True).stdout
+    for n in names:
+        assert re.search(rf"\bT {n}\b", out), n
+
+
+def test_library_has_no_libcuda_dependency(ra):
+    out = subprocess.run(["ldd", ra.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out
+
+
+def test_param_struct_layout_matches_c(ra):
+    prog = r'''
+#include <stdio.h>
+#include <stddef.h>
+#include "ropeattn.h"
+int main(void) {
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(ropeattn_params),
+    offsetof(ropeattn_params, kind), offsetof(ropeattn_params, rope_base), offsetof(ropeattn_params, interp),
+    offsetof(ropeattn_params, seg1_len), offsetof(ropeattn_params, term_start), offsetof(ropeattn_params, window),
+    offsetof(ropeattn_params, w0), offsetof(ropeattn_params, w_pretrained), offsetof(ropeattn_params, softmax_scale),
+    offsetof(ropeattn_params, reserved));
+  return 0;
+}
+'''
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "t.c")
+        exe = os.path.join(d, "t")
+        open(c, "w").write(prog)
+        subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), c, "-o", exe], check=True)
+        got = list(map(int, subprocess.run([exe], capture_output=True, text=True).stdout.split()))
+    P = ra.CParams
+    want = [ctypes.sizeof(P)] + [getattr(P, f).offset for f in
+            ("kind", "rope_base", "interp", "seg1_len", "term_start", "window", "w0", "w_pretrained",
+             "softmax_scale", "reserved")]
+    assert got == want
+
+
+def _p(**kw):
+    from position_remapping_b200.inputs import MapParams
+    return MapParams(**kw)
+
+
+def test_host_argument_checks(ra):
+    from position_remapping_b200.inputs import BIFOCAL, ENDPROMPT, NOPE, PERIODIC, STANDARD
+    lib = ra.lib
+    cp = ra.to_cparams
+    nullp = ctypes.c_void_p(0)
+    # bad head_dim, head ratio: rejected before any device work
+    for D, Hq, Hkv in ((96, 4, 2), (128, 6, 4), (64, 0, 1)):
+        rc = lib.ropeattn_prefill(nullp, nullp, nullp, nullp, nullp, 1, 16, Hq, Hkv, D,
+                                  ctypes.byref(cp(_p(kind=STANDARD))), nullp, 0, nullp)
+        assert rc == ra.ERR_INVALID_ARG
+        assert lib.ropeattn_last_error().decode()
+    bad = [_p(kind=9), _p(kind=PERIODIC, window=0), _p(kind=BIFOCAL, w0=-1, w_pretrained=8),
+           _p(kind=BIFOCAL, w0=4, w_pretrained=0), _p(kind=ENDPROMPT, interp=0.5),
+           _p(kind=STANDARD, rope_base=1.0), _p(kind=STANDARD, softmax_scale=-1.0)]
+    for p in bad:
+        rc = lib.ropeattn_prefill(nullp, nullp, nullp, nullp, nullp, 1, 16, 2, 1, 64,
+                                  ctypes.byref(cp(p)), nullp, 0, nullp)
+        assert rc == ra.ERR_INVALID_ARG, p
+    c = cp(_p(kind=STANDARD))
+    c.reserved[1] = 3
+    assert lib.ropeattn_prefill(nullp, nullp, nullp, nullp, nullp, 1, 16, 2, 1, 64, ctypes.byref(c),
+                                nullp, 0, nullp) == ra.ERR_INVALID_ARG
+    # null tensors with work to do
+    assert lib.ropeattn_prefill(nullp, nullp, nullp, nullp, nullp, 1, 16, 2, 1, 64,
+                                ctypes.byref(cp(_p(kind=NOPE))), nullp, 0, nullp) == ra.ERR_INVALID_ARG
+    # empty problems are no-ops
+    assert lib.ropeattn_prefill(nullp, nullp, nullp, nullp, nullp, 0, 16, 2, 1, 64,
+                                ctypes.byref(cp(_p(kind=NOPE))), nullp, 0, nullp) == ra.OK
+    assert lib.ropeattn_decode(nullp, nullp, nullp, nullp, nullp, 1, 0, 2, 1, 64,
+                               ctypes.byref(cp(_p(kind=NOPE))), nullp, 0, nullp) == ra.OK
+    # decode group-size limit
+    assert lib.ropeattn_decode(nullp, nullp, nullp, nullp, nullp, 1, 64, 16, 2, 128,
+                               ctypes.byref(cp(_p(kind=NOPE))), nullp, 0, nullp) == ra.ERR_INVALID_ARG
+    # posmap: BIFOCAL needs the remote output
+    G = ctypes.c_int32(0)
+    assert lib.ropeattn_posmap(ctypes.byref(cp(_p(kind=BIFOCAL, w0=2, w_pretrained=8))), 10, nullp, nullp,
+                               ctypes.byref(G), nullp) == ra.ERR_INVALID_ARG
+    assert lib.ropeattn_posmap(ctypes.byref(cp(_p(kind=BIFOCAL, w0=2, w_pretrained=8))), 0, nullp, nullp,
+                               ctypes.byref(G), nullp) == ra.OK and G.value == 1
+
+
+def test_workspace_sizes(ra):
+    from position_remapping_b200.inputs import WORKLOADS
+    w = WORKLOADS["bifocal_prefill_s131072"]
+    n = ra.prefill_workspace_size(w.params, w.B, w.S, w.Hq, w.Hkv, w.D)
+    # two rotated key copies + two query angle tables
+    assert n == 2 * (w.B * w.S * w.Hkv * w.D * 2) + 2 * (w.S * w.D // 2 * 8)
+    nope = WORKLOADS["nope_s32768"]
+    assert ra.prefill_workspace_size(nope.params, nope.B, nope.S, nope.Hq, nope.Hkv, nope.D) == 0
+    # a bifocal map that fits the pretrained window is the standard map: one copy
+    short = w.params.replace(w_pretrained=1 << 20)
+    assert ra.prefill_workspace_size(short, 1, 4096, 32, 8, 128) == 4096 * 8 * 128 * 2 + 4096 * 64 * 8
+    assert ra.decode_workspace_size(1, 131072, 16, 8, 128) > 0

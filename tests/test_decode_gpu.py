@@ -1,0 +1,71 @@
+"""Decode parity: the split-KV CUDA kernel (through the C ABI) against the
+float64 oracle on the same seeded bf16 query and cache."""
+import zlib
+
+import pytest
+import torch
+
+import oracle as O
+from parity_util import assert_close
+from position_remapping_b200.inputs import WORKLOADS, MapParams, make_qkv
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    ("standard", 2, 1000, 4, 2, 128, MapParams(O.STANDARD, rope_base=1e4)),
+    ("standard_n1", 1, 1, 2, 1, 128, MapParams(O.STANDARD, rope_base=1e4)),
+    ("endprompt", 1, 777, 4, 1, 128, MapParams(O.ENDPROMPT, rope_base=5e5, interp=8.0, seg1_len=600, term_start=65000)),
+    ("periodic", 2, 3000, 2, 2, 64, MapParams(O.PERIODIC, window=1024)),
+    ("periodic_w_gt_n", 1, 300, 2, 1, 64, MapParams(O.PERIODIC, window=1000)),
+    ("nope_g8", 1, 2049, 8, 1, 64, MapParams(O.NOPE)),
+    ("bifocal_g2", 1, 5000, 16, 8, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=300, w_pretrained=2500)),
+    ("bifocal_g10", 2, 1001, 4, 2, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=50, w_pretrained=100)),
+    ("bifocal_g3_grp4", 1, 9000, 8, 2, 128, MapParams(O.BIFOCAL, rope_base=1e4, w0=1000, w_pretrained=3001)),
+    ("bifocal_w0_0_d64", 1, 4097, 4, 1, 64, MapParams(O.BIFOCAL, rope_base=1e4, w0=0, w_pretrained=1024)),
+    ("bifocal_inside_window", 1, 500, 4, 2, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=100, w_pretrained=512)),
+]
+
+
+def _run(q, kc, vc, params):
+    from position_remapping_b200 import ropeattn as ra
+    out, lse = ra.decode(q.cuda(), kc.cuda(), vc.cuda(), params)
+    torch.cuda.synchronize()
+    ra.status()
+    return out, lse
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+def test_decode_small(case):
+    name, B, n, Hq, Hkv, D, params = case
+    q, kc, vc = make_qkv(B, n, Hq, Hkv, D, seed=zlib.crc32(name.encode()) % 10000, q_len=1)
+    out, lse = _run(q, kc, vc, params)
+    ref_o, ref_l = O.decode(q, kc, vc, params)
+    assert_close(out.cpu().numpy(), lse.cpu().numpy(), ref_o, ref_l, name)
+
+
+def test_decode_full_size():
+    w = WORKLOADS["bifocal_decode_n131072"]
+    q, kc, vc = make_qkv(w.B, w.S, w.Hq, w.Hkv, w.D, w.seed, q_len=1)
+    out, lse = _run(q, kc, vc, w.params)
+    ref_o, ref_l = O.decode(q, kc, vc, w.params)
+    assert_close(out.cpu().numpy(), lse.cpu().numpy(), ref_o, ref_l, w.name)
+
+
+def test_decode_deterministic_and_repeatable():
+    w = WORKLOADS["bifocal_decode_n131072"]
+    q, kc, vc = (t.cuda() for t in make_qkv(w.B, w.S, w.Hq, w.Hkv, w.D, w.seed, q_len=1))
+    from position_remapping_b200 import ropeattn as ra
+    ws = torch.empty(ra.decode_workspace_size(w.B, w.S, w.Hq, w.Hkv, w.D), dtype=torch.uint8, device="cuda")
+    a = ra.decode(q, kc, vc, w.params, workspace=ws)
+    a = (a[0].clone(), a[1].clone())
+    b = ra.decode(q, kc, vc, w.params, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_decode_workspace_error():
+    from position_remapping_b200 import ropeattn as ra
+    q, kc, vc = (t.cuda() for t in make_qkv(1, 1000, 4, 2, 128, seed=3, q_len=1))
+    with pytest.raises(ra.RopeAttnError) as e:
+        ra.decode(q, kc, vc, MapParams(O.STANDARD), workspace=torch.empty(8, dtype=torch.uint8, device="cuda"))
+    assert e.value.code == ra.ERR_WORKSPACE
