@@ -1,0 +1,446 @@
+"""Benchmark of the remapped-RoPE attention hot path on B200.
+
+One step = one Jet-Long bifocal prefill of 131072 tokens (32 q / 8 kv heads,
+head_dim 128, w_pretrained 32768 -> G = 4, w0 = 2048, base 1e6: the key
+rotation pre-pass and the attention kernel) followed by one bifocal decode
+step over a 131072-token cache (16 q / 8 kv heads, head_dim 128). Inputs are
+seeded iid N(0,1) bf16 tensors resident in HBM; every input is larger than
+the 126 MB L2, so no explicit flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0). ``value`` is prefill TFLOP/s over all ranks
+(4*D FLOPs per attended (query, key) pair per query head, each pair once);
+decode microseconds per token ride along. Multi-GPU runs are weak scaling:
+each rank runs its own independent problem, no collective on the data path;
+times are the max over ranks. ``--impl reference`` times the float64 CPU
+oracle on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, HERE)
+
+from position_remapping_b200.inputs import WORKLOADS, make_qkv  # noqa: E402
+
+METRIC = "128K bifocal-RoPE prefill TFLOP/s + decode µs/token; % of B200 roofline"
+PREFILL = WORKLOADS["bifocal_prefill_s131072"]
+DECODE = WORKLOADS["bifocal_decode_n131072"]
+PEAK_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def prefill_flops(w) -> float:
+    pairs = w.S * (w.S + 1) // 2          # causal pairs per (batch, head)
+    return 4.0 * w.D * pairs * w.Hq * w.B
+
+
+def decode_bytes(w) -> int:
+    kv = 2 * w.B * w.S * w.Hkv * w.D * 2
+    return kv + w.B * w.Hq * w.D * 2 + w.B * w.Hq * (w.D + 1) * 4
+
+
+def load_peaks():
+    path = os.path.join(HERE, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return dict(PEAK_FALLBACK), "fallback"
+
+
+def source_hash(*names) -> str:
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(HERE, "position_remapping_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_record(kernel: str, src_hash: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    try:
+        with open(os.path.join(HERE, "profiles", "traffic.json")) as f:
+            rec = json.load(f).get(kernel)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("source_hash") != src_hash:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str):
+        self.uuid = uuid
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        mhz, maxes, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8 or (self.uuid and self.uuid not in parts[0]):
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                maxes.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max(maxes), "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads", 0) for p in threadpool_info() if p.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle (baseline / reference arm): bounded samples of the same workload
+# ----------------------------------------------------------------------------
+def oracle_rows(n_rows: int):
+    S = PREFILL.S
+    step = S // n_rows
+    return [min(S - 1, i * step + step // 2) for i in range(n_rows)]
+
+
+def oracle_step(n_rows: int, q, k, v, qd, kd, vd):
+    """Times the oracle on `n_rows` rows of the prefill (all heads) and on one
+    full decode. Returns (prefill TFLOP/s, decode us/token, seconds, sample)."""
+    import oracle as O
+    rows = oracle_rows(n_rows)
+    flops = sum(4.0 * PREFILL.D * (t + 1) * PREFILL.Hq for t in rows)
+    t0 = time.perf_counter()
+    O.prefill(q, k, v, PREFILL.params, rows=rows, stage_bf16=True)
+    t1 = time.perf_counter()
+    O.decode(qd, kd, vd, DECODE.params)
+    t2 = time.perf_counter()
+    sample = (f"{n_rows} query rows (evenly spaced) x {PREFILL.Hq} heads of the {PREFILL.S}-token bifocal "
+              f"prefill, plus one full {DECODE.S}-key bifocal decode")
+    return flops / (t1 - t0) / 1e12, (t2 - t1) * 1e6, t2 - t0, sample
+
+
+def run_reference(args):
+    q, k, v = make_qkv(PREFILL.B, PREFILL.S, PREFILL.Hq, PREFILL.Hkv, PREFILL.D, PREFILL.seed)
+    qd, kd, vd = make_qkv(DECODE.B, DECODE.S, DECODE.Hq, DECODE.Hkv, DECODE.D, DECODE.seed, q_len=1)
+    n_rows = 4
+    vals, decs, secs = [], [], []
+    sample = ""
+    for i in range(args.warmup + args.steps):
+        tf, dus, s, sample = oracle_step(n_rows, q, k, v, qd, kd, vd)
+        if i >= args.warmup:
+            vals.append(tf)
+            decs.append(dus)
+            secs.append(s)
+    value = statistics.median(vals)
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.median(secs), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded iid N(0,1) bf16)",
+        "config": config_dict(args.gpus),
+        "decode_us_per_token": statistics.median(decs),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(n_gpus):
+    return {"workload": f"{PREFILL.name} + {DECODE.name}",
+            "prefill": {"B": PREFILL.B, "S": PREFILL.S, "Hq": PREFILL.Hq, "Hkv": PREFILL.Hkv, "D": PREFILL.D,
+                        "w0": PREFILL.params.w0, "w_pretrained": PREFILL.params.w_pretrained,
+                        "rope_base": PREFILL.params.rope_base},
+            "decode": {"B": DECODE.B, "n": DECODE.S, "Hq": DECODE.Hq, "Hkv": DECODE.Hkv, "D": DECODE.D},
+            "l2": "inputs larger than L2 (no flush)",
+            "parallelism": f"independent problem per GPU x{n_gpus}"}
+
+
+# ----------------------------------------------------------------------------
+# GPU arm
+# ----------------------------------------------------------------------------
+def run_profile_case(which: str):
+    """Capture-sized cases for ncu (a few GB on the device at most, inputs
+    still larger than L2). prefill: the 131072-token workload's kernel on a
+    32768-token sequence with w_pretrained 8192, so G = 4 as in the full run;
+    decode: the full 131072-key decode (512 MiB of cache)."""
+    from position_remapping_b200 import ropeattn as ra
+    dev = torch.device("cuda", 0)
+    if which == "prefill":
+        P = PREFILL
+        S = 32768
+        params = P.params.replace(w_pretrained=8192)
+        q, k, v = make_qkv(P.B, S, P.Hq, P.Hkv, P.D, P.seed, device=dev)
+        ws = torch.empty(ra.prefill_workspace_size(params, P.B, S, P.Hq, P.Hkv, P.D), dtype=torch.uint8, device=dev)
+        out = torch.empty((P.B, S, P.Hq, P.D), dtype=torch.float32, device=dev)
+        lse = torch.empty((P.B, P.Hq, S), dtype=torch.float32, device=dev)
+        for _ in range(3):
+            ra.prefill(q, k, v, params, out=out, lse=lse, workspace=ws)
+    else:
+        Dd = DECODE
+        qd, kd, vd = make_qkv(Dd.B, Dd.S, Dd.Hq, Dd.Hkv, Dd.D, Dd.seed, device=dev, q_len=1)
+        for _ in range(3):
+            ra.decode(qd, kd, vd, Dd.params)
+    torch.cuda.synchronize()
+    ra.status()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["prefill", "decode"], default=None,
+                    help="run a capture-sized case of one kernel three times (for ncu); no timing, no JSON")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args)
+        return
+    if args.profile:
+        run_profile_case(args.profile)
+        return
+
+    import datetime
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    from position_remapping_b200 import ropeattn as ra
+
+    # inputs resident in HBM (each rank its own seeded problem)
+    P, Dd = PREFILL, DECODE
+    q, k, v = make_qkv(P.B, P.S, P.Hq, P.Hkv, P.D, P.seed + 17 * rank, device=dev)
+    qd, kd, vd = make_qkv(Dd.B, Dd.S, Dd.Hq, Dd.Hkv, Dd.D, Dd.seed + 17 * rank, device=dev, q_len=1)
+    out = torch.empty((P.B, P.S, P.Hq, P.D), dtype=torch.float32, device=dev)
+    lse = torch.empty((P.B, P.Hq, P.S), dtype=torch.float32, device=dev)
+    ws = torch.empty(ra.prefill_workspace_size(P.params, P.B, P.S, P.Hq, P.Hkv, P.D), dtype=torch.uint8, device=dev)
+    outd = torch.empty((Dd.B, Dd.Hq, Dd.D), dtype=torch.float32, device=dev)
+    lsed = torch.empty((Dd.B, Dd.Hq), dtype=torch.float32, device=dev)
+    wsd = torch.empty(ra.decode_workspace_size(Dd.B, Dd.S, Dd.Hq, Dd.Hkv, Dd.D), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        ra.prefill_prepare(k, P.Hq, P.params, ws, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        ra.prefill_attend(q, k, v, P.params, out, lse, ws, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        ra.decode(qd, kd, vd, Dd.params, out=outd, lse=lsed, workspace=wsd, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ra.status()
+
+    uuid = ""
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.3)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    ra.status()
+
+    total_ms = t_start.elapsed_time(t_end)
+    prep_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    attn_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+    dec_ms = sum(e[2].elapsed_time(e[3]) for e in evs)
+
+    # ---- end to end through the public API with host buffers
+    qh = q.cpu().pin_memory(); kh = k.cpu().pin_memory(); vh = v.cpu().pin_memory()
+    qdh = qd.cpu().pin_memory()
+    outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    lseh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    outdh = torch.empty(outd.shape, dtype=outd.dtype).pin_memory()
+    lsedh = torch.empty(lsed.shape, dtype=lsed.dtype).pin_memory()
+    h2d = (qh.numel() + kh.numel() + vh.numel() + qdh.numel()) * 2
+    d2h = (outh.numel() + lseh.numel() + outdh.numel() + lsedh.numel()) * 4
+
+    def e2e_step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        q.copy_(qh, non_blocking=True); k.copy_(kh, non_blocking=True); v.copy_(vh, non_blocking=True)
+        ra.prefill(q, k, v, P.params, out=out, lse=lse, workspace=ws, stream=stream)
+        outh.copy_(out, non_blocking=True); lseh.copy_(lse, non_blocking=True)
+        if ev is not None:
+            ev[1].record(stream)
+        qd.copy_(qdh, non_blocking=True)
+        ra.decode(qd, kd, vd, Dd.params, out=outd, lse=lsed, workspace=wsd, stream=stream)
+        outdh.copy_(outd, non_blocking=True); lsedh.copy_(lsed, non_blocking=True)
+        if ev is not None:
+            ev[2].record(stream)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        e2e_step(e_evs[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e2e_pre_ms = sum(e[0].elapsed_time(e[1]) for e in e_evs)
+    e2e_dec_ms = sum(e[1].elapsed_time(e[2]) for e in e_evs)
+    ra.status()
+
+    times = torch.tensor([total_ms, prep_ms, attn_ms, dec_ms, e2e_pre_ms, e2e_dec_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    total_ms, prep_ms, attn_ms, dec_ms, e2e_pre_ms, e2e_dec_ms = times.tolist()
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    K = args.steps
+    flops = prefill_flops(P)
+    value = world * flops * K / ((prep_ms + attn_ms) / 1e3) / 1e12
+    attn_tflops = flops * K / (attn_ms / 1e3) / 1e12
+    dec_us = dec_ms * 1e3 / K
+    dec_gbs = decode_bytes(Dd) * K / (dec_ms / 1e3) / 1e9
+    peaks, peak_src = load_peaks()
+    # the attention kernel runs for ~0.1 s per launch inside a long step: sustained peak
+    tpeak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    hpeak = float(peaks.get("hbm_gbs"))
+    src_p = source_hash("prefill_sm100.cuh", "common.cuh")
+    src_d = source_hash("decode_sm100.cuh", "common.cuh")
+    tr_p = traffic_record("prefill_kernel", src_p)
+    tr_d = traffic_record("decode_kernel", src_d)
+
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms / K,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded iid N(0,1) bf16, no weights)",
+        "config": config_dict(world),
+        "prefill_ms": (prep_ms + attn_ms) / K,
+        "prefill_prepare_ms": prep_ms / K,
+        "prefill_attend_ms": attn_ms / K,
+        "prefill_tokens_per_s": world * P.S * P.B * K / ((prep_ms + attn_ms) / 1e3),
+        "decode_us_per_token": dec_us,
+        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": tpeak, "unit": "TFLOP/s",
+                     "frac": attn_tflops / tpeak, "traffic": tr_p,
+                     "kernel": "prefill_kernel<128,2> (attention)",
+                     "peak_source": f"{peak_src} bf16_tflops_sustained",
+                     "algorithmic": f"{flops:.6g} FLOP per launch"},
+        "roofline_decode": {"bound": "hbm", "achieved": dec_gbs, "peak": hpeak, "unit": "GB/s",
+                            "frac": dec_gbs / hpeak, "traffic": tr_d,
+                            "kernel": "decode_kernel<128,2> (+ counter memset)",
+                            "peak_source": f"{peak_src} hbm_gbs",
+                            "algorithmic": f"{decode_bytes(Dd)} B per launch"},
+        "clocks": clocks,
+        "gpu_launches": 3 * K,
+        "e2e": {"value": world * flops * K / (e2e_pre_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "decode_us_per_token": e2e_dec_ms * 1e3 / K},
+    }
+
+    if world == 1 and not args.no_cpu_baseline:
+        torch.cuda.synchronize()
+        qc, kc, vc = make_qkv(P.B, P.S, P.Hq, P.Hkv, P.D, P.seed)
+        qdc, kdc, vdc = make_qkv(Dd.B, Dd.S, Dd.Hq, Dd.Hkv, Dd.D, Dd.seed, q_len=1)
+        tf, dus, secs, sample = oracle_step(8, qc, kc, vc, qdc, kdc, vdc)
+        line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": sample, "decode_us_per_token": dus, "seconds": secs}
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

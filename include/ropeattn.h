@@ -124,6 +124,23 @@ int ropeattn_prefill(const void* q, const void* k, const void* v,
                      const ropeattn_params* params,
                      void* workspace, size_t workspace_bytes, void* stream);
 
+/* The two halves of ropeattn_prefill, for callers that reuse the rotated
+ * keys (several query blocks against the same keys) or time the stages:
+ *   ropeattn_prefill_prepare writes the rotated keys and the query angle
+ *   tables into `workspace` (reads k only; no-op for NOPE);
+ *   ropeattn_prefill_attend runs the attention kernel on a workspace that a
+ *   prepare call with the same params and shapes filled earlier on the same
+ *   stream (k is read directly only for NOPE).
+ * ropeattn_prefill(...) == prepare(...) followed by attend(...).
+ * Same arguments, layouts and errors as ropeattn_prefill. */
+int ropeattn_prefill_prepare(const void* k, int64_t B, int64_t S, int32_t Hq, int32_t Hkv, int32_t D,
+                             const ropeattn_params* params, void* workspace, size_t workspace_bytes,
+                             void* stream);
+int ropeattn_prefill_attend(const void* q, const void* k, const void* v, float* out, float* lse,
+                            int64_t B, int64_t S, int32_t Hq, int32_t Hkv, int32_t D,
+                            const ropeattn_params* params,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
 /* Bytes of device workspace ropeattn_decode needs (split-KV partials and
  * per-head arrival counters). Depends on the current device's SM count. */
 size_t ropeattn_decode_workspace_size(int64_t B, int64_t n, int32_t Hq,

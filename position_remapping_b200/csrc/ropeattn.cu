@@ -288,9 +288,15 @@ size_t ropeattn_prefill_workspace_size(const ropeattn_params* params, int64_t B,
   return prefill_layout(eff, B, S, Hkv, D).total;
 }
 
-int ropeattn_prefill(const void* q, const void* k, const void* v, float* out, float* lse, int64_t B, int64_t S,
-                     int32_t Hq, int32_t Hkv, int32_t D, const ropeattn_params* params, void* workspace,
-                     size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+enum : int { kStagePrepare = 1, kStageAttend = 2 };
+
+int prefill_impl(int stages, const void* q, const void* k, const void* v, float* out, float* lse, int64_t B,
+                 int64_t S, int32_t Hq, int32_t Hkv, int32_t D, const ropeattn_params* params, void* workspace,
+                 size_t workspace_bytes, void* stream) {
   g_last_error.clear();
   int rc = check_shapes(B, S, Hq, Hkv, D);
   if (rc) return rc;
@@ -299,9 +305,13 @@ int ropeattn_prefill(const void* q, const void* k, const void* v, float* out, fl
   rc = check_params(params, S, D, &m, &eff);
   if (rc) return rc;
   if (B == 0 || S == 0) return ROPEATTN_OK;
-  if (!q || !k || !v || !out || !lse) return fail(ROPEATTN_ERR_INVALID_ARG, "null tensor pointer");
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
-    return fail(ROPEATTN_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (!k) return fail(ROPEATTN_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(k)) return fail(ROPEATTN_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (stages & kStageAttend) {
+    if (!q || !v || !out || !lse) return fail(ROPEATTN_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned16(q) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+      return fail(ROPEATTN_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  }
   if ((static_cast<long long>((S + kBM - 1) / kBM)) * Hq * B > 0x7fffffffLL)
     return fail(ROPEATTN_ERR_INVALID_ARG, "too many query tiles");
   rc = check_device();
@@ -318,7 +328,7 @@ int ropeattn_prefill(const void* q, const void* k, const void* v, float* out, fl
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   m.kind = eff;
 
-  // 1) keys rotated once per map, and the query angle tables
+  // workspace views: keys rotated once per map, and the query angle tables
   const void* kmap0 = k;
   const void* kmap1 = k;
   PrefillParams pp{};
@@ -334,17 +344,19 @@ int ropeattn_prefill(const void* q, const void* k, const void* v, float* out, fl
     a.Hkv = Hkv;
     a.D = D;
     a.m = m;
-    fill_theta(params, D, a.theta);
-    const int rows = 256 / (D / 2);
-    rope_prep_kernel<<<static_cast<unsigned>((S + rows - 1) / rows), 256, 0, st>>>(a);
-    CUDA_TRY(cudaGetLastError(), "rope_prep launch");
+    if (stages & kStagePrepare) {
+      fill_theta(params, D, a.theta);
+      const int rows = 256 / (D / 2);
+      rope_prep_kernel<<<static_cast<unsigned>((S + rows - 1) / rows), 256, 0, st>>>(a);
+      CUDA_TRY(cudaGetLastError(), "rope_prep launch");
+    }
     kmap0 = a.k_rot0;
     kmap1 = lay.nmaps > 1 ? static_cast<const void*>(a.k_rot1) : kmap0;
     pp.tab0 = a.tab0;
     pp.tab1 = a.tab1;
   }
+  if (!(stages & kStageAttend)) return ROPEATTN_OK;
 
-  // 2) attention
   CUtensorMap tq, tk0, tk1, tv;
   if ((rc = make_map(&tq, q, D, Hq, S, B, 64, kBM, true))) return rc;
   if ((rc = make_map(&tk0, kmap0, D, Hkv, S, B, 64, kBN, true))) return rc;
@@ -364,6 +376,30 @@ int ropeattn_prefill(const void* q, const void* k, const void* v, float* out, fl
   const int grid = pp.nqt * Hq * static_cast<int>(B);
   if (D == 128) return launch_prefill<128, 2>(tq, tk0, tk1, tv, pp, grid, st);
   return launch_prefill<64, 4>(tq, tk0, tk1, tv, pp, grid, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int ropeattn_prefill(const void* q, const void* k, const void* v, float* out, float* lse, int64_t B, int64_t S,
+                     int32_t Hq, int32_t Hkv, int32_t D, const ropeattn_params* params, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  return prefill_impl(kStagePrepare | kStageAttend, q, k, v, out, lse, B, S, Hq, Hkv, D, params, workspace,
+                      workspace_bytes, stream);
+}
+
+int ropeattn_prefill_prepare(const void* k, int64_t B, int64_t S, int32_t Hq, int32_t Hkv, int32_t D,
+                             const ropeattn_params* params, void* workspace, size_t workspace_bytes, void* stream) {
+  return prefill_impl(kStagePrepare, nullptr, k, nullptr, nullptr, nullptr, B, S, Hq, Hkv, D, params, workspace,
+                      workspace_bytes, stream);
+}
+
+int ropeattn_prefill_attend(const void* q, const void* k, const void* v, float* out, float* lse, int64_t B,
+                            int64_t S, int32_t Hq, int32_t Hkv, int32_t D, const ropeattn_params* params,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  return prefill_impl(kStageAttend, q, k, v, out, lse, B, S, Hq, Hkv, D, params, workspace, workspace_bytes,
+                      stream);
 }
 
 size_t ropeattn_decode_workspace_size(int64_t B, int64_t n, int32_t Hq, int32_t Hkv, int32_t D) {

@@ -22,6 +22,7 @@ ERR_INVALID_ARG, ERR_UNSUPPORTED_DEVICE, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = 
 
 # every symbol include/ropeattn.h declares
 EXPORTS = ("ropeattn_posmap", "ropeattn_prefill_workspace_size", "ropeattn_prefill",
+           "ropeattn_prefill_prepare", "ropeattn_prefill_attend",
            "ropeattn_decode_workspace_size", "ropeattn_decode", "ropeattn_status",
            "ropeattn_last_error", "ropeattn_version")
 
@@ -73,6 +74,8 @@ def _load() -> ctypes.CDLL:
     lib.ropeattn_prefill_workspace_size.argtypes = [P, i64, i64, i32, i32, i32]
     lib.ropeattn_prefill_workspace_size.restype = sz
     lib.ropeattn_prefill.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, P, vp, sz, vp]
+    lib.ropeattn_prefill_prepare.argtypes = [vp, i64, i64, i32, i32, i32, P, vp, sz, vp]
+    lib.ropeattn_prefill_attend.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, P, vp, sz, vp]
     lib.ropeattn_decode_workspace_size.argtypes = [i64, i64, i32, i32, i32]
     lib.ropeattn_decode_workspace_size.restype = sz
     lib.ropeattn_decode.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, P, vp, sz, vp]
@@ -80,7 +83,8 @@ def _load() -> ctypes.CDLL:
     lib.ropeattn_last_error.argtypes = []
     lib.ropeattn_last_error.restype = ctypes.c_char_p
     lib.ropeattn_version.argtypes = []
-    for name in ("ropeattn_posmap", "ropeattn_prefill", "ropeattn_decode", "ropeattn_status", "ropeattn_version"):
+    for name in ("ropeattn_posmap", "ropeattn_prefill", "ropeattn_prefill_prepare", "ropeattn_prefill_attend",
+                 "ropeattn_decode", "ropeattn_status", "ropeattn_version"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -155,6 +159,26 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, params: MapParams
     _check(lib.ropeattn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, S, Hq, Hkv, D,
                                 ctypes.byref(cp), _ptr(workspace), ws_bytes, _stream(stream)))
     return out, lse
+
+
+def prefill_prepare(k: torch.Tensor, Hq: int, params: MapParams, workspace: torch.Tensor, stream=None) -> None:
+    """First half of prefill: rotated keys and query angle tables into ``workspace``."""
+    B, S, Hkv, D = k.shape
+    cp = to_cparams(params)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.ropeattn_prefill_prepare(_ptr(k), B, S, Hq, Hkv, D, ctypes.byref(cp), _ptr(workspace), ws_bytes,
+                                        _stream(stream)))
+
+
+def prefill_attend(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, params: MapParams,
+                   out: torch.Tensor, lse: torch.Tensor, workspace: Optional[torch.Tensor], stream=None) -> None:
+    """Second half of prefill: attention on a workspace filled by prefill_prepare."""
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    cp = to_cparams(params)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.ropeattn_prefill_attend(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, S, Hq, Hkv, D,
+                                       ctypes.byref(cp), _ptr(workspace), ws_bytes, _stream(stream)))
 
 
 def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, params: MapParams,
