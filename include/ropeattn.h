@@ -167,6 +167,28 @@ int ropeattn_decode(const void* q, const void* k_cache, const void* v_cache,
                     const ropeattn_params* params,
                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* ropeattn_decode for callers that cannot allocate device memory when they
+ * call: for example a plug-in running inside an engine that owns every device
+ * allocation, or a latency-critical serving loop where a cudaMalloc (which can
+ * synchronize the device) is not acceptable. The pages have no counterpart:
+ * this is a library convenience, not part of the method.
+ * Same arguments, layouts, results and errors as ropeattn_decode, without the
+ * workspace: the split-KV scratch lives in a 4 MiB array inside the library
+ * (a file-scope __device__ array that every GPU loading the library holds
+ * until process exit). Shapes whose ropeattn_decode_workspace_size exceeds
+ * 4 MiB are rejected with ROPEATTN_ERR_WORKSPACE before any launch.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture. The call itself allocates nothing: it clears the scratch counters
+ * with cudaMemsetAsync on `stream` and launches the decode kernel.
+ * All calls share the one array: calls that may overlap on the GPU (different
+ * streams without ordering, or different host threads) race and must not be
+ * issued; calls on one stream are safe. */
+int ropeattn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                            float* out, float* lse,
+                            int64_t B, int64_t n, int32_t Hq, int32_t Hkv, int32_t D,
+                            const ropeattn_params* params, void* stream);
+
 /* Reads and clears the device status word of the current device (waits for
  * the device to be idle first). Returns ROPEATTN_OK, or ROPEATTN_ERR_TIMEOUT
  * if any kernel since the last call gave up on a bounded wait (its outputs

@@ -476,4 +476,52 @@ int ropeattn_decode(const void* q, const void* k_cache, const void* v_cache, flo
   return launch_decode<64, 8>(tk, tv, dp, grid, st);
 }
 
+
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode without a caller-provided workspace: the scratch is a fixed array
+// owned by the library. Callers that cannot allocate device memory pass only
+// inputs and outputs.
+// ---------------------------------------------------------------------------
+static constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (the host-side name is only a stand-in, never a device address).
+int noalloc_scratch_ptr(void** out) {
+  static std::mutex mu;
+  static void* ptrs[64];
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(ROPEATTN_ERR_UNSUPPORTED_DEVICE, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    CUDA_TRY(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress(scratch)");
+    ptrs[dev] = p;
+  }
+  *out = ptrs[dev];
+  return ROPEATTN_OK;
+}
+
+}  // namespace
+
+extern "C" int ropeattn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, float* out,
+                                       float* lse, int64_t B, int64_t n, int32_t Hq, int32_t Hkv, int32_t D,
+                                       const ropeattn_params* params, void* stream) {
+  g_last_error.clear();
+  const size_t need = ropeattn_decode_workspace_size(B, n, Hq, Hkv, D);
+  if (need > kNoAllocScratchBytes)
+    return fail(ROPEATTN_ERR_WORKSPACE,
+                "this decode needs %zu bytes of scratch; the built-in scratch holds %zu (use ropeattn_decode)", need,
+                kNoAllocScratchBytes);
+  void* ws = nullptr;
+  if (need > 0) {
+    const int rc = noalloc_scratch_ptr(&ws);
+    if (rc) return rc;
+  }
+  return ropeattn_decode(q, k_cache, v_cache, out, lse, B, n, Hq, Hkv, D, params, ws, kNoAllocScratchBytes, stream);
+}

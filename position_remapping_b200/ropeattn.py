@@ -23,7 +23,7 @@ ERR_INVALID_ARG, ERR_UNSUPPORTED_DEVICE, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = 
 # every symbol include/ropeattn.h declares
 EXPORTS = ("ropeattn_posmap", "ropeattn_prefill_workspace_size", "ropeattn_prefill",
            "ropeattn_prefill_prepare", "ropeattn_prefill_attend",
-           "ropeattn_decode_workspace_size", "ropeattn_decode", "ropeattn_status",
+           "ropeattn_decode_workspace_size", "ropeattn_decode", "ropeattn_decode_noalloc", "ropeattn_status",
            "ropeattn_last_error", "ropeattn_version")
 
 
@@ -79,6 +79,8 @@ def _load() -> ctypes.CDLL:
     lib.ropeattn_decode_workspace_size.argtypes = [i64, i64, i32, i32, i32]
     lib.ropeattn_decode_workspace_size.restype = sz
     lib.ropeattn_decode.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, P, vp, sz, vp]
+    lib.ropeattn_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, P, vp]
+    lib.ropeattn_decode_noalloc.restype = ctypes.c_int
     lib.ropeattn_status.argtypes = []
     lib.ropeattn_last_error.argtypes = []
     lib.ropeattn_last_error.restype = ctypes.c_char_p
