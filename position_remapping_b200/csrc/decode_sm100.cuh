@@ -1,18 +1,23 @@
 // One decode step over an untouched RoPE key cache (Jet-Long §3.2), sm_100a.
 //
 // Split-KV: CTA (split, kv head, batch) owns a contiguous key range of one KV
-// head. Warp 8 streams that range through shared memory with TMA, 32 keys per
-// stage (no swizzle, no multicast); warps 0-7 consume it, each lane group of
-// 8 lanes taking one key per stage with two 16-byte shared loads per lane.
+// head; the grid is one wave (one CTA per SM). The range streams through a
+// shared-memory ring by TMA, 64 keys per stage (no swizzle, no multicast).
+// All 8 warps consume; the last warp to release a slot issues the copy of the
+// stage that reuses it, so no thread polls.
 //
-// Scores: the query is rotated once to its position p(n-1) in fp32. For the
-// bifocal map, keys with (n-1) - k > w0 are read through the correction
-// rotation of Eq. 6, k_remote = R(Delta k) k_cache[k] with
-// Delta k = floor(k/G) - k = -u(k), against the query corrected by
-// Delta q = floor((n-1)/G) - (n-1). Each lane carries the phasors
-// exp(i u(k) theta_i) of its pairs and advances them from one key of its
-// stream to the next (32 positions apart) by one complex multiply; they are
-// re-seeded exactly (argument reduced in double) every 32 stages.
+// Scores: the query is rotated once to its position p(n-1) in fp32 and
+// prescaled by softmax_scale * log2(e). For the bifocal map the query is then
+// corrected by Delta q = f(n-1) - (n-1) (Eq. 5-6), and every cached key k is
+// read through a rotation R(-u theta): remote keys ((n-1) - k > w0) use
+// u = u(k) = k - floor(k/G), i.e. the correction Delta k of Eq. 6; local keys
+// use u = u(n-1), which turns q_remote . R(Delta q) k_cache back into
+// q_local . k_cache exactly (R_a R_b = R_{a+b}), so one query view serves both
+// windows. Each lane carries the phasors exp(i u theta) of its pairs and
+// advances them by one complex multiply per stage (a key moves 64 positions);
+// they are re-seeded exactly (argument reduced in double) every 16 stages.
+// Packed fp32x2 FMAs carry the rotation, the dot products and the
+// accumulation. Each lane group of 8 lanes takes two keys per stage.
 //
 // Each lane group keeps an online softmax per query head of the GQA group;
 // the CTA merges its groups and warps, writes (O, m, l) for its split, and the
@@ -24,11 +29,24 @@
 
 namespace ropeattn {
 
-constexpr int kDecKeys = 32;         // keys per stage
-constexpr int kDecStages = 6;        // ring depth
-constexpr int kDecConsumerWarps = 8;
-constexpr int kDecThreads = (kDecConsumerWarps + 1) * 32;
-constexpr int kDecReseed = 32;       // stages between exact phasor re-seeds
+constexpr int kDecKeys = 64;         // keys per stage: one per lane group of 16 warps
+constexpr int kDecReseed = 16;       // stages between exact phasor re-seeds
+
+// Warps per CTA and keys per lane group per stage: 16 warps x 1 key (more
+// warps to hide latency) or 8 warps x 2 keys (more independent work per
+// warp); a stage is always 64 keys. The stage multipliers of the phasor
+// recurrence are held in registers with 2 keys per group, else read from
+// shared memory each stage.
+#ifndef ROPEATTN_DECODE_KPG
+#define ROPEATTN_DECODE_KPG 1
+#endif
+template <int D, int GRP>
+struct DecodeShape {
+  static constexpr int kKeysPerGroup = (GRP * D <= 256) ? ROPEATTN_DECODE_KPG : 2;
+  static constexpr int kWarps = 16 / kKeysPerGroup;
+  static constexpr int kThreads = kWarps * 32;
+  static constexpr bool kMulInRegs = kKeysPerGroup == 2;
+};
 
 struct DecodeParams {
   const __nv_bfloat16* q;  // [B, Hq, D]
@@ -40,8 +58,8 @@ struct DecodeParams {
   int B, n, Hq, Hkv;
   int nsplit, keys_per_split;
   int k_begin;             // first attended key (Periodic RoPE window), else 0
-  int k_local;             // keys >= k_local are read without correction
-  int bifocal;             // 1 when remote keys need the correction rotation
+  int k_local;             // keys >= k_local are local (exact-position) keys
+  int bifocal;             // 1 when keys are read through the correction rotation
   PosMap m;
   float scale_log2;
   double theta[kMaxPairs];
@@ -59,26 +77,40 @@ __device__ __forceinline__ float2 phase_cs(double phase) {
 
 template <int D>
 struct DecodeSmem {
+  static constexpr int kStages = D == 128 ? 6 : 10;             // ring depth
   static constexpr int kRowBytes = D * 2;
   static constexpr int kStageBytes = 2 * kDecKeys * kRowBytes;  // K then V
-  static constexpr int kRing = kDecStages * kStageBytes;
-  static constexpr int kBar = kRing;                             // full[], empty[]
-  static constexpr int kMisc = kBar + 2 * kDecStages * 8;       // abort flag, last flag
+  static constexpr int kRing = kStages * kStageBytes;
+  static constexpr int kMul = kRing;                             // [2][D/2] float2 stage multipliers
+  static constexpr int kBar = kMul + D * 8;                      // full[] mbarriers
+  static constexpr int kCnt = kBar + kStages * 8;                // release counters per slot
+  static constexpr int kMisc = kCnt + kStages * 4;               // abort flag, last flag
   static constexpr int kTotal = kMisc + 16;
 };
 
+// Packed fp32x2 helpers (Blackwell FFMA2 / FMUL2).
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 neg2(float2 a) { return make_float2(-a.x, -a.y); }
+
 template <int D, int GRP>
-__global__ void __launch_bounds__(kDecThreads)
+__global__ void __launch_bounds__(DecodeShape<D, GRP>::kThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const DecodeParams p) {
   using L = DecodeSmem<D>;
-  constexpr int NV = D / 64;         // 16-byte vectors per lane per row
-  constexpr int NE = 8 * NV;         // elements per lane
-  constexpr int NP = 4 * NV;         // rotation pairs per lane
+  using SH = DecodeShape<D, GRP>;
+  constexpr int NS = L::kStages;
+  constexpr int NW = SH::kWarps;
+  constexpr int NV = D / 64;              // 16-byte vectors per lane per row
+  constexpr int NJ = 2 * NV;              // pair-pairs per lane (two rotation pairs each)
+  constexpr int KPG = SH::kKeysPerGroup;  // keys per lane group per stage
+  constexpr int RS = kDecKeys / KPG;      // row stride between a group's keys in a stage
 
   extern __shared__ __align__(128) uint8_t smem[];
+  float2* mul_tab = reinterpret_cast<float2*>(smem + L::kMul);   // [carry][pair] (cos, sin)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  uint64_t* empty = full + kDecStages;
+  int* released = reinterpret_cast<int*>(smem + L::kCnt);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc);
   volatile int* last_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
@@ -92,298 +124,390 @@ __global__ void __launch_bounds__(kDecThreads)
   const int kb = min(p.n, p.k_begin + split * p.keys_per_split);
   const int ke = min(p.n, kb + p.keys_per_split);
   const int nstage = (ke - kb + kDecKeys - 1) / kDecKeys;
+  const int G = p.m.G;
+  const int stage_q = kDecKeys / G, stage_r = kDecKeys - stage_q * G;
 
+  auto issue = [&](int st) {  // copy stage st (K rows then V rows) into its slot
+    const int slot = st % NS;
+    uint8_t* dst = smem + slot * L::kStageBytes;
+    mbar_arrive_expect_tx(full + slot, L::kStageBytes);
+    tma_load_4d(dst, &tmK, full + slot, 0, hkv, kb + st * kDecKeys, b);
+    tma_load_4d(dst + kDecKeys * L::kRowBytes, &tmV, full + slot, 0, hkv, kb + st * kDecKeys, b);
+  };
   if (tid == 0) {
-    for (int i = 0; i < kDecStages; ++i) {
+    for (int i = 0; i < NS; ++i) {
       mbar_init(full + i, 1);
-      mbar_init(empty + i, kDecConsumerWarps);
+      released[i] = 0;
     }
     *abort_flag = 0;
     *last_flag = 0;
     mbar_fence_init();
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    for (int st = 0; st < NS && st < nstage; ++st) issue(st);
+  }
+  if (p.bifocal) {
+    // per pair: (cos, sin) of the stage advance of u without and with a
+    // group-boundary carry: 64 - 64/G and 63 - 64/G positions
+    for (int i = tid; i < D / 2; i += SH::kThreads) {
+      const double du = kDecKeys - stage_q;
+      mul_tab[i] = phase_cs(du * p.theta[i]);
+      mul_tab[D / 2 + i] = phase_cs((du - 1.0) * p.theta[i]);
+    }
   }
   __syncthreads();
 
-  if (warp == kDecConsumerWarps) {
-    // ---------------------------------------------------------------- TMA
-    if (lane == 0) {
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      for (int st = 0; st < nstage; ++st) {
-        const int slot = st % kDecStages;
-        if (!mbar_wait(empty + slot, ((st / kDecStages) & 1) ^ 1, abort_flag)) break;
-        uint8_t* dst = smem + slot * L::kStageBytes;
-        mbar_arrive_expect_tx(full + slot, L::kStageBytes);
-        tma_load_4d(dst, &tmK, full + slot, 0, hkv, kb + st * kDecKeys, b);
-        tma_load_4d(dst + kDecKeys * L::kRowBytes, &tmV, full + slot, 0, hkv, kb + st * kDecKeys, b);
-      }
-    }
-  } else {
-    // ----------------------------------------------------------- consumers
-    const int j4 = lane >> 3;             // lane group within the warp
-    const int l8 = lane & 7;              // lane within the group
-    const int ks = warp * 4 + j4;         // key stream 0..31 == row in a stage
-    const int t = p.n - 1;                // query position index
-    // element e of this lane is dimension 64*(e/8) + 8*l8 + e%8; pair e/2
-    auto pair_index = [&](int pp) { return 32 * (pp >> 2) + 4 * l8 + (pp & 3); };
+  const int j4 = lane >> 3;             // lane group within the warp
+  const int l8 = lane & 7;              // lane within the group
+  const int ks = warp * 4 + j4;         // key stream: rows ks + RS * kk of every stage
+  const unsigned gmask = 0xFFu << (8 * j4);
+  const int t = p.n - 1;                // query position index
+  const int u_t = t - t / G;            // u of the query: local keys are read at u(t)
+  // Lane pair-pair j holds rotation pairs c = 0, 1 at word 2(j%2)+c of the
+  // 16-byte vector j/2: global pair 32 (j/2) + 4 l8 + 2 (j%2) + c.
+  auto gpair = [&](int j, int c) { return 32 * (j >> 1) + 4 * l8 + 2 * (j & 1) + c; };
+  const float2 kNeg = f2(-1.f, -1.f);
 
-    // query: rotate to p(t) (the local view) and, for the bifocal map, apply
-    // the correction Delta q on top (the remote view, Eq. 5-6). Only one view
-    // is held in registers; a stream switches from remote to local once.
-    float qc[GRP][NE];
-    auto load_query = [&](bool remote_view) {
-      const int pq = pos_primary(p.m, t);
-      const int dq = pos_remote(p.m, t) - t;
-#pragma unroll
-      for (int gi = 0; gi < GRP; ++gi) {
-        const int hq = hkv * GRP + gi;
-        const uint4* qs = reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(b) * p.Hq + hq) * D);
-#pragma unroll
-        for (int v = 0; v < NV; ++v) {
-          const uint4 xq = __ldg(qs + v * 8 + l8);
-          const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int pp = v * 4 + e;
-            const double th = p.theta[pair_index(pp)];
-            float a0 = bf16lo(xw[e]), a1 = bf16hi(xw[e]);
-            if (p.m.kind != kNope) {
-              const float2 cs = phase_cs(static_cast<double>(pq) * th);
-              rot_pair(bf16lo(xw[e]), bf16hi(xw[e]), cs.x, cs.y, a0, a1);
-            }
-            if (remote_view) {
-              const float2 cd = phase_cs(static_cast<double>(dq) * th);
-              const float b0 = a0, b1 = a1;
-              rot_pair(b0, b1, cd.x, cd.y, a0, a1);
-            }
-            qc[gi][2 * pp] = a0;
-            qc[gi][2 * pp + 1] = a1;
-          }
-        }
-      }
-    };
-    bool q_remote = p.bifocal && (kb + ks) < p.k_local;
-    load_query(q_remote);
-
-    // phasors exp(i u theta) for this lane's pairs, u(k) = k - floor(k/G)
-    const int G = p.m.G;
-    const int step_lo = kDecKeys - kDecKeys / G;  // u(k+32) - u(k) is step_lo or step_lo - 1
-    float2 ph[NP], mul_a[NP], mul_b[NP];
-    auto useed = [&](int k) { return k - k / G; };
-    auto reseed = [&](int k) {
-      const int u = useed(k);
-#pragma unroll
-      for (int pp = 0; pp < NP; ++pp) ph[pp] = phase_cs(static_cast<double>(u) * p.theta[pair_index(pp)]);
-    };
-    if (p.bifocal) {
-#pragma unroll
-      for (int pp = 0; pp < NP; ++pp) {
-        const double th = p.theta[pair_index(pp)];
-        mul_a[pp] = phase_cs(static_cast<double>(step_lo) * th);
-        mul_b[pp] = phase_cs(static_cast<double>(step_lo - 1) * th);
-      }
-      reseed(kb + ks);
-    }
-
-    float m_run[GRP], l_run[GRP], acc[GRP][NE];
+  // query, prescaled by softmax scale * log2(e): rotated to p(t) and, for
+  // the bifocal map, corrected by Delta q on top (the remote view, Eq. 5-6)
+  float2 Q0[GRP][NJ], Q1[GRP][NJ];
+  {
+    const int pq = pos_primary(p.m, t);
+    const int dq = pos_remote(p.m, t) - t;
 #pragma unroll
     for (int gi = 0; gi < GRP; ++gi) {
-      m_run[gi] = -INFINITY;
-      l_run[gi] = 0.f;
-#pragma unroll
-      for (int e = 0; e < NE; ++e) acc[gi][e] = 0.f;
-    }
-
-    bool ok = true;
-    for (int st = 0; st < nstage; ++st) {
-      const int slot = st % kDecStages;
-      ok = __all_sync(0xffffffffu, mbar_wait(full + slot, (st / kDecStages) & 1, abort_flag));
-      if (!ok) break;
-      const uint8_t* row = smem + slot * L::kStageBytes + ks * L::kRowBytes;
-      uint4 kv[NV], vv[NV];
+      const int hq = hkv * GRP + gi;
+      const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(b) * p.Hq + hq) * D);
 #pragma unroll
       for (int v = 0; v < NV; ++v) {
-        kv[v] = *reinterpret_cast<const uint4*>(row + v * 128 + l8 * 16);
-        vv[v] = *reinterpret_cast<const uint4*>(row + kDecKeys * L::kRowBytes + v * 128 + l8 * 16);
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty + slot);
-
-      const int k = kb + st * kDecKeys + ks;
-      const bool valid = k < ke;                      // rows past the range are ignored
-      const bool remote = p.bifocal && k < p.k_local;
-      if (q_remote && !remote) {                      // this stream reached the local window
-        load_query(false);
-        q_remote = false;
-      }
-      float x[NE];
-#pragma unroll
-      for (int v = 0; v < NV; ++v) {
-        const uint32_t w[4] = {kv[v].x, kv[v].y, kv[v].z, kv[v].w};
+        const uint4 xq = __ldg(qsrc + v * 8 + l8);
+        const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
+        float r0[4], r1[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          x[v * 8 + 2 * e] = bf16lo(w[e]);
-          x[v * 8 + 2 * e + 1] = bf16hi(w[e]);
+          const double th = p.theta[32 * v + 4 * l8 + e];
+          float a0 = bf16lo(xw[e]), a1 = bf16hi(xw[e]);
+          if (p.m.kind != kNope) {
+            const float2 cs = phase_cs(static_cast<double>(pq) * th);
+            rot_pair(bf16lo(xw[e]), bf16hi(xw[e]), cs.x, cs.y, a0, a1);
+          }
+          if (p.bifocal) {
+            const float2 cd = phase_cs(static_cast<double>(dq) * th);
+            const float b0 = a0, b1 = a1;
+            rot_pair(b0, b1, cd.x, cd.y, a0, a1);
+          }
+          r0[e] = a0 * p.scale_log2;
+          r1[e] = a1 * p.scale_log2;
         }
+        Q0[gi][2 * v] = f2(r0[0], r0[1]);
+        Q0[gi][2 * v + 1] = f2(r0[2], r0[3]);
+        Q1[gi][2 * v] = f2(r1[0], r1[1]);
+        Q1[gi][2 * v + 1] = f2(r1[2], r1[3]);
       }
-      if (remote) {
-        // k_remote = R(-u theta) k_cache: (x0 c + x1 s, -x0 s + x1 c)
+    }
+  }
+
+  // phasors exp(i u theta) of the stream's two keys (u = u(k) for remote
+  // keys, u(t) for local ones), and the stage multiplier
+  // exp(i (64 - 64/G) theta) (no-carry case) in registers; a carry (G not
+  // dividing 64) takes the multiplier from shared memory
+  int a0[KPG], r0[KPG];
+  float2 PC[KPG][NJ], PS[KPG][NJ];
+  float2 MC[NJ], MS[NJ], MSN[NJ];
+  auto seed = [&](int kk, int u) {
 #pragma unroll
-        for (int pp = 0; pp < NP; ++pp) {
-          const float x0 = x[2 * pp], x1 = x[2 * pp + 1];
-          x[2 * pp] = fmaf(x0, ph[pp].x, x1 * ph[pp].y);
-          x[2 * pp + 1] = fmaf(x1, ph[pp].x, -x0 * ph[pp].y);
+    for (int j = 0; j < NJ; ++j) {
+      const float2 x = phase_cs(static_cast<double>(u) * p.theta[gpair(j, 0)]);
+      const float2 y = phase_cs(static_cast<double>(u) * p.theta[gpair(j, 1)]);
+      PC[kk][j] = f2(x.x, y.x);
+      PS[kk][j] = f2(x.y, y.y);
+    }
+  };
+#pragma unroll
+  for (int kk = 0; kk < KPG; ++kk) {
+    const int k = kb + ks + RS * kk;
+    a0[kk] = k / G;
+    r0[kk] = k - a0[kk] * G;
+    if (p.bifocal) seed(kk, k < p.k_local ? k - a0[kk] : u_t);
+  }
+  if (p.bifocal && SH::kMulInRegs) {
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+      const float2 x = mul_tab[gpair(j, 0)], y = mul_tab[gpair(j, 1)];
+      MC[j] = f2(x.x, y.x);
+      MS[j] = f2(x.y, y.y);
+      MSN[j] = f2(-x.y, -y.y);
+    }
+  }
+
+  float m_run[GRP], l_run[GRP];
+  float2 A0[GRP][NJ], A1[GRP][NJ];
+#pragma unroll
+  for (int gi = 0; gi < GRP; ++gi) {
+    m_run[gi] = -INFINITY;
+    l_run[gi] = 0.f;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) A0[gi][j] = A1[gi][j] = f2(0.f, 0.f);
+  }
+
+  bool ok = true;
+  for (int st = 0; st < nstage; ++st) {
+    const int slot = st % NS;
+    ok = __all_sync(0xffffffffu, mbar_wait(full + slot, (st / NS) & 1, abort_flag));
+    if (!ok) break;
+    const uint8_t* rows = smem + slot * L::kStageBytes + ks * L::kRowBytes;
+    uint4 kr[KPG][NV], vr[KPG][NV];
+#pragma unroll
+    for (int kk = 0; kk < KPG; ++kk)
+#pragma unroll
+      for (int v = 0; v < NV; ++v) {
+        kr[kk][v] = *reinterpret_cast<const uint4*>(rows + RS * kk * L::kRowBytes + v * 128 + l8 * 16);
+        vr[kk][v] = *reinterpret_cast<const uint4*>(rows + (kDecKeys + RS * kk) * L::kRowBytes + v * 128 + l8 * 16);
+      }
+    __syncwarp();
+    if (lane == 0) {
+      // the last warp to release the slot refills it with stage st + NS; the
+      // fences order every warp's reads of the slot before the copy's writes
+      __threadfence_block();
+      if (atomicAdd(released + slot, 1) == NW - 1) {
+        __threadfence_block();
+        released[slot] = 0;
+        if (st + NS < nstage) issue(st + NS);
+      }
+    }
+
+    const int k0 = kb + st * kDecKeys + ks;
+    float sc[KPG][GRP];
+#pragma unroll
+    for (int kk = 0; kk < KPG; ++kk) {
+      float2 X0[NJ], X1[NJ];
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        const uint4 w = kr[kk][j >> 1];
+        const uint32_t wa = (j & 1) ? w.z : w.x, wb = (j & 1) ? w.w : w.y;
+        X0[j] = f2(bf16lo(wa), bf16lo(wb));
+        X1[j] = f2(bf16hi(wa), bf16hi(wb));
+      }
+      if (p.bifocal) {
+        // R(-u theta) k_cache: (x0 c + x1 s, x1 c - x0 s)
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+          const float2 y0 = fma2(X1[j], PS[kk][j], mul2(X0[j], PC[kk][j]));
+          const float2 y1 = fma2(mul2(X0[j], kNeg), PS[kk][j], mul2(X1[j], PC[kk][j]));
+          X0[j] = y0;
+          X1[j] = y1;
         }
       }
-      float sc[GRP];
 #pragma unroll
       for (int gi = 0; gi < GRP; ++gi) {
-        float a = 0.f;
+        float2 acc0 = mul2(Q0[gi][0], X0[0]);
+        float2 acc1 = mul2(Q1[gi][0], X1[0]);
 #pragma unroll
-        for (int e = 0; e < NE; ++e) a = fmaf(qc[gi][e], x[e], a);
-        a += __shfl_xor_sync(0xffffffffu, a, 1);
-        a += __shfl_xor_sync(0xffffffffu, a, 2);
-        a += __shfl_xor_sync(0xffffffffu, a, 4);
-        sc[gi] = a * p.scale_log2;
-      }
-      if (valid) {
-        float vf[NE];
-#pragma unroll
-        for (int v = 0; v < NV; ++v) {
-          const uint32_t w[4] = {vv[v].x, vv[v].y, vv[v].z, vv[v].w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            vf[v * 8 + 2 * e] = bf16lo(w[e]);
-            vf[v * 8 + 2 * e + 1] = bf16hi(w[e]);
-          }
+        for (int j = 1; j < NJ; ++j) {
+          acc0 = fma2(Q0[gi][j], X0[j], acc0);
+          acc1 = fma2(Q1[gi][j], X1[j], acc1);
         }
+        const float2 a = __fadd2_rn(acc0, acc1);
+        sc[kk][gi] = a.x + a.y;
+      }
+    }
+#pragma unroll
+    for (int off = 1; off <= 4; off <<= 1)
+#pragma unroll
+      for (int kk = 0; kk < KPG; ++kk)
+#pragma unroll
+        for (int gi = 0; gi < GRP; ++gi) sc[kk][gi] += __shfl_xor_sync(gmask, sc[kk][gi], off);
+    bool vk[KPG];
+#pragma unroll
+    for (int kk = 0; kk < KPG; ++kk) vk[kk] = k0 + RS * kk < ke;
+#pragma unroll
+    for (int gi = 0; gi < GRP; ++gi) {
+      float mx = -INFINITY;
+#pragma unroll
+      for (int kk = 0; kk < KPG; ++kk) {
+        sc[kk][gi] = vk[kk] ? sc[kk][gi] : -INFINITY;
+        mx = fmaxf(mx, sc[kk][gi]);
+      }
+      if (mx > m_run[gi]) {
+        const float corr = ex2(m_run[gi] - mx);
+        l_run[gi] *= corr;
+        const float2 c2 = f2(corr, corr);
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+          A0[gi][j] = mul2(A0[gi][j], c2);
+          A1[gi][j] = mul2(A1[gi][j], c2);
+        }
+        m_run[gi] = mx;
+      }
+#pragma unroll
+      for (int kk = 0; kk < KPG; ++kk) {
+        sc[kk][gi] = vk[kk] ? ex2(sc[kk][gi] - m_run[gi]) : 0.f;
+        l_run[gi] += sc[kk][gi];
+      }
+    }
+#pragma unroll
+    for (int kk = 0; kk < KPG; ++kk) {
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        const uint4 w = vr[kk][j >> 1];
+        const uint32_t wa = (j & 1) ? w.z : w.x, wb = (j & 1) ? w.w : w.y;
+        const float2 V0 = f2(bf16lo(wa), bf16lo(wb));
+        const float2 V1 = f2(bf16hi(wa), bf16hi(wb));
 #pragma unroll
         for (int gi = 0; gi < GRP; ++gi) {
-          if (sc[gi] > m_run[gi]) {
-            const float corr = ex2(m_run[gi] - sc[gi]);
-            l_run[gi] *= corr;
-#pragma unroll
-            for (int e = 0; e < NE; ++e) acc[gi][e] *= corr;
-            m_run[gi] = sc[gi];
-          }
-          const float pr = ex2(sc[gi] - m_run[gi]);
-          l_run[gi] += pr;
-#pragma unroll
-          for (int e = 0; e < NE; ++e) acc[gi][e] = fmaf(pr, vf[e], acc[gi][e]);
-        }
-        // advance this stream's phasors to its next key (32 positions on)
-        const int kn = k + kDecKeys;
-        if (p.bifocal && kn < p.k_local && kn < ke) {
-          if (((st + 1) % kDecReseed) == 0) {
-            reseed(kn);
-          } else {
-            const bool a_step = (useed(kn) - useed(k)) == step_lo;
-#pragma unroll
-            for (int pp = 0; pp < NP; ++pp) {
-              const float2 mm = a_step ? mul_a[pp] : mul_b[pp];
-              const float c = ph[pp].x * mm.x - ph[pp].y * mm.y;
-              const float s = ph[pp].x * mm.y + ph[pp].y * mm.x;
-              ph[pp] = make_float2(c, s);
-            }
-          }
+          const float2 p2 = f2(sc[kk][gi], sc[kk][gi]);
+          A0[gi][j] = fma2(p2, V0, A0[gi][j]);
+          A1[gi][j] = fma2(p2, V1, A1[gi][j]);
         }
       }
     }
 
-    // ------------------------------------------- merge lane groups of a warp
+    // advance both keys' phasors to their keys of the next stage
+    if (p.bifocal) {
+      const bool reseed_now = ((st + 1) % kDecReseed) == 0;
+#pragma unroll
+      for (int kk = 0; kk < KPG; ++kk) {
+        const int k = k0 + RS * kk;
+        const int kn = k + kDecKeys;
+        r0[kk] += stage_r;
+        const bool carry = r0[kk] >= G;
+        if (carry) r0[kk] -= G;
+        a0[kk] += stage_q + (carry ? 1 : 0);
+        if (kn >= ke || k >= p.k_local) continue;        // no next key, or already at u(t)
+        if (kn >= p.k_local) {
+          seed(kk, u_t);                                  // entering the local window
+        } else if (reseed_now) {
+          seed(kk, kn - a0[kk]);
+        } else if (!carry && SH::kMulInRegs) {
+#pragma unroll
+          for (int j = 0; j < NJ; ++j) {
+            const float2 c = fma2(PC[kk][j], MC[j], mul2(PS[kk][j], MSN[j]));
+            const float2 sn = fma2(PC[kk][j], MS[j], mul2(PS[kk][j], MC[j]));
+            PC[kk][j] = c;
+            PS[kk][j] = sn;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < NJ; ++j) {
+            const int base = carry ? D / 2 : 0;
+            const float2 x = mul_tab[base + gpair(j, 0)], y = mul_tab[base + gpair(j, 1)];
+            const float2 mc = f2(x.x, y.x), ms = f2(x.y, y.y);
+            const float2 c = fma2(PC[kk][j], mc, mul2(PS[kk][j], mul2(ms, kNeg)));
+            const float2 sn = fma2(PC[kk][j], ms, mul2(PS[kk][j], mc));
+            PC[kk][j] = c;
+            PS[kk][j] = sn;
+          }
+        }
+      }
+    }
+  }
+
+  // --------------------------------------------- merge lane groups of a warp
+#pragma unroll
+  for (int gi = 0; gi < GRP; ++gi) {
+#pragma unroll
+    for (int off = 8; off <= 16; off <<= 1) {
+      const float mo = __shfl_xor_sync(0xffffffffu, m_run[gi], off);
+      const float lo = __shfl_xor_sync(0xffffffffu, l_run[gi], off);
+      const float M = fmaxf(m_run[gi], mo);
+      const float fa = (l_run[gi] > 0.f) ? ex2(m_run[gi] - M) : 0.f;
+      const float fb = (lo > 0.f) ? ex2(mo - M) : 0.f;
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        float2 o0, o1;
+        o0.x = __shfl_xor_sync(0xffffffffu, A0[gi][j].x, off);
+        o0.y = __shfl_xor_sync(0xffffffffu, A0[gi][j].y, off);
+        o1.x = __shfl_xor_sync(0xffffffffu, A1[gi][j].x, off);
+        o1.y = __shfl_xor_sync(0xffffffffu, A1[gi][j].y, off);
+        A0[gi][j] = fma2(A0[gi][j], f2(fa, fa), mul2(o0, f2(fb, fb)));
+        A1[gi][j] = fma2(A1[gi][j], f2(fa, fa), mul2(o1, f2(fb, fb)));
+      }
+      l_run[gi] = l_run[gi] * fa + lo * fb;
+      m_run[gi] = M;
+    }
+  }
+  // -------------------------------------------------- merge warps via smem
+  // (the ring is free: every issued stage was waited for above; after an
+  // abort the buffers may still be written by a late copy, and the results
+  // are void anyway)
+  __syncthreads();
+  float* red_o = reinterpret_cast<float*>(smem);                       // [NW][GRP][D]
+  float2* red_ml = reinterpret_cast<float2*>(smem + NW * GRP * D * 4);  // [NW][GRP]
+  if (j4 == 0) {
 #pragma unroll
     for (int gi = 0; gi < GRP; ++gi) {
+      float* dst = red_o + (warp * GRP + gi) * D;
 #pragma unroll
-      for (int off = 8; off <= 16; off <<= 1) {
-        const float mo = __shfl_xor_sync(0xffffffffu, m_run[gi], off);
-        const float lo = __shfl_xor_sync(0xffffffffu, l_run[gi], off);
-        const float M = fmaxf(m_run[gi], mo);
-        const float a = (l_run[gi] > 0.f) ? ex2(m_run[gi] - M) : 0.f;
-        const float c = (lo > 0.f) ? ex2(mo - M) : 0.f;
-#pragma unroll
-        for (int e = 0; e < NE; ++e) {
-          const float ao = __shfl_xor_sync(0xffffffffu, acc[gi][e], off);
-          acc[gi][e] = acc[gi][e] * a + ao * c;
-        }
-        l_run[gi] = l_run[gi] * a + lo * c;
-        m_run[gi] = M;
+      for (int j = 0; j < NJ; ++j) {
+        const int g0 = gpair(j, 0), g1 = gpair(j, 1);
+        dst[2 * g0] = A0[gi][j].x;
+        dst[2 * g0 + 1] = A1[gi][j].x;
+        dst[2 * g1] = A0[gi][j].y;
+        dst[2 * g1 + 1] = A1[gi][j].y;
+      }
+      if (l8 == 0) red_ml[warp * GRP + gi] = make_float2(m_run[gi], l_run[gi]);
+    }
+  }
+  __syncthreads();
+  for (int idx = tid; idx < GRP * D; idx += SH::kThreads) {
+    const int gi = idx / D, d = idx % D;
+    float M = -INFINITY;
+    for (int w = 0; w < NW; ++w) {
+      const float2 ml = red_ml[w * GRP + gi];
+      if (ml.y > 0.f) M = fmaxf(M, ml.x);
+    }
+    float o = 0.f, l = 0.f;
+    for (int w = 0; w < NW; ++w) {
+      const float2 ml = red_ml[w * GRP + gi];
+      if (ml.y > 0.f) {
+        const float f = ex2(ml.x - M);
+        o = fmaf(red_o[(w * GRP + gi) * D + d], f, o);
+        l = fmaf(ml.y, f, l);
       }
     }
-    // ------------------------------------------------ merge warps via smem
-    // (the stage ring is free: every stage issued was consumed above)
-    named_barrier_sync(1, kDecConsumerWarps * 32);
-    float* red_o = reinterpret_cast<float*>(smem);                       // [8][GRP][D]
-    float2* red_ml = reinterpret_cast<float2*>(smem + kDecConsumerWarps * GRP * D * 4);  // [8][GRP]
-    if (j4 == 0) {
-#pragma unroll
-      for (int gi = 0; gi < GRP; ++gi) {
-#pragma unroll
-        for (int e = 0; e < NE; ++e) red_o[(warp * GRP + gi) * D + 64 * (e >> 3) + 8 * l8 + (e & 7)] = acc[gi][e];
-        if (l8 == 0) red_ml[warp * GRP + gi] = make_float2(m_run[gi], l_run[gi]);
-      }
-    }
-    named_barrier_sync(1, kDecConsumerWarps * 32);
-    for (int idx = tid; idx < GRP * D; idx += kDecConsumerWarps * 32) {
+    const int hq = hkv * GRP + gi;
+    const size_t slot = (static_cast<size_t>(b) * p.Hq + hq) * p.nsplit + split;
+    p.part_o[slot * D + d] = o;
+    if (d == 0) p.part_ml[slot] = make_float2(M, l);
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const int prev = atomicAdd(p.counters + b * p.Hkv + hkv, 1);
+    *last_flag = (prev == p.nsplit - 1) ? 1 : 0;
+  }
+  __syncthreads();
+  if (*last_flag) {
+    // last CTA of this (batch, kv head): merge every split, in split order
+    __threadfence();
+    for (int idx = tid; idx < GRP * D; idx += SH::kThreads) {
       const int gi = idx / D, d = idx % D;
+      const int hq = hkv * GRP + gi;
+      const size_t base = (static_cast<size_t>(b) * p.Hq + hq) * p.nsplit;
       float M = -INFINITY;
-      for (int w = 0; w < kDecConsumerWarps; ++w) {
-        const float2 ml = red_ml[w * GRP + gi];
+      for (int sp = 0; sp < p.nsplit; ++sp) {
+        const float2 ml = __ldcg(p.part_ml + base + sp);
         if (ml.y > 0.f) M = fmaxf(M, ml.x);
       }
       float o = 0.f, l = 0.f;
-      for (int w = 0; w < kDecConsumerWarps; ++w) {
-        const float2 ml = red_ml[w * GRP + gi];
+      for (int sp = 0; sp < p.nsplit; ++sp) {
+        const float2 ml = __ldcg(p.part_ml + base + sp);
         if (ml.y > 0.f) {
           const float f = ex2(ml.x - M);
-          o = fmaf(red_o[(w * GRP + gi) * D + d], f, o);
+          o = fmaf(__ldcg(p.part_o + (base + sp) * D + d), f, o);
           l = fmaf(ml.y, f, l);
         }
       }
-      const int hq = hkv * GRP + gi;
-      const size_t slot = (static_cast<size_t>(b) * p.Hq + hq) * p.nsplit + split;
-      p.part_o[slot * D + d] = o;
-      if (d == 0) p.part_ml[slot] = make_float2(M, l);
+      p.out[(static_cast<size_t>(b) * p.Hq + hq) * D + d] = o / l;
+      if (d == 0) p.lse[static_cast<size_t>(b) * p.Hq + hq] = (M + __log2f(l)) * 0.69314718055994530942f;
     }
-    __threadfence();
-    named_barrier_sync(1, kDecConsumerWarps * 32);
-    if (tid == 0) {
-      const int prev = atomicAdd(p.counters + b * p.Hkv + hkv, 1);
-      *last_flag = (prev == p.nsplit - 1) ? 1 : 0;
-    }
-    named_barrier_sync(1, kDecConsumerWarps * 32);
-    if (*last_flag) {
-      // last CTA of this (batch, kv head): merge every split, in split order
-      __threadfence();
-      for (int idx = tid; idx < GRP * D; idx += kDecConsumerWarps * 32) {
-        const int gi = idx / D, d = idx % D;
-        const int hq = hkv * GRP + gi;
-        const size_t base = (static_cast<size_t>(b) * p.Hq + hq) * p.nsplit;
-        float M = -INFINITY;
-        for (int s = 0; s < p.nsplit; ++s) {
-          const float2 ml = __ldcg(p.part_ml + base + s);
-          if (ml.y > 0.f) M = fmaxf(M, ml.x);
-        }
-        float o = 0.f, l = 0.f;
-        for (int s = 0; s < p.nsplit; ++s) {
-          const float2 ml = __ldcg(p.part_ml + base + s);
-          if (ml.y > 0.f) {
-            const float f = ex2(ml.x - M);
-            o = fmaf(__ldcg(p.part_o + (base + s) * D + d), f, o);
-            l = fmaf(ml.y, f, l);
-          }
-        }
-        p.out[(static_cast<size_t>(b) * p.Hq + hq) * D + d] = o / l;
-        if (d == 0) p.lse[static_cast<size_t>(b) * p.Hq + hq] = (M + __log2f(l)) * 0.69314718055994530942f;
-      }
-      if (tid == 0) p.counters[b * p.Hkv + hkv] = 0;
-    }
-    (void)ok;
+    if (tid == 0) p.counters[b * p.Hkv + hkv] = 0;
   }
-  __syncthreads();
   if (*abort_flag) {
     const unsigned long long t0 = globaltimer_ns();
     while (globaltimer_ns() - t0 < 20000000ull) __nanosleep(100000);
   }
+  (void)ok;
 }
 
 }  // namespace ropeattn

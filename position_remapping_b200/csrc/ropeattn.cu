@@ -210,8 +210,10 @@ struct DecodeLayout {
   size_t off_o, off_ml, off_cnt, total;
 };
 
+// One CTA per SM is resident (shared-memory ring), so the grid is sized to
+// one wave: splits per (batch, kv head) = SMs / (B * Hkv), at least one.
 int decode_nsplit(long long B, long long keys, int Hkv) {
-  long long want = (2LL * sm_count() + Hkv * B - 1) / (Hkv * B);
+  long long want = static_cast<long long>(sm_count()) / (Hkv * B);
   long long cap = (keys + 255) / 256;
   long long ns = want < cap ? want : cap;
   return static_cast<int>(ns < 1 ? 1 : ns);
@@ -237,7 +239,7 @@ int launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodePara
     attr_err = cudaFuncSetAttribute(decode_kernel<D, GRP>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal);
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(decode)");
-  decode_kernel<D, GRP><<<grid, kDecThreads, L::kTotal, st>>>(tk, tv, dp);
+  decode_kernel<D, GRP><<<grid, DecodeShape<D, GRP>::kThreads, L::kTotal, st>>>(tk, tv, dp);
   CUDA_TRY(cudaGetLastError(), "decode launch");
   return ROPEATTN_OK;
 }
