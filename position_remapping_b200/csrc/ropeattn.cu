@@ -314,7 +314,7 @@ int prefill_impl(int stages, const void* q, const void* k, const void* v, float*
     if (!aligned16(q) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
       return fail(ROPEATTN_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
   }
-  if ((static_cast<long long>((S + kBM - 1) / kBM)) * Hq * B > 0x7fffffffLL)
+  if ((static_cast<long long>((S + kBlockRows - 1) / kBlockRows)) * Hq * B > 0x7fffffffLL)
     return fail(ROPEATTN_ERR_INVALID_ARG, "too many query tiles");
   rc = check_device();
   if (rc) return rc;
@@ -370,14 +370,14 @@ int prefill_impl(int stages, const void* q, const void* k, const void* v, float*
   pp.S = static_cast<int>(S);
   pp.Hq = Hq;
   pp.Hkv = Hkv;
-  pp.nqt = static_cast<int>((S + kBM - 1) / kBM);
+  pp.nqb = static_cast<int>((S + kBlockRows - 1) / kBlockRows);
   pp.kind = eff;
   pp.window = m.window;
   pp.w0 = m.w0;
   pp.scale_log2 = scale_log2(params, D);
-  const int grid = pp.nqt * Hq * static_cast<int>(B);
-  if (D == 128) return launch_prefill<128, 2>(tq, tk0, tk1, tv, pp, grid, st);
-  return launch_prefill<64, 4>(tq, tk0, tk1, tv, pp, grid, st);
+  const int grid = pp.nqb * Hq * static_cast<int>(B);
+  if (D == 128) return launch_prefill<128, 4>(tq, tk0, tk1, tv, pp, grid, st);
+  return launch_prefill<64, 8>(tq, tk0, tk1, tv, pp, grid, st);
 }
 
 }  // namespace
