@@ -39,6 +39,10 @@ METRIC = "128K bifocal-RoPE prefill TFLOP/s + decode µs/token; % of B200 roofli
 PREFILL = WORKLOADS["bifocal_prefill_s131072"]
 DECODE = WORKLOADS["bifocal_decode_n131072"]
 PEAK_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# oracle samples (query rows, kv heads): the reference arm's step (~4 s on 8
+# host cores) and the GPU arm's cpu_baseline (~10-15 s)
+REF_ROWS, REF_KV = 2, 1
+CPU_ROWS, CPU_KV = 16, 3
 
 
 def prefill_flops(w) -> float:
@@ -49,6 +53,26 @@ def prefill_flops(w) -> float:
 def decode_bytes(w) -> int:
     kv = 2 * w.B * w.S * w.Hkv * w.D * 2
     return kv + w.B * w.Hq * w.D * 2 + w.B * w.Hq * (w.D + 1) * 4
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Weak scaling: every rank runs its own independent draw of the workload."""
+    return seed + 17 * rank
+
+
+def max_over_ranks(values, world: int, device) -> list:
+    """Element-wise max of per-rank timings (the job is as slow as its
+    slowest rank). One all_reduce, taken by every rank in the same order."""
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_tflops(world: int, flops_per_step: float, steps: int, ms: float) -> float:
+    """Whole-job throughput: every rank's FLOPs over the slowest rank's time."""
+    return world * flops_per_step * steps / (ms / 1e3) / 1e12
 
 
 def load_peaks():
@@ -156,30 +180,40 @@ def oracle_rows(n_rows: int):
     return [min(S - 1, i * step + step // 2) for i in range(n_rows)]
 
 
-def oracle_step(n_rows: int, q, k, v, qd, kd, vd):
-    """Times the oracle on `n_rows` rows of the prefill (all heads) and on one
-    full decode. Returns (prefill TFLOP/s, decode us/token, seconds, sample)."""
+def oracle_step(n_rows: int, n_kv: int, q, k, v, qd, kd, vd):
+    """Times the oracle on a bounded sample of one step: `n_rows` evenly
+    spaced query rows of the prefill for the query heads of the first `n_kv`
+    kv heads (the oracle rotates every key of each kv head it is given, the
+    full 131072-token sequence, so L and G are those of the workload), and
+    one decode over the full cache for the query heads of the first `n_kv`
+    kv heads. Returns (prefill TFLOP/s, decode us per token of the sampled
+    heads scaled to all heads, seconds, sample description)."""
     import oracle as O
+    P, Dd = PREFILL, DECODE
+    hq_p = n_kv * (P.Hq // P.Hkv)
+    hq_d = n_kv * (Dd.Hq // Dd.Hkv)
     rows = oracle_rows(n_rows)
-    flops = sum(4.0 * PREFILL.D * (t + 1) * PREFILL.Hq for t in rows)
+    flops = sum(4.0 * P.D * (t + 1) * hq_p for t in rows)
+    qs, ks, vs = q[:, :, :hq_p], k[:, :, :n_kv], v[:, :, :n_kv]
+    qds, kds, vds = qd[:, :hq_d], kd[:, :, :n_kv], vd[:, :, :n_kv]
     t0 = time.perf_counter()
-    O.prefill(q, k, v, PREFILL.params, rows=rows, stage_bf16=True)
+    O.prefill(qs, ks, vs, P.params, rows=rows, stage_bf16=True)
     t1 = time.perf_counter()
-    O.decode(qd, kd, vd, DECODE.params)
+    O.decode(qds, kds, vds, Dd.params)
     t2 = time.perf_counter()
-    sample = (f"{n_rows} query rows (evenly spaced) x {PREFILL.Hq} heads of the {PREFILL.S}-token bifocal "
-              f"prefill, plus one full {DECODE.S}-key bifocal decode")
-    return flops / (t1 - t0) / 1e12, (t2 - t1) * 1e6, t2 - t0, sample
+    sample = (f"{n_rows} query rows (evenly spaced) x {hq_p} of {P.Hq} query heads ({n_kv} of {P.Hkv} kv heads) "
+              f"of the {P.S}-token bifocal prefill, plus a {Dd.S}-key bifocal decode of {hq_d} of {Dd.Hq} "
+              f"query heads (decode time scaled by {Dd.Hkv}/{n_kv})")
+    return flops / (t1 - t0) / 1e12, (t2 - t1) * 1e6 * Dd.Hkv / n_kv, t2 - t0, sample
 
 
 def run_reference(args):
     q, k, v = make_qkv(PREFILL.B, PREFILL.S, PREFILL.Hq, PREFILL.Hkv, PREFILL.D, PREFILL.seed)
     qd, kd, vd = make_qkv(DECODE.B, DECODE.S, DECODE.Hq, DECODE.Hkv, DECODE.D, DECODE.seed, q_len=1)
-    n_rows = 4
     vals, decs, secs = [], [], []
     sample = ""
     for i in range(args.warmup + args.steps):
-        tf, dus, s, sample = oracle_step(n_rows, q, k, v, qd, kd, vd)
+        tf, dus, s, sample = oracle_step(REF_ROWS, REF_KV, q, k, v, qd, kd, vd)
         if i >= args.warmup:
             vals.append(tf)
             decs.append(dus)
@@ -273,8 +307,8 @@ def main():
 
     # inputs resident in HBM (each rank its own seeded problem)
     P, Dd = PREFILL, DECODE
-    q, k, v = make_qkv(P.B, P.S, P.Hq, P.Hkv, P.D, P.seed + 17 * rank, device=dev)
-    qd, kd, vd = make_qkv(Dd.B, Dd.S, Dd.Hq, Dd.Hkv, Dd.D, Dd.seed + 17 * rank, device=dev, q_len=1)
+    q, k, v = make_qkv(P.B, P.S, P.Hq, P.Hkv, P.D, rank_seed(P.seed, rank), device=dev)
+    qd, kd, vd = make_qkv(Dd.B, Dd.S, Dd.Hq, Dd.Hkv, Dd.D, rank_seed(Dd.seed, rank), device=dev, q_len=1)
     out = torch.empty((P.B, P.S, P.Hq, P.D), dtype=torch.float32, device=dev)
     lse = torch.empty((P.B, P.Hq, P.S), dtype=torch.float32, device=dev)
     ws = torch.empty(ra.prefill_workspace_size(P.params, P.B, P.S, P.Hq, P.Hkv, P.D), dtype=torch.uint8, device=dev)
@@ -369,10 +403,8 @@ def main():
     e2e_dec_ms = sum(e[1].elapsed_time(e[2]) for e in e_evs)
     ra.status()
 
-    times = torch.tensor([total_ms, prep_ms, attn_ms, dec_ms, e2e_pre_ms, e2e_dec_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    total_ms, prep_ms, attn_ms, dec_ms, e2e_pre_ms, e2e_dec_ms = times.tolist()
+    total_ms, prep_ms, attn_ms, dec_ms, e2e_pre_ms, e2e_dec_ms = max_over_ranks(
+        [total_ms, prep_ms, attn_ms, dec_ms, e2e_pre_ms, e2e_dec_ms], world, dev)
 
     if rank != 0:
         if world > 1:
@@ -381,7 +413,7 @@ def main():
 
     K = args.steps
     flops = prefill_flops(P)
-    value = world * flops * K / ((prep_ms + attn_ms) / 1e3) / 1e12
+    value = job_tflops(world, flops, K, prep_ms + attn_ms)
     attn_tflops = flops * K / (attn_ms / 1e3) / 1e12
     dec_us = dec_ms * 1e3 / K
     dec_gbs = decode_bytes(Dd) * K / (dec_ms / 1e3) / 1e9
@@ -425,7 +457,7 @@ def main():
                             "algorithmic": f"{decode_bytes(Dd)} B per launch"},
         "clocks": clocks,
         "gpu_launches": 3 * K,
-        "e2e": {"value": world * flops * K / (e2e_pre_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": job_tflops(world, flops, K, e2e_pre_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "decode_us_per_token": e2e_dec_ms * 1e3 / K},
     }
@@ -434,7 +466,7 @@ def main():
         torch.cuda.synchronize()
         qc, kc, vc = make_qkv(P.B, P.S, P.Hq, P.Hkv, P.D, P.seed)
         qdc, kdc, vdc = make_qkv(Dd.B, Dd.S, Dd.Hq, Dd.Hkv, Dd.D, Dd.seed, q_len=1)
-        tf, dus, secs, sample = oracle_step(8, qc, kc, vc, qdc, kdc, vdc)
+        tf, dus, secs, sample = oracle_step(CPU_ROWS, CPU_KV, qc, kc, vc, qdc, kdc, vdc)
         line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
                                 "sample": sample, "decode_us_per_token": dus, "seconds": secs}
     print(json.dumps(line), flush=True)

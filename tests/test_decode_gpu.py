@@ -23,6 +23,9 @@ SMALL = [
     ("bifocal_g3_grp4", 1, 9000, 8, 2, 128, MapParams(O.BIFOCAL, rope_base=1e4, w0=1000, w_pretrained=3001)),
     ("bifocal_w0_0_d64", 1, 4097, 4, 1, 64, MapParams(O.BIFOCAL, rope_base=1e4, w0=0, w_pretrained=1024)),
     ("bifocal_inside_window", 1, 500, 4, 2, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=100, w_pretrained=512)),
+    ("bifocal_g4_d64_grp4", 2, 4097, 8, 2, 64, MapParams(O.BIFOCAL, rope_base=1e4, w0=300, w_pretrained=1100)),
+    ("bifocal_g8_d128", 1, 8000, 4, 4, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=2048, w_pretrained=1000)),
+    ("bifocal_g2_edge_local", 1, 3000, 2, 1, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=2900, w_pretrained=1500)),
 ]
 
 
