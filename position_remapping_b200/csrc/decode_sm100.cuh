@@ -3,21 +3,34 @@
 // Split-KV: CTA (split, kv head, batch) owns a contiguous key range of one KV
 // head; the grid is one wave (one CTA per SM). The range streams through a
 // shared-memory ring by TMA, 64 keys per stage (no swizzle, no multicast).
-// All 8 warps consume; the last warp to release a slot issues the copy of the
-// stage that reuses it, so no thread polls.
+// A lane group of 8 lanes holds D/8 dimensions of one key and of the query:
+// 16 warps take one key per group per stage, or 8 warps two keys when the
+// GQA group is too large for 128 registers a thread. The last warp to
+// release a slot issues the copy of the stage that reuses it; no thread polls.
 //
 // Scores: the query is rotated once to its position p(n-1) in fp32 and
-// prescaled by softmax_scale * log2(e). For the bifocal map the query is then
-// corrected by Delta q = f(n-1) - (n-1) (Eq. 5-6), and every cached key k is
-// read through a rotation R(-u theta): remote keys ((n-1) - k > w0) use
-// u = u(k) = k - floor(k/G), i.e. the correction Delta k of Eq. 6; local keys
-// use u = u(n-1), which turns q_remote . R(Delta q) k_cache back into
-// q_local . k_cache exactly (R_a R_b = R_{a+b}), so one query view serves both
-// windows. Each lane carries the phasors exp(i u theta) of its pairs and
-// advances them by one complex multiply per stage (a key moves 64 positions);
-// they are re-seeded exactly (argument reduced in double) every 16 stages.
-// Packed fp32x2 FMAs carry the rotation, the dot products and the
-// accumulation. Each lane group of 8 lanes takes two keys per stage.
+// prescaled by softmax_scale * log2(e). For the bifocal map a remote key k
+// ((n-1) - k > w0) is read through the correction of Eq. 6: with
+// u(k) = k - f(k) = k - floor(k/G),
+//   score = q_remote . R(-u(k)) k_cache,   q_remote = R(Delta q) q_local,
+// and a local key through q_local . k_cache. R(-u(k)) is applied one of two
+// ways (template parameter ROT):
+//  * stage table (G divides 64, one key per group): every stage starts at a
+//    multiple of G, so u(k0 + r) = u(k0) + d(r) with d(r) = r - floor(r/G)
+//    the same in every stage. The group of row r keeps R(d(r)) q_remote, and
+//    all keys of a stage share R(-u(k0)), whose (cos, sin) table is computed
+//    once per stage, NS stages ahead, by one warp (warp st mod 16 while it
+//    works on stage st); the slot's barrier counts that warp's arrival with
+//    the copy's. A group switches to q_local when its keys become local.
+//  * phasor recurrence (any G): each lane carries exp(i u theta) for its
+//    pairs and advances it by one complex multiply per stage, re-seeded
+//    exactly every 16 stages; local keys use u(n-1), which turns
+//    q_remote . R(Delta q) k_cache back into q_local . k_cache, so one query
+//    view serves both windows.
+// Every angle is an integer position times theta_i, taken from theta_i's
+// fraction of a turn in 64-bit fixed point, so it is exact modulo a turn
+// before the fp32 sincospi. Packed fp32x2 FMAs carry the rotation, the dot
+// products and the accumulation.
 //
 // Each lane group keeps an online softmax per query head of the GQA group;
 // the CTA merges its groups and warps, writes (O, m, l) for its split, and the
@@ -29,23 +42,18 @@
 
 namespace ropeattn {
 
-constexpr int kDecKeys = 64;         // keys per stage: one per lane group of 16 warps
+constexpr int kDecKeys = 64;         // keys per stage
 constexpr int kDecReseed = 16;       // stages between exact phasor re-seeds
 
-// Warps per CTA and keys per lane group per stage: 16 warps x 1 key (more
-// warps to hide latency) or 8 warps x 2 keys (more independent work per
-// warp); a stage is always 64 keys. The stage multipliers of the phasor
-// recurrence are held in registers with 2 keys per group, else read from
-// shared memory each stage.
-#ifndef ROPEATTN_DECODE_KPG
-#define ROPEATTN_DECODE_KPG 1
-#endif
+// how remote keys are rotated
+enum DecodeRot : int { kRotNone = 0, kRotTable = 1, kRotPhasor = 2 };
+
 template <int D, int GRP>
 struct DecodeShape {
-  static constexpr int kKeysPerGroup = (GRP * D <= 256) ? ROPEATTN_DECODE_KPG : 2;
+  static constexpr int kKeysPerGroup = (GRP * D <= 256) ? 1 : 2;
   static constexpr int kWarps = 16 / kKeysPerGroup;
   static constexpr int kThreads = kWarps * 32;
-  static constexpr bool kMulInRegs = kKeysPerGroup == 2;
+  static constexpr bool kMulInRegs = kKeysPerGroup == 2;   // phasor multipliers in registers
 };
 
 struct DecodeParams {
@@ -62,16 +70,18 @@ struct DecodeParams {
   int bifocal;             // 1 when keys are read through the correction rotation
   PosMap m;
   float scale_log2;
-  double theta[kMaxPairs];
+  unsigned long long turns[kMaxPairs];  // theta_i / (2 pi) mod 1, in units of 2^-64
 };
 
-// (cos, sin) of phase * theta, with the argument reduced modulo 2*pi in double
-// before the fp32 sincos.
-__device__ __forceinline__ float2 phase_cs(double phase) {
-  const double two_pi = 6.283185307179586476925286766559;
-  const double r = phase - two_pi * rint(phase * (1.0 / two_pi));
+// (cos, sin) of u * theta for an integer position u, with theta given as its
+// fraction of a turn in 64-bit fixed point: the product modulo 2^64 is the
+// angle modulo one turn, exactly; its top 32 bits, as a signed value, are the
+// angle in half-turns in [-1, 1) for sincospi.
+__device__ __forceinline__ float2 turn_cs(int u, unsigned long long turn) {
+  const unsigned long long ph = turn * static_cast<unsigned long long>(static_cast<long long>(u));
+  const float x = static_cast<float>(static_cast<int>(ph >> 32)) * 4.656612873077392578125e-10f;  // 2^-31
   float s, c;
-  sincosf(static_cast<float>(r), &s, &c);
+  sincospif(x, &s, &c);
   return make_float2(c, s);
 }
 
@@ -81,8 +91,10 @@ struct DecodeSmem {
   static constexpr int kRowBytes = D * 2;
   static constexpr int kStageBytes = 2 * kDecKeys * kRowBytes;  // K then V
   static constexpr int kRing = kStages * kStageBytes;
-  static constexpr int kMul = kRing;                             // [2][D/2] float2 stage multipliers
-  static constexpr int kBar = kMul + D * 8;                      // full[] mbarriers
+  static constexpr int kMul = kRing;                             // [2][D/2] float2 phasor stage multipliers
+  static constexpr int kTab = kMul + D * 8;                      // [2 kStages][D/4] float4 stage tables
+  static constexpr int kQloc = kTab + 2 * kStages * D * 4;       // [GRP][D/4] float4 local query view
+  static constexpr int kBar = kQloc + 2048;                      // full[] mbarriers (GRP * D <= 512)
   static constexpr int kCnt = kBar + kStages * 8;                // release counters per slot
   static constexpr int kMisc = kCnt + kStages * 4;               // abort flag, last flag
   static constexpr int kTotal = kMisc + 16;
@@ -94,7 +106,7 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 neg2(float2 a) { return make_float2(-a.x, -a.y); }
 
-template <int D, int GRP>
+template <int D, int GRP, int ROT>
 __global__ void __launch_bounds__(DecodeShape<D, GRP>::kThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const DecodeParams p) {
@@ -106,9 +118,14 @@ __global__ void __launch_bounds__(DecodeShape<D, GRP>::kThreads, 1)
   constexpr int NJ = 2 * NV;              // pair-pairs per lane (two rotation pairs each)
   constexpr int KPG = SH::kKeysPerGroup;  // keys per lane group per stage
   constexpr int RS = kDecKeys / KPG;      // row stride between a group's keys in a stage
+  constexpr int NPP = D / 4;              // pair-pairs per row
+  static_assert(GRP * D <= 512, "local query view table holds GRP * D <= 512 values");
+  static_assert(ROT != kRotTable || KPG == 1, "stage tables need one key per group");
 
   extern __shared__ __align__(128) uint8_t smem[];
   float2* mul_tab = reinterpret_cast<float2*>(smem + L::kMul);   // [carry][pair] (cos, sin)
+  float4* stab = reinterpret_cast<float4*>(smem + L::kTab);      // [slot][pair-pair] (c0, c1, s0, s1)
+  float4* qloc = reinterpret_cast<float4*>(smem + L::kQloc);     // [gi][pair-pair] (q0 x2, q1 x2)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBar);
   int* released = reinterpret_cast<int*>(smem + L::kCnt);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc);
@@ -126,7 +143,27 @@ __global__ void __launch_bounds__(DecodeShape<D, GRP>::kThreads, 1)
   const int nstage = (ke - kb + kDecKeys - 1) / kDecKeys;
   const int G = p.m.G;
   const int stage_q = kDecKeys / G, stage_r = kDecKeys - stage_q * G;
+  const int t = p.n - 1;                // query position index
 
+  // Stage table of stage st (table slot st mod 2 NS): (cos, sin) of
+  // u(k0) theta for every pair, k0 the stage's first key. The entry of
+  // pair-pair pp (pairs 2pp, 2pp+1) = (c0, c1, s0, s1) sits at
+  // 16 (pp / 16) + 8 (pp % 2) + (pp % 16) / 2, so the 8 lanes of a group read
+  // 128 consecutive bytes. One warp writes it, then arrives on the stage's
+  // ring barrier.
+  auto tab_pos = [](int pp) { return 16 * (pp >> 4) + 8 * (pp & 1) + ((pp & 15) >> 1); };
+  auto fill_table = [&](int st) {
+    const int k0 = kb + st * kDecKeys;
+    const int u0 = k0 - k0 / G;
+    float4* tab = stab + (st % (2 * NS)) * NPP;
+    for (int pp = lane; pp < NPP; pp += 32) {
+      const float2 x = turn_cs(u0, p.turns[2 * pp]);
+      const float2 y = turn_cs(u0, p.turns[2 * pp + 1]);
+      tab[tab_pos(pp)] = make_float4(x.x, y.x, x.y, y.y);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(full + st % NS);
+  };
   auto issue = [&](int st) {  // copy stage st (K rows then V rows) into its slot
     const int slot = st % NS;
     uint8_t* dst = smem + slot * L::kStageBytes;
@@ -135,8 +172,10 @@ __global__ void __launch_bounds__(DecodeShape<D, GRP>::kThreads, 1)
     tma_load_4d(dst + kDecKeys * L::kRowBytes, &tmV, full + slot, 0, hkv, kb + st * kDecKeys, b);
   };
   if (tid == 0) {
+    // the copy's arrival, plus the stage table's
+    const uint32_t arrivals = ROT == kRotTable ? 2 : 1;
     for (int i = 0; i < NS; ++i) {
-      mbar_init(full + i, 1);
+      mbar_init(full + i, arrivals);
       released[i] = 0;
     }
     *abort_flag = 0;
@@ -146,97 +185,120 @@ __global__ void __launch_bounds__(DecodeShape<D, GRP>::kThreads, 1)
     tma_prefetch_desc(&tmV);
     for (int st = 0; st < NS && st < nstage; ++st) issue(st);
   }
-  if (p.bifocal) {
+  if constexpr (ROT == kRotPhasor) {
     // per pair: (cos, sin) of the stage advance of u without and with a
     // group-boundary carry: 64 - 64/G and 63 - 64/G positions
     for (int i = tid; i < D / 2; i += SH::kThreads) {
-      const double du = kDecKeys - stage_q;
-      mul_tab[i] = phase_cs(du * p.theta[i]);
-      mul_tab[D / 2 + i] = phase_cs((du - 1.0) * p.theta[i]);
+      const int du = kDecKeys - stage_q;
+      mul_tab[i] = turn_cs(du, p.turns[i]);
+      mul_tab[D / 2 + i] = turn_cs(du - 1, p.turns[i]);
     }
   }
+  // local query view R(p(t)) q prescaled by softmax scale * log2(e): entry
+  // (q0 of pairs 2pp, 2pp+1; q1 of pairs 2pp, 2pp+1) per pair-pair
+  if (tid >= 32 && tid < 32 + GRP * NPP) {
+    const int i = tid - 32, gi = i / NPP, pp = i % NPP;
+    const int hq = hkv * GRP + gi;
+    const uint2 xq = __ldg(reinterpret_cast<const uint2*>(p.q + (static_cast<size_t>(b) * p.Hq + hq) * D) + pp);
+    const int pq = pos_primary(p.m, t);
+    const uint32_t xw[2] = {xq.x, xq.y};
+    float r0[2], r1[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      float a0 = bf16lo(xw[e]), a1 = bf16hi(xw[e]);
+      if (p.m.kind != kNope) {
+        const float2 cs = turn_cs(pq, p.turns[2 * pp + e]);
+        rot_pair(bf16lo(xw[e]), bf16hi(xw[e]), cs.x, cs.y, a0, a1);
+      }
+      r0[e] = a0 * p.scale_log2;
+      r1[e] = a1 * p.scale_log2;
+    }
+    qloc[gi * NPP + pp] = make_float4(r0[0], r0[1], r1[0], r1[1]);
+  }
   __syncthreads();
+  if constexpr (ROT == kRotTable) {
+    if (warp < NS && warp < nstage) fill_table(warp);
+  }
 
   const int j4 = lane >> 3;             // lane group within the warp
   const int l8 = lane & 7;              // lane within the group
   const int ks = warp * 4 + j4;         // key stream: rows ks + RS * kk of every stage
   const unsigned gmask = 0xFFu << (8 * j4);
-  const int t = p.n - 1;                // query position index
   const int u_t = t - t / G;            // u of the query: local keys are read at u(t)
   // Lane pair-pair j holds rotation pairs c = 0, 1 at word 2(j%2)+c of the
-  // 16-byte vector j/2: global pair 32 (j/2) + 4 l8 + 2 (j%2) + c.
+  // 16-byte vector j/2: global pair 32 (j/2) + 4 l8 + 2 (j%2) + c, i.e.
+  // global pair-pair 16 (j/2) + 2 l8 + (j%2).
   auto gpair = [&](int j, int c) { return 32 * (j >> 1) + 4 * l8 + 2 * (j & 1) + c; };
+  auto gpp = [&](int j) { return 16 * (j >> 1) + 2 * l8 + (j & 1); };
   const float2 kNeg = f2(-1.f, -1.f);
 
-  // query, prescaled by softmax scale * log2(e): rotated to p(t) and, for
-  // the bifocal map, corrected by Delta q on top (the remote view, Eq. 5-6)
   float2 Q0[GRP][NJ], Q1[GRP][NJ];
-  {
-    const int pq = pos_primary(p.m, t);
-    const int dq = pos_remote(p.m, t) - t;
+  auto load_local = [&]() {
 #pragma unroll
-    for (int gi = 0; gi < GRP; ++gi) {
-      const int hq = hkv * GRP + gi;
-      const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(b) * p.Hq + hq) * D);
+    for (int gi = 0; gi < GRP; ++gi)
 #pragma unroll
-      for (int v = 0; v < NV; ++v) {
-        const uint4 xq = __ldg(qsrc + v * 8 + l8);
-        const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
-        float r0[4], r1[4];
+      for (int j = 0; j < NJ; ++j) {
+        const float4 x = qloc[gi * NPP + gpp(j)];
+        Q0[gi][j] = f2(x.x, x.y);
+        Q1[gi][j] = f2(x.z, x.w);
+      }
+  };
+  // rotate the query view by +shift positions
+  auto rotate_query = [&](int shift) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const double th = p.theta[32 * v + 4 * l8 + e];
-          float a0 = bf16lo(xw[e]), a1 = bf16hi(xw[e]);
-          if (p.m.kind != kNope) {
-            const float2 cs = phase_cs(static_cast<double>(pq) * th);
-            rot_pair(bf16lo(xw[e]), bf16hi(xw[e]), cs.x, cs.y, a0, a1);
-          }
-          if (p.bifocal) {
-            const float2 cd = phase_cs(static_cast<double>(dq) * th);
-            const float b0 = a0, b1 = a1;
-            rot_pair(b0, b1, cd.x, cd.y, a0, a1);
-          }
-          r0[e] = a0 * p.scale_log2;
-          r1[e] = a1 * p.scale_log2;
-        }
-        Q0[gi][2 * v] = f2(r0[0], r0[1]);
-        Q0[gi][2 * v + 1] = f2(r0[2], r0[3]);
-        Q1[gi][2 * v] = f2(r1[0], r1[1]);
-        Q1[gi][2 * v + 1] = f2(r1[2], r1[3]);
+    for (int j = 0; j < NJ; ++j) {
+      const float2 x = turn_cs(shift, p.turns[gpair(j, 0)]);
+      const float2 y = turn_cs(shift, p.turns[gpair(j, 1)]);
+      const float2 C = f2(x.x, y.x), Sn = f2(x.y, y.y);
+#pragma unroll
+      for (int gi = 0; gi < GRP; ++gi) {
+        // (a0 c - a1 s, a0 s + a1 c)
+        const float2 y0 = fma2(mul2(Q1[gi][j], kNeg), Sn, mul2(Q0[gi][j], C));
+        const float2 y1 = fma2(Q0[gi][j], Sn, mul2(Q1[gi][j], C));
+        Q0[gi][j] = y0;
+        Q1[gi][j] = y1;
       }
     }
+  };
+  load_local();
+  const int dq = pos_remote(p.m, t) - t;   // Delta q (Eq. 5)
+  bool q_remote = false;                   // stage-table view: query currently R(d(ks)) q_remote
+  if constexpr (ROT == kRotPhasor) rotate_query(dq);
+  if constexpr (ROT == kRotTable) {
+    q_remote = kb + ks < p.k_local;
+    if (q_remote) rotate_query(dq + (ks - ks / G));
   }
 
-  // phasors exp(i u theta) of the stream's two keys (u = u(k) for remote
-  // keys, u(t) for local ones), and the stage multiplier
-  // exp(i (64 - 64/G) theta) (no-carry case) in registers; a carry (G not
-  // dividing 64) takes the multiplier from shared memory
+  // phasor recurrence state: exp(i u theta) of the stream's keys (u = u(k)
+  // for remote keys, u(t) for local ones) and the no-carry stage multiplier
   int a0[KPG], r0[KPG];
   float2 PC[KPG][NJ], PS[KPG][NJ];
   float2 MC[NJ], MS[NJ], MSN[NJ];
   auto seed = [&](int kk, int u) {
 #pragma unroll
     for (int j = 0; j < NJ; ++j) {
-      const float2 x = phase_cs(static_cast<double>(u) * p.theta[gpair(j, 0)]);
-      const float2 y = phase_cs(static_cast<double>(u) * p.theta[gpair(j, 1)]);
+      const float2 x = turn_cs(u, p.turns[gpair(j, 0)]);
+      const float2 y = turn_cs(u, p.turns[gpair(j, 1)]);
       PC[kk][j] = f2(x.x, y.x);
       PS[kk][j] = f2(x.y, y.y);
     }
   };
+  if constexpr (ROT == kRotPhasor) {
 #pragma unroll
-  for (int kk = 0; kk < KPG; ++kk) {
-    const int k = kb + ks + RS * kk;
-    a0[kk] = k / G;
-    r0[kk] = k - a0[kk] * G;
-    if (p.bifocal) seed(kk, k < p.k_local ? k - a0[kk] : u_t);
-  }
-  if (p.bifocal && SH::kMulInRegs) {
+    for (int kk = 0; kk < KPG; ++kk) {
+      const int k = kb + ks + RS * kk;
+      a0[kk] = k / G;
+      r0[kk] = k - a0[kk] * G;
+      seed(kk, k < p.k_local ? k - a0[kk] : u_t);
+    }
+    if constexpr (SH::kMulInRegs) {
 #pragma unroll
-    for (int j = 0; j < NJ; ++j) {
-      const float2 x = mul_tab[gpair(j, 0)], y = mul_tab[gpair(j, 1)];
-      MC[j] = f2(x.x, y.x);
-      MS[j] = f2(x.y, y.y);
-      MSN[j] = f2(-x.y, -y.y);
+      for (int j = 0; j < NJ; ++j) {
+        const float2 x = mul_tab[gpair(j, 0)], y = mul_tab[gpair(j, 1)];
+        MC[j] = f2(x.x, y.x);
+        MS[j] = f2(x.y, y.y);
+        MSN[j] = f2(-x.y, -y.y);
+      }
     }
   }
 
@@ -251,12 +313,16 @@ __global__ void __launch_bounds__(DecodeShape<D, GRP>::kThreads, 1)
   }
 
   bool ok = true;
+  int slot = 0, tslot = 0;
+  uint32_t phase = 0;
   for (int st = 0; st < nstage; ++st) {
-    const int slot = st % NS;
-    ok = __all_sync(0xffffffffu, mbar_wait(full + slot, (st / NS) & 1, abort_flag));
+    ok = __all_sync(0xffffffffu, mbar_wait(full + slot, phase, abort_flag));
     if (!ok) break;
+    const int k0 = kb + st * kDecKeys + ks;
     const uint8_t* rows = smem + slot * L::kStageBytes + ks * L::kRowBytes;
     uint4 kr[KPG][NV], vr[KPG][NV];
+    float4 tb[NJ];
+    const bool rem_t = ROT == kRotTable && k0 < p.k_local;
 #pragma unroll
     for (int kk = 0; kk < KPG; ++kk)
 #pragma unroll
@@ -264,6 +330,13 @@ __global__ void __launch_bounds__(DecodeShape<D, GRP>::kThreads, 1)
         kr[kk][v] = *reinterpret_cast<const uint4*>(rows + RS * kk * L::kRowBytes + v * 128 + l8 * 16);
         vr[kk][v] = *reinterpret_cast<const uint4*>(rows + (kDecKeys + RS * kk) * L::kRowBytes + v * 128 + l8 * 16);
       }
+    if constexpr (ROT == kRotTable) {
+      if (rem_t) {
+        const float4* tt = stab + tslot * NPP;
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) tb[j] = tt[16 * (j >> 1) + 8 * (j & 1) + l8];
+      }
+    }
     __syncwarp();
     if (lane == 0) {
       // the last warp to release the slot refills it with stage st + NS; the
@@ -276,7 +349,6 @@ __global__ void __launch_bounds__(DecodeShape<D, GRP>::kThreads, 1)
       }
     }
 
-    const int k0 = kb + st * kDecKeys + ks;
     float sc[KPG][GRP];
 #pragma unroll
     for (int kk = 0; kk < KPG; ++kk) {
@@ -288,7 +360,7 @@ __global__ void __launch_bounds__(DecodeShape<D, GRP>::kThreads, 1)
         X0[j] = f2(bf16lo(wa), bf16lo(wb));
         X1[j] = f2(bf16hi(wa), bf16hi(wb));
       }
-      if (p.bifocal) {
+      if constexpr (ROT == kRotPhasor) {
         // R(-u theta) k_cache: (x0 c + x1 s, x1 c - x0 s)
 #pragma unroll
         for (int j = 0; j < NJ; ++j) {
@@ -296,6 +368,23 @@ __global__ void __launch_bounds__(DecodeShape<D, GRP>::kThreads, 1)
           const float2 y1 = fma2(mul2(X0[j], kNeg), PS[kk][j], mul2(X1[j], PC[kk][j]));
           X0[j] = y0;
           X1[j] = y1;
+        }
+      }
+      if constexpr (ROT == kRotTable) {
+        if (rem_t) {
+          // R(-u(k0) theta) k_cache with the stage's shared table
+#pragma unroll
+          for (int j = 0; j < NJ; ++j) {
+            const float2 C = f2(tb[j].x, tb[j].y), Sn = f2(tb[j].z, tb[j].w);
+            const float2 y0 = fma2(X1[j], Sn, mul2(X0[j], C));
+            const float2 y1 = fma2(neg2(X0[j]), Sn, mul2(X1[j], C));
+            X0[j] = y0;
+            X1[j] = y1;
+          }
+        } else if (q_remote) {
+          // this stream's keys became local: exact-position query view
+          load_local();
+          q_remote = false;
         }
       }
 #pragma unroll
@@ -362,8 +451,8 @@ __global__ void __launch_bounds__(DecodeShape<D, GRP>::kThreads, 1)
       }
     }
 
-    // advance both keys' phasors to their keys of the next stage
-    if (p.bifocal) {
+    // advance the phasors to the keys of the next stage
+    if constexpr (ROT == kRotPhasor) {
       const bool reseed_now = ((st + 1) % kDecReseed) == 0;
 #pragma unroll
       for (int kk = 0; kk < KPG; ++kk) {
@@ -399,6 +488,15 @@ __global__ void __launch_bounds__(DecodeShape<D, GRP>::kThreads, 1)
           }
         }
       }
+    }
+    // the table of the stage that reuses the slot, by one warp in turn
+    if constexpr (ROT == kRotTable) {
+      if (warp == st % NW && st + NS < nstage) fill_table(st + NS);
+    }
+    if (++tslot == 2 * NS) tslot = 0;
+    if (++slot == NS) {
+      slot = 0;
+      phase ^= 1u;
     }
   }
 
@@ -466,9 +564,9 @@ __global__ void __launch_bounds__(DecodeShape<D, GRP>::kThreads, 1)
       }
     }
     const int hq = hkv * GRP + gi;
-    const size_t slot = (static_cast<size_t>(b) * p.Hq + hq) * p.nsplit + split;
-    p.part_o[slot * D + d] = o;
-    if (d == 0) p.part_ml[slot] = make_float2(M, l);
+    const size_t pslot = (static_cast<size_t>(b) * p.Hq + hq) * p.nsplit + split;
+    p.part_o[pslot * D + d] = o;
+    if (d == 0) p.part_ml[pslot] = make_float2(M, l);
   }
   __threadfence();
   __syncthreads();

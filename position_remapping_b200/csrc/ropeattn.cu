@@ -158,6 +158,20 @@ void fill_theta(const ropeattn_params* p, int D, double* theta) {
   for (int i = 0; i < D / 2; ++i) theta[i] = std::pow(p->rope_base, -2.0 * i / D) / s;
 }
 
+// theta_i / (2 pi) modulo 1 in 64-bit fixed point (units of 2^-64 turn),
+// computed in long double from the double theta_i of fill_theta.
+void fill_turns(const ropeattn_params* p, int D, unsigned long long* turns) {
+  double theta[kMaxPairs];
+  fill_theta(p, D, theta);
+  const long double two_pi = 2.0L * std::acos(-1.0L);
+  for (int i = 0; i < D / 2; ++i) {
+    long double f = std::fmod(static_cast<long double>(theta[i]) / two_pi, 1.0L);
+    if (f < 0) f += 1.0L;
+    const long double r = std::floor(std::ldexp(f, 64) + 0.5L);
+    turns[i] = r >= 18446744073709551616.0L ? 0ull : static_cast<unsigned long long>(r);   // 2^64 wraps to 0
+  }
+}
+
 float scale_log2(const ropeattn_params* p, int D) {
   const double sc = p->softmax_scale > 0.0f ? static_cast<double>(p->softmax_scale) : 1.0 / std::sqrt(double(D));
   return static_cast<float>(sc * 1.4426950408889634074);
@@ -230,18 +244,31 @@ DecodeLayout decode_layout(long long B, long long keys, int Hq, int Hkv, int D) 
   return L;
 }
 
-template <int D, int GRP>
-int launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& dp, dim3 grid, cudaStream_t st) {
+template <int D, int GRP, int ROT>
+int launch_decode_rot(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& dp, dim3 grid,
+                      cudaStream_t st) {
   using L = DecodeSmem<D>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(decode_kernel<D, GRP>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal);
+    attr_err = cudaFuncSetAttribute(decode_kernel<D, GRP, ROT>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal);
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(decode)");
-  decode_kernel<D, GRP><<<grid, DecodeShape<D, GRP>::kThreads, L::kTotal, st>>>(tk, tv, dp);
+  decode_kernel<D, GRP, ROT><<<grid, DecodeShape<D, GRP>::kThreads, L::kTotal, st>>>(tk, tv, dp);
   CUDA_TRY(cudaGetLastError(), "decode launch");
   return ROPEATTN_OK;
+}
+
+// Rotation of remote keys: none (no bifocal map), a shared per-stage table
+// when one key per lane group and G divides the 64-key stage, else the
+// per-lane phasor recurrence.
+template <int D, int GRP>
+int launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& dp, dim3 grid, cudaStream_t st) {
+  if (!dp.bifocal) return launch_decode_rot<D, GRP, kRotNone>(tk, tv, dp, grid, st);
+  if constexpr (DecodeShape<D, GRP>::kKeysPerGroup == 1) {
+    if (kDecKeys % dp.m.G == 0) return launch_decode_rot<D, GRP, kRotTable>(tk, tv, dp, grid, st);
+  }
+  return launch_decode_rot<D, GRP, kRotPhasor>(tk, tv, dp, grid, st);
 }
 
 }  // namespace
@@ -460,7 +487,7 @@ int ropeattn_decode(const void* q, const void* k_cache, const void* v_cache, flo
   m.kind = eff;
   dp.m = m;
   dp.scale_log2 = scale_log2(params, D);
-  fill_theta(params, D, dp.theta);
+  fill_turns(params, D, dp.turns);
 
   CUtensorMap tk, tv;
   if ((rc = make_map(&tk, k_cache, D, Hkv, n, B, D, kDecKeys, false))) return rc;
