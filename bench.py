@@ -447,12 +447,12 @@ def main():
         "decode_us_per_token": dec_us,
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": tpeak, "unit": "TFLOP/s",
                      "frac": attn_tflops / tpeak, "traffic": tr_p,
-                     "kernel": "prefill_kernel<128,2> (attention)",
+                     "kernel": "prefill_kernel<128,4> (attention; D=128, 4 ring slots)",
                      "peak_source": f"{peak_src} bf16_tflops_sustained",
                      "algorithmic": f"{flops:.6g} FLOP per launch"},
         "roofline_decode": {"bound": "hbm", "achieved": dec_gbs, "peak": hpeak, "unit": "GB/s",
                             "frac": dec_gbs / hpeak, "traffic": tr_d,
-                            "kernel": "decode_kernel<128,2> (+ counter memset)",
+                            "kernel": "decode_kernel<128,2,1> (D=128, GQA 2, stage-table rotation; + counter memset)",
                             "peak_source": f"{peak_src} hbm_gbs",
                             "algorithmic": f"{decode_bytes(Dd)} B per launch"},
         "clocks": clocks,
