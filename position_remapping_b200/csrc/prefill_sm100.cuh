@@ -4,24 +4,30 @@
 // (batch, query head) against the key tiles of its passes:
 //   warps 0-3, 4-7  softmax warpgroups, one per query tile (one TMEM lane =
 //              one query row per thread): rotate the staged query tile in
-//              shared memory, then per key tile read S from TMEM, mask,
-//              online softmax in the exp2 domain, write P (bf16) back over S,
+//              shared memory, then per key tile copy S from TMEM into
+//              registers (and release S at once), mask, online softmax in the
+//              exp2 domain, write P (bf16) to the tile's own TMEM columns,
 //              and at the end normalise, merge and store O and the LSE.
 //   warp 8     TMA producer: the query tiles, then K and V tiles through one
 //              ring of NSLOT tile slots (128-byte swizzle, no multicast).
-//   warp 9     MMA issuer (one thread), per key tile j:
-//                S0 = Q0 K_j^T;  O1 += P1(j-1) V_(j-1);  S1 = Q1 K_j^T;
-//                O0 += P0(j) V_j
-//              so the tensor core works on one tile while the other tile's
-//              softmax runs, and when S_a(j) is ready the PV that last wrote
-//              O_a has completed (tcgen05.commit tracks all earlier MMAs),
-//              which lets the softmax rescale O_a in place without waiting.
-//   warps 10-11 idle (they complete the third warpgroup, whose registers are
+//   warp 9     QK issuer (one thread), per key tile j: S = Q0 K_j^T, then
+//              S = Q1 K_j^T. Both tiles share one S buffer: a QK only waits
+//              until the previous S has been copied into registers by its
+//              softmax, so the QKs of the next key tile overlap the
+//              exponentials of this one.
+//   warp 10    PV issuer (one thread), per key tile j: O0 += P0(j) V_j, then
+//              O1 += P1(j) V_j, each once its P is stored. Two issuers split
+//              the barrier waits and commits (each costs the issuing thread
+//              about a hundred cycles), so one keeps the tensor pipe fed while
+//              the other waits. A softmax waits for its tile's previous PV
+//              (one barrier per tile, committed after each PV) before
+//              rescaling O or overwriting P.
+//   warp 11    idle (it completes the third warpgroup, whose registers are
 //              handed to the softmax warpgroups with setmaxnreg: 216 per
 //              softmax thread, 72 per thread of warps 8-11; 384 x 168 at
 //              launch = 256 x 216 + 128 x 72).
-// TMEM (512 columns): S0/P0 [0,128), S1/P1 [128,256), O0 [256,256+D),
-// O1 [256+D, 256+2D).
+// TMEM (512 columns): S [0,128), P0 [128,192), P1 [192,256) (bf16 pairs),
+// O0 [256,256+D), O1 [256+D, 256+2D).
 //
 // A pass is a sweep over key tiles with one query rotation, one key tensor
 // and one distance band hi_off <= t - s <= lo_off:
@@ -109,8 +115,8 @@ struct PrefillSmem {
   static constexpr int kRing = kQ + kQT * kQBytes;
   static constexpr int kBar = kRing + NSLOT * kTileBytes;
   // barriers: q_full, q_ready[2], q_free, ring_full[NSLOT], ring_empty[NSLOT],
-  // s_full[2], p_full[2], o_final, o_free[2]
-  static constexpr int kNumBars = 11 + 2 * NSLOT;
+  // s_full[2], s_free, p_full[2], o_done[2], o_free[2]
+  static constexpr int kNumBars = 13 + 2 * NSLOT;
   static constexpr int kMisc = kBar + kNumBars * 8;  // tmem base (u32), abort flag (int)
   static constexpr int kTotal = kMisc + 16;
   static constexpr int kAlloc = kTotal + 1024;       // slack to align the base to 1024
@@ -138,10 +144,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint64_t* q_free = bars + 3;
   uint64_t* ring_full = bars + 4;          // [NSLOT]
   uint64_t* ring_empty = ring_full + NSLOT;
-  uint64_t* s_full = ring_empty + NSLOT;   // [2]
-  uint64_t* p_full = s_full + 2;           // [2]
-  uint64_t* o_final = p_full + 2;
-  uint64_t* o_free = o_final + 1;          // [2]
+  uint64_t* s_full = ring_empty + NSLOT;   // [2] S holds Q_a K^T
+  uint64_t* s_free = s_full + 2;           // S copied out by a softmax warpgroup
+  uint64_t* p_full = s_free + 1;           // [2]
+  uint64_t* o_done = p_full + 2;           // [2] PV of tile a completed
+  uint64_t* o_free = o_done + 2;           // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
@@ -173,9 +180,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(s_full + a, 1);
       mbar_init(p_full + a, kBM);
+      mbar_init(o_done + a, 1);
       mbar_init(o_free + a, kBM);
     }
-    mbar_init(o_final, 1);
+    mbar_init(s_free, kBM);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -193,7 +201,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem;            // S_a/P_a at columns 128 a
+  const uint32_t tS = tmem;            // S, shared by the two tiles
+  const uint32_t tP = tmem + 128;      // P_a at 128 + 64 a
   const uint32_t tO = tmem + 256;      // O_a at 256 + a D
 
   if (warp == 8) {
@@ -223,70 +232,69 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       }
     }
   } else if (warp == 9) {
-    // ------------------------------------------------------------------ MMA
+    // ---------------------------------------------------------- MMA: QK^T
+    reg_dealloc<kProducerRegs>();
+    if (lane == 0) {
+      int pos = 0, nqk = 0;
+      bool ok = true;
+      for (int pi = 0; pi < npass && ok; ++pi) {
+        if (!mbar_wait(q_ready + 0, pi & 1, abort_flag) || !mbar_wait(q_ready + 1, pi & 1, abort_flag)) break;
+        const int T = passes[pi].j_hi - passes[pi].j_lo + 1;
+        for (int i = 0; i < T && ok; ++i, pos += 2) {
+          const int kslot = pos % NSLOT;
+          if (!mbar_wait(ring_full + kslot, (pos / NSLOT) & 1, abort_flag)) { ok = false; break; }
+          const uint32_t kaddr = smem_u32(sRing + kslot * L::kTileBytes);
+          for (int a = 0; a < kQT; ++a) {
+            // S = Q_a K^T, once the previous S has been copied out
+            if (nqk > 0 && !mbar_wait(s_free, (nqk - 1) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t qaddr = smem_u32(sQ + a * L::kQBytes);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * kBlockBytes + (kk & 3) * 32;
+              umma_ss(tS, sdesc_sw128(qaddr + off, 16, 1024), sdesc_sw128(kaddr + off, 16, 1024), kIdescQK,
+                      kk > 0 ? 1u : 0u);
+            }
+            umma_commit(s_full + a);
+            ++nqk;
+          }
+          if (!ok) break;
+          umma_commit(ring_empty + kslot);
+          if (i == T - 1 && pi + 1 < npass) umma_commit(q_free);   // last read of this pass's Q
+        }
+      }
+    }
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ MMA: PV
     reg_dealloc<kProducerRegs>();
     if (lane == 0) {
       int pos = 0, g = 0;
       bool ok = true;
-      auto qk = [&](int a, uint32_t kaddr) {
-        const uint32_t qaddr = smem_u32(sQ + a * L::kQBytes);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kBlockBytes + (kk & 3) * 32;
-          umma_ss(tS + a * 128, sdesc_sw128(qaddr + off, 16, 1024), sdesc_sw128(kaddr + off, 16, 1024), kIdescQK,
-                  kk > 0 ? 1u : 0u);
-        }
-        umma_commit(s_full + a);
-      };
-      auto pv = [&](int a, uint32_t vaddr, bool accumulate) {
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t bdesc = sdesc_sw128(vaddr + kk * 2048, kBlockBytes, 1024);
-          umma_ts(tO + a * D, tS + a * 128 + kk * 8, bdesc, kIdescPV, (kk > 0 || accumulate) ? 1u : 0u);
-        }
-      };
       for (int pi = 0; pi < npass && ok; ++pi) {
-        if (!mbar_wait(q_ready + 0, pi & 1, abort_flag) || !mbar_wait(q_ready + 1, pi & 1, abort_flag)) break;
-        tc_fence_after();
         const int T = passes[pi].j_hi - passes[pi].j_lo + 1;
-        int vslot_prev = 0;
-        for (int i = 0; i < T; ++i, ++g) {
-          const int kpos = pos, vpos = pos + 1;
-          pos += 2;
-          const int kslot = kpos % NSLOT, vslot = vpos % NSLOT;
-          if (!mbar_wait(ring_full + kslot, (kpos / NSLOT) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t kaddr = smem_u32(sRing + kslot * L::kTileBytes);
-          qk(0, kaddr);
-          if (i > 0) {
-            // PV of tile 1 for the previous key tile
-            if (!mbar_wait(p_full + 1, (g - 1) & 1, abort_flag)) { ok = false; break; }
-            if (i == 1 && pi > 0 && !mbar_wait(o_free + 1, (pi - 1) & 1, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            pv(1, smem_u32(sRing + vslot_prev * L::kTileBytes), i > 1);
-            umma_commit(ring_empty + vslot_prev);
-          }
-          qk(1, kaddr);
-          umma_commit(ring_empty + kslot);
-          if (!mbar_wait(p_full + 0, g & 1, abort_flag)) { ok = false; break; }
+        for (int i = 0; i < T && ok; ++i, ++g, pos += 2) {
+          const int vpos = pos + 1, vslot = vpos % NSLOT;
           if (!mbar_wait(ring_full + vslot, (vpos / NSLOT) & 1, abort_flag)) { ok = false; break; }
-          if (i == 0 && pi > 0 && !mbar_wait(o_free + 0, (pi - 1) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          pv(0, smem_u32(sRing + vslot * L::kTileBytes), i > 0);
-          vslot_prev = vslot;
+          const uint32_t vaddr = smem_u32(sRing + vslot * L::kTileBytes);
+          for (int a = 0; a < kQT; ++a) {
+            // O_a += P_a V once P_a is stored (and, for a later pass, once the
+            // previous pass's partial has been read out of O_a)
+            if (!mbar_wait(p_full + a, g & 1, abort_flag)) { ok = false; break; }
+            if (i == 0 && pi > 0 && !mbar_wait(o_free + a, (pi - 1) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < kBN / 16; ++kk) {
+              const uint64_t bdesc = sdesc_sw128(vaddr + kk * 2048, kBlockBytes, 1024);
+              umma_ts(tO + a * D, tP + a * 64 + kk * 8, bdesc, kIdescPV, (kk > 0 || i > 0) ? 1u : 0u);
+            }
+            umma_commit(o_done + a);
+          }
+          if (!ok) break;
+          umma_commit(ring_empty + vslot);
         }
-        if (!ok) break;
-        // PV of tile 1 for the last key tile of the pass
-        if (!mbar_wait(p_full + 1, (g - 1) & 1, abort_flag)) break;
-        if (T == 1 && pi > 0 && !mbar_wait(o_free + 1, (pi - 1) & 1, abort_flag)) break;
-        tc_fence_after();
-        pv(1, smem_u32(sRing + vslot_prev * L::kTileBytes), T > 1);
-        umma_commit(ring_empty + vslot_prev);
-        umma_commit(o_final);
-        if (pi + 1 < npass) umma_commit(q_free);
       }
     }
-  } else if (warp >= 10) {
+  } else if (warp == 11) {
     reg_dealloc<kProducerRegs>();
   } else {
     // -------------------------------------------------------------- softmax
@@ -297,7 +305,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int t = qa0 + row;
     const bool row_ok = t < p.S;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tSa = tS + a * 128 + lane_off;
+    const uint32_t tSw = tS + lane_off;
+    const uint32_t tPa = tP + a * 64 + lane_off;
     const uint32_t tOa = tO + a * D + lane_off;
     uint8_t* sQa = sQ + a * L::kQBytes;
     // waits are made warp-uniform so the warp-collective TMEM accesses that
@@ -352,11 +361,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         {
           uint32_t r[kBN];
 #pragma unroll
-          for (int c = 0; c < kBN / 32; ++c) tmem_ld32(tSa + c * 32, *reinterpret_cast<uint32_t(*)[32]>(r + c * 32));
+          for (int c = 0; c < kBN / 32; ++c) tmem_ld32(tSw + c * 32, *reinterpret_cast<uint32_t(*)[32]>(r + c * 32));
           tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < kBN; ++e) s[e] = __uint_as_float(r[e]);
         }
+        // S is in registers: the other tile's QK may overwrite it
+        tc_fence_before();
+        mbar_arrive(s_free);
         const int kv0 = j * kBN;
         const bool full = (qa0 - kv0 - (kBN - 1) >= ps.hi_off) && (qa0 + kBM - 1 - kv0 <= ps.lo_off);
         if (!full) {
@@ -382,8 +394,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const float m_new = need ? mx : m;
         const float alpha = need ? ex2(m - m_new) : 1.0f;
         l *= alpha;
+        // the previous PV of this tile must have completed before O_a is
+        // rescaled or P_a is overwritten
+        if (g > 0 && !wwait(o_done + a, (g - 1) & 1)) { ok = false; break; }
+        tc_fence_after();
         if (j != ps.j_lo && __any_sync(0xffffffffu, need)) {
-          // the PV that last wrote O_a completed before S_a(j) was committed
           uint32_t r[32];
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
@@ -407,7 +422,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             lsum[(e >> 1) & 3] += p0 + p1;
             pk[e >> 1] = pack_bf16x2(p0, p1);
           }
-          tmem_st16(tSa + c * 16, pk);
+          tmem_st16(tPa + c * 16, pk);
         }
         l += (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
         tmem_st_wait();
@@ -416,8 +431,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       }
       if (!ok) break;
 
-      // ---- pass epilogue
-      if (!wwait(o_final, pi & 1)) { ok = false; break; }
+      // ---- pass epilogue: wait for the last PV of this tile
+      if (!wwait(o_done + a, (g - 1) & 1)) { ok = false; break; }
       tc_fence_after();
       const bool remote_partial = bif && ps.sel == 1;
       if (remote_partial) {
