@@ -99,6 +99,27 @@ int ropeattn_posmap(const ropeattn_params* params, int64_t L,
                     int32_t* d_pos_local, int32_t* d_pos_remote, int32_t* h_G,
                     void* stream);
 
+/* Writes tokens into a decode cache (Jet-Long §3.2 Eq. 4: each key is stored
+ * rotated at its own position, so the cache is never rewritten when the
+ * bifocal group size G changes as the sequence grows):
+ *   k_cache[b, start + i, h, :] = R(p(start + i)) k[b, i, h, :]  (bf16, RNE)
+ *   v_cache[b, start + i, h, :] = v[b, i, h, :]
+ * for i < count, p the kind's primary position of the absolute token index
+ * (t for STANDARD and BIFOCAL, EndPrompt's two segments, t mod W for
+ * PERIODIC; NOPE stores keys unrotated). Angles p * theta_i in double
+ * precision, rotation in fp32, as the prefill's key pre-pass does.
+ *   k, v:             [B, count, Hkv, D] bf16, device, 4-byte aligned
+ *   k_cache, v_cache: [B, cache_len, Hkv, D] bf16, device; caller-owned
+ *   v, v_cache:       both NULL to write keys only
+ *   start + count <= cache_len. A prefill of S tokens emits its cache with
+ *   start = 0, count = S; a decode step appends its token with start = n-1
+ *   before ropeattn_decode reads the first n rows.
+ * count == 0 or B == 0 is a no-op. Errors: INVALID_ARG, UNSUPPORTED_DEVICE,
+ * CUDA. */
+int ropeattn_cache_write(const void* k, const void* v, void* k_cache, void* v_cache,
+                         int64_t B, int64_t start, int64_t count, int64_t cache_len,
+                         int32_t Hkv, int32_t D, const ropeattn_params* params, void* stream);
+
 /* Bytes of device workspace ropeattn_prefill needs for these shapes:
  * rotated keys (one copy per position map the kind uses) and the query
  * angle tables. 0 for NOPE. */

@@ -24,9 +24,9 @@ What it computes, and where each step is defined:
 * Bifocal score: RoPE at (q, k) when q - k <= w0, else RoPE at (f(q), f(k)),
   with G = max(1, ceil(L / w_pretrained)) and f(x) = floor(x / G): Jet-Long,
   §3 Eq. 1, §3.1 Eq. 2-3.
-* Decode with an untouched cache k_cache[k] = RoPE(x_k, k) and the correction
-  rotation by Delta = f(x) - x on the query and on each cached key: Jet-Long,
-  §3.2 Eq. 4-6.
+* Decode with an untouched cache k_cache[k] = RoPE(x_k, k) (``cache_keys``)
+  and the correction rotation by Delta = f(x) - x on the query and on each
+  cached key: Jet-Long, §3.2 Eq. 4-6.
 * The literal three-call inclusion-exclusion merge: Jet-Long, §3.3 Eq. 7
   (kept as a self-check; the routed softmax is the definition it reaches).
 
@@ -53,7 +53,7 @@ __all__ = [
     "round_bf16", "rope_frequencies", "rotation_matrix", "rotate",
     "periodic_position", "endprompt_position", "group_size", "remote_position",
     "position_maps", "softmax_scale", "prefill", "prefill_three_call",
-    "decode", "brute_prefill", "brute_decode", "to_f64",
+    "decode", "cache_keys", "brute_prefill", "brute_decode", "to_f64",
 ]
 
 
@@ -288,6 +288,27 @@ def prefill_three_call(q, k, v, params, stage_bf16: bool = True):
 # ----------------------------------------------------------------------------
 # decode (Jet-Long §3.2): untouched cache + correction rotation
 # ----------------------------------------------------------------------------
+def cache_keys(k, params, start: int = 0):
+    """The decode cache entries of keys k [B,count,Hkv,D] at absolute token
+    indices start..start+count-1: each key rotated at the kind's own position
+    of its index (Jet-Long §3.2 Eq. 4, k_cache[k] = RoPE(x_k, k); the other
+    kinds store keys at their own positions: EndPrompt's two segments, t mod W
+    for Periodic RoPE; NoPE stores keys unrotated). The result does not depend
+    on the sequence length, so the cache is never rewritten as L (and G)
+    grows. Float64, not rounded."""
+    k = to_f64(k)
+    count, D = k.shape[1], k.shape[3]
+    if int(params.kind) == NOPE:
+        return k.copy()
+    p_loc = position_maps(params, int(start) + count)[0][int(start):]
+    freqs = _freqs(params, D)
+    out = np.empty_like(k)
+    for b in range(k.shape[0]):
+        for h in range(k.shape[2]):
+            out[b, :, h] = rotate(k[b, :, h], p_loc, freqs)
+    return out
+
+
 def decode(q, k_cache, v_cache, params):
     """One query token at position n-1 against a cache of n keys.
 

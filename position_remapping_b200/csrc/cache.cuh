@@ -1,0 +1,60 @@
+// Decode-cache writer (Jet-Long §3.2 Eq. 4): each new key is stored rotated
+// at its own position, and the cache is never rewritten afterwards, however
+// the bifocal group size G changes as the sequence grows.
+//
+// One thread per (token, rotation pair), as in the prefill key pre-pass: the
+// angle p * theta_i is taken in double precision (p the kind's primary
+// position of the token's absolute index), sincos in double, rounded to fp32;
+// the pair is rotated in fp32 and rounded to bf16 (nearest even) for every
+// (batch, kv head) row of the token. The value pair is copied alongside.
+// Consecutive threads touch consecutive 4-byte words of a row.
+#pragma once
+
+#include "common.cuh"
+#include "posmap.cuh"
+
+namespace ropeattn {
+
+struct CacheArgs {
+  const uint32_t* k;   // [B, count, Hkv, D] bf16 pairs
+  const uint32_t* v;   // same layout, or null
+  uint32_t* k_cache;   // [B, cache_len, Hkv, D]
+  uint32_t* v_cache;   // same layout, or null
+  long long start, count, cache_len;
+  int B, Hkv, D;
+  PosMap m;
+  double theta[kMaxPairs];
+};
+
+__global__ void __launch_bounds__(256) cache_write_kernel(const CacheArgs a) {
+  const int P = a.D >> 1;
+  const int rows = blockDim.x / P;
+  const long long i_tok = static_cast<long long>(blockIdx.x) * rows + threadIdx.x / P;
+  const int i = threadIdx.x % P;
+  if (i_tok >= a.count) return;
+  const long long t = a.start + i_tok;
+  float c = 1.f, s = 0.f;
+  if (a.m.kind != kNope) {
+    double sd, cd;
+    sincos(static_cast<double>(pos_primary(a.m, static_cast<int>(t))) * a.theta[i], &sd, &cd);
+    c = static_cast<float>(cd);
+    s = static_cast<float>(sd);
+  }
+  for (int b = 0; b < a.B; ++b) {
+    for (int h = 0; h < a.Hkv; ++h) {
+      const size_t src = ((static_cast<size_t>(b) * a.count + i_tok) * a.Hkv + h) * P + i;
+      const size_t dst = ((static_cast<size_t>(b) * a.cache_len + t) * a.Hkv + h) * P + i;
+      const uint32_t x = __ldg(a.k + src);
+      if (a.m.kind == kNope) {
+        a.k_cache[dst] = x;
+      } else {
+        float y0, y1;
+        rot_pair(bf16lo(x), bf16hi(x), c, s, y0, y1);
+        a.k_cache[dst] = pack_bf16x2(y0, y1);
+      }
+      if (a.v != nullptr) a.v_cache[dst] = __ldg(a.v + src);
+    }
+  }
+}
+
+}  // namespace ropeattn

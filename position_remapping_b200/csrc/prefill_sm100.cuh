@@ -15,17 +15,17 @@
 //              until the previous S has been copied into registers by its
 //              softmax, so the QKs of the next key tile overlap the
 //              exponentials of this one.
-//   warp 10    PV issuer (one thread), per key tile j: O0 += P0(j) V_j, then
-//              O1 += P1(j) V_j, each once its P is stored. Two issuers split
-//              the barrier waits and commits (each costs the issuing thread
-//              about a hundred cycles), so one keeps the tensor pipe fed while
-//              the other waits. A softmax waits for its tile's previous PV
-//              (one barrier per tile, committed after each PV) before
+//   warps 10, 11  PV issuers (one thread each), per key tile j:
+//              O_a += P_a(j) V_j for tile a = warp - 10, once P_a is stored.
+//              Separate issuers split the barrier waits and commits (each
+//              costs the issuing thread about a hundred cycles, and the issue
+//              queue is about one MMA deep), so one keeps the tensor pipe fed
+//              while another waits. A softmax waits for its tile's previous
+//              PV (one barrier per tile, committed after each PV) before
 //              rescaling O or overwriting P.
-//   warp 11    idle (it completes the third warpgroup, whose registers are
-//              handed to the softmax warpgroups with setmaxnreg: 216 per
-//              softmax thread, 72 per thread of warps 8-11; 384 x 168 at
-//              launch = 256 x 216 + 128 x 72).
+//   Registers: warps 8-11 (the third warpgroup) hand theirs to the softmax
+//              warpgroups with setmaxnreg: 216 per softmax thread, 72 per
+//              thread of warps 8-11; 384 x 168 at launch = 256 x 216 + 128 x 72.
 // TMEM (512 columns): S [0,128), P0 [128,192), P1 [192,256) (bf16 pairs),
 // O0 [256,256+D), O1 [256+D, 256+2D).
 //
@@ -128,6 +128,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                    const __grid_constant__ CUtensorMap tmK1, const __grid_constant__ CUtensorMap tmV,
                    const PrefillParams p) {
   using L = PrefillSmem<D, NSLOT>;
+  static_assert(NSLOT % 2 == 0, "K and V tiles alternate over an even number of ring slots");
   constexpr int kCB = D / 64;              // 64-column (128-byte) swizzle blocks per row
   constexpr int kBlockBytes = kBM * 128;   // one swizzle block of a 128-row tile
   constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, false);
@@ -173,9 +174,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     mbar_init(q_ready + 0, kBM);
     mbar_init(q_ready + 1, kBM);
     mbar_init(q_free, 1);
+    // K tiles sit at even ring positions (released by the QK issuer), V tiles
+    // at odd ones (released by both PV issuers); NSLOT is even
     for (int i = 0; i < NSLOT; ++i) {
       mbar_init(ring_full + i, 1);
-      mbar_init(ring_empty + i, 1);
+      mbar_init(ring_empty + i, (i & 1) ? 2 : 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(s_full + a, 1);
@@ -264,10 +267,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
       }
     }
-  } else if (warp == 10) {
-    // ------------------------------------------------------------ MMA: PV
+  } else if (warp == 10 || warp == 11) {
+    // --------------------------------------------- MMA: PV of tile warp - 10
     reg_dealloc<kProducerRegs>();
     if (lane == 0) {
+      const int a = warp - 10;
       int pos = 0, g = 0;
       bool ok = true;
       for (int pi = 0; pi < npass && ok; ++pi) {
@@ -275,27 +279,22 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         for (int i = 0; i < T && ok; ++i, ++g, pos += 2) {
           const int vpos = pos + 1, vslot = vpos % NSLOT;
           if (!mbar_wait(ring_full + vslot, (vpos / NSLOT) & 1, abort_flag)) { ok = false; break; }
+          // O_a += P_a V once P_a is stored (and, for a later pass, once the
+          // previous pass's partial has been read out of O_a)
+          if (!mbar_wait(p_full + a, g & 1, abort_flag)) { ok = false; break; }
+          if (i == 0 && pi > 0 && !mbar_wait(o_free + a, (pi - 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
           const uint32_t vaddr = smem_u32(sRing + vslot * L::kTileBytes);
-          for (int a = 0; a < kQT; ++a) {
-            // O_a += P_a V once P_a is stored (and, for a later pass, once the
-            // previous pass's partial has been read out of O_a)
-            if (!mbar_wait(p_full + a, g & 1, abort_flag)) { ok = false; break; }
-            if (i == 0 && pi > 0 && !mbar_wait(o_free + a, (pi - 1) & 1, abort_flag)) { ok = false; break; }
-            tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < kBN / 16; ++kk) {
-              const uint64_t bdesc = sdesc_sw128(vaddr + kk * 2048, kBlockBytes, 1024);
-              umma_ts(tO + a * D, tP + a * 64 + kk * 8, bdesc, kIdescPV, (kk > 0 || i > 0) ? 1u : 0u);
-            }
-            umma_commit(o_done + a);
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            const uint64_t bdesc = sdesc_sw128(vaddr + kk * 2048, kBlockBytes, 1024);
+            umma_ts(tO + a * D, tP + a * 64 + kk * 8, bdesc, kIdescPV, (kk > 0 || i > 0) ? 1u : 0u);
           }
-          if (!ok) break;
-          umma_commit(ring_empty + vslot);
+          umma_commit(o_done + a);
+          umma_commit(ring_empty + vslot);   // one of the V slot's two releases
         }
       }
     }
-  } else if (warp == 11) {
-    reg_dealloc<kProducerRegs>();
   } else {
     // -------------------------------------------------------------- softmax
     reg_alloc<kSoftmaxRegs>();
@@ -379,13 +378,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             if (d < ps.hi_off || d > ps.lo_off) s[c] = -INFINITY;
           }
         }
+        // row max: 8 independent chains of 3-input max over columns e + 8k
         float mx8[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) mx8[e] = s[e];
+        for (int e = 0; e < 8; ++e) {
+          float x = fmax3(s[e], s[e + 8], s[e + 16]);
 #pragma unroll
-        for (int c = 8; c < kBN; c += 8)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], s[c + e]);
+          for (int k = 3; k + 1 < kBN / 8; k += 2) x = fmax3(x, s[e + 8 * k], s[e + 8 * k + 8]);
+          mx8[e] = fmaxf(x, s[e + kBN - 8]);
+        }
         float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                          fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         mx *= sl2;
@@ -411,20 +412,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
         m = m_new;
         const float mu = (m == -INFINITY) ? 0.f : m;
-        float lsum[4] = {0.f, 0.f, 0.f, 0.f};
+        const float2 sl2x2 = make_float2(sl2, sl2), nmu2 = make_float2(-mu, -mu);
+        float2 lsum[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int c = 0; c < kBN / 32; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float p0 = ex2(fmaf(s[c * 32 + e], sl2, -mu));
-            const float p1 = ex2(fmaf(s[c * 32 + e + 1], sl2, -mu));
-            lsum[(e >> 1) & 3] += p0 + p1;
-            pk[e >> 1] = pack_bf16x2(p0, p1);
+            const float2 x = __ffma2_rn(make_float2(s[c * 32 + e], s[c * 32 + e + 1]), sl2x2, nmu2);
+            const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+            lsum[(e >> 1) & 1] = __fadd2_rn(lsum[(e >> 1) & 1], pp);
+            pk[e >> 1] = pack_bf16x2(pp.x, pp.y);
           }
           tmem_st16(tPa + c * 16, pk);
         }
-        l += (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
+        l += (lsum[0].x + lsum[0].y) + (lsum[1].x + lsum[1].y);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(p_full + a);

@@ -11,6 +11,7 @@
 
 #include "../../include/ropeattn.h"
 #include "common.cuh"
+#include "cache.cuh"
 #include "decode_sm100.cuh"
 #include "posmap.cuh"
 #include "prefill_sm100.cuh"
@@ -306,6 +307,50 @@ int ropeattn_posmap(const ropeattn_params* params, int64_t L, int32_t* d_pos_loc
   posmap_kernel<<<static_cast<unsigned>(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(
       m, static_cast<int>(L), d_pos_local, d_pos_remote);
   CUDA_TRY(cudaGetLastError(), "posmap launch");
+  return ROPEATTN_OK;
+}
+
+int ropeattn_cache_write(const void* k, const void* v, void* k_cache, void* v_cache, int64_t B, int64_t start,
+                         int64_t count, int64_t cache_len, int32_t Hkv, int32_t D, const ropeattn_params* params,
+                         void* stream) {
+  g_last_error.clear();
+  if (B < 0 || start < 0 || count < 0 || cache_len < 0)
+    return fail(ROPEATTN_ERR_INVALID_ARG, "B, start, count and cache_len must be >= 0");
+  if (start + count > cache_len)
+    return fail(ROPEATTN_ERR_INVALID_ARG, "start + count (%lld) exceeds cache_len (%lld)",
+                static_cast<long long>(start + count), static_cast<long long>(cache_len));
+  int rc = check_shapes(B, cache_len, Hkv, Hkv, D);
+  if (rc) return rc;
+  PosMap m;
+  int eff;
+  rc = check_params(params, cache_len, D, &m, &eff);
+  if (rc) return rc;
+  if (B == 0 || count == 0) return ROPEATTN_OK;
+  if (!k || !k_cache) return fail(ROPEATTN_ERR_INVALID_ARG, "k and k_cache must not be NULL");
+  if ((v == nullptr) != (v_cache == nullptr))
+    return fail(ROPEATTN_ERR_INVALID_ARG, "v and v_cache must be both given or both NULL");
+  if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v) |
+       reinterpret_cast<uintptr_t>(v_cache)) & 3u)
+    return fail(ROPEATTN_ERR_INVALID_ARG, "tensor pointers must be 4-byte aligned");
+  rc = check_device();
+  if (rc) return rc;
+  CacheArgs a{};
+  a.k = static_cast<const uint32_t*>(k);
+  a.v = static_cast<const uint32_t*>(v);
+  a.k_cache = static_cast<uint32_t*>(k_cache);
+  a.v_cache = static_cast<uint32_t*>(v_cache);
+  a.start = start;
+  a.count = count;
+  a.cache_len = cache_len;
+  a.B = static_cast<int>(B);
+  a.Hkv = Hkv;
+  a.D = D;
+  m.kind = params->kind == ROPEATTN_BIFOCAL ? ROPEATTN_STANDARD : params->kind;  // primary position: t
+  a.m = m;
+  fill_theta(params, D, a.theta);
+  const int rows = 256 / (D / 2);
+  cache_write_kernel<<<static_cast<unsigned>((count + rows - 1) / rows), 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
+  CUDA_TRY(cudaGetLastError(), "cache_write launch");
   return ROPEATTN_OK;
 }
 

@@ -21,7 +21,7 @@ OK = 0
 ERR_INVALID_ARG, ERR_UNSUPPORTED_DEVICE, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = -1, -2, -3, -4, -5
 
 # every symbol include/ropeattn.h declares
-EXPORTS = ("ropeattn_posmap", "ropeattn_prefill_workspace_size", "ropeattn_prefill",
+EXPORTS = ("ropeattn_posmap", "ropeattn_cache_write", "ropeattn_prefill_workspace_size", "ropeattn_prefill",
            "ropeattn_prefill_prepare", "ropeattn_prefill_attend",
            "ropeattn_decode_workspace_size", "ropeattn_decode", "ropeattn_decode_noalloc", "ropeattn_status",
            "ropeattn_last_error", "ropeattn_version")
@@ -71,6 +71,7 @@ def _load() -> ctypes.CDLL:
     vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
     P = ctypes.POINTER(CParams)
     lib.ropeattn_posmap.argtypes = [P, i64, vp, vp, ctypes.POINTER(i32), vp]
+    lib.ropeattn_cache_write.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i32, i32, P, vp]
     lib.ropeattn_prefill_workspace_size.argtypes = [P, i64, i64, i32, i32, i32]
     lib.ropeattn_prefill_workspace_size.restype = sz
     lib.ropeattn_prefill.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, P, vp, sz, vp]
@@ -85,7 +86,7 @@ def _load() -> ctypes.CDLL:
     lib.ropeattn_last_error.argtypes = []
     lib.ropeattn_last_error.restype = ctypes.c_char_p
     lib.ropeattn_version.argtypes = []
-    for name in ("ropeattn_posmap", "ropeattn_prefill", "ropeattn_prefill_prepare", "ropeattn_prefill_attend",
+    for name in ("ropeattn_posmap", "ropeattn_cache_write", "ropeattn_prefill", "ropeattn_prefill_prepare", "ropeattn_prefill_attend",
                  "ropeattn_decode", "ropeattn_status", "ropeattn_version"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
@@ -125,6 +126,17 @@ def posmap(params: MapParams, L: int, device="cuda", stream=None) -> Tuple[torch
     G = ctypes.c_int32(0)
     _check(lib.ropeattn_posmap(ctypes.byref(cp), int(L), _ptr(loc), _ptr(rem), ctypes.byref(G), _stream(stream)))
     return loc[:L], rem[:L], int(G.value)
+
+
+def cache_write(k: torch.Tensor, v: Optional[torch.Tensor], k_cache: torch.Tensor, v_cache: Optional[torch.Tensor],
+                params: MapParams, start: int, stream=None) -> None:
+    """Stores k [B,count,Hkv,D] rotated at positions start..start+count-1 (and
+    v as is) into rows start.. of k_cache / v_cache [B,cache_len,Hkv,D]."""
+    B, count, Hkv, D = k.shape
+    cache_len = k_cache.shape[1]
+    cp = to_cparams(params)
+    _check(lib.ropeattn_cache_write(_ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), B, int(start), count, cache_len,
+                                    Hkv, D, ctypes.byref(cp), _stream(stream)))
 
 
 def prefill_workspace_size(params: MapParams, B, S, Hq, Hkv, D) -> int:

@@ -117,6 +117,28 @@ def test_host_argument_checks(ra):
                                ctypes.byref(G), nullp) == ra.OK and G.value == 1
 
 
+def test_cache_write_argument_checks(ra):
+    from position_remapping_b200.inputs import BIFOCAL, STANDARD
+    lib = ra.lib
+    nullp = ctypes.c_void_p(0)
+    p = ctypes.byref(ra.to_cparams(_p(kind=BIFOCAL, w0=4, w_pretrained=8)))
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: rejected before any device work
+    # rows past the end of the cache
+    assert lib.ropeattn_cache_write(fake, fake, fake, fake, 1, 90, 20, 100, 2, 64, p, nullp) == ra.ERR_INVALID_ARG
+    # negative sizes, bad head_dim
+    assert lib.ropeattn_cache_write(fake, fake, fake, fake, 1, -1, 2, 100, 2, 64, p, nullp) == ra.ERR_INVALID_ARG
+    assert lib.ropeattn_cache_write(fake, fake, fake, fake, 1, 0, 2, 100, 2, 96, p, nullp) == ra.ERR_INVALID_ARG
+    # v and v_cache must come together; k must be given
+    assert lib.ropeattn_cache_write(fake, fake, fake, nullp, 1, 0, 2, 100, 2, 64, p, nullp) == ra.ERR_INVALID_ARG
+    assert lib.ropeattn_cache_write(nullp, nullp, fake, nullp, 1, 0, 2, 100, 2, 64, p, nullp) == ra.ERR_INVALID_ARG
+    # misaligned pointer
+    odd = ctypes.c_void_p((1 << 20) + 2)
+    assert lib.ropeattn_cache_write(odd, nullp, fake, nullp, 1, 0, 2, 100, 2, 64, p, nullp) == ra.ERR_INVALID_ARG
+    # nothing to write
+    q = ctypes.byref(ra.to_cparams(_p(kind=STANDARD)))
+    assert lib.ropeattn_cache_write(nullp, nullp, nullp, nullp, 1, 5, 0, 100, 2, 64, q, nullp) == ra.OK
+
+
 def test_workspace_sizes(ra):
     from position_remapping_b200.inputs import WORKLOADS
     w = WORKLOADS["bifocal_prefill_s131072"]

@@ -398,3 +398,39 @@ def test_decode_equals_last_prefill_row():
     dec = O.decode(qn[:, 29], _cache(kn, params, 16), vn, params)
     assert np.allclose(dec[0], pre[0][:, 0], atol=1e-12)
     assert np.allclose(dec[1], pre[1][:, :, 0], atol=1e-12)
+
+
+@pytest.mark.parametrize("kind", [O.STANDARD, O.ENDPROMPT, O.PERIODIC, O.NOPE, O.BIFOCAL])
+def test_cache_keys_match_complex_form_and_offsets(kind):
+    # Eq. 4: the cache entry of token t is its key rotated at the kind's
+    # position of t, whatever the chunk it is written in
+    params = {O.STANDARD: MapParams(O.STANDARD, rope_base=1e4),
+              O.ENDPROMPT: MapParams(O.ENDPROMPT, rope_base=5e5, interp=8.0, seg1_len=11, term_start=65500),
+              O.PERIODIC: MapParams(O.PERIODIC, window=5),
+              O.NOPE: MapParams(O.NOPE),
+              O.BIFOCAL: MapParams(O.BIFOCAL, rope_base=1e6, w0=3, w_pretrained=6)}[kind]
+    _, kf, _ = make_qkv(2, 23, 2, 2, 8, seed=31)
+    kn = O.to_f64(kf)
+    whole = O.cache_keys(kn, params)
+    assert np.allclose(whole, _cache(kn, params, 8), atol=1e-12)
+    parts = np.concatenate([O.cache_keys(kn[:, :7], params, 0), O.cache_keys(kn[:, 7:16], params, 7),
+                            O.cache_keys(kn[:, 16:], params, 16)], axis=1)
+    assert np.allclose(parts, whole, atol=1e-12)
+
+
+def test_decode_over_growing_cache_crosses_group_changes():
+    # Jet-Long §3.2: the cache written once (Eq. 4) serves every later step,
+    # including the lengths where G = ceil(L / w_pre) changes; each step's
+    # decode equals the last row of a prefill of that length (L = n)
+    params = MapParams(O.BIFOCAL, rope_base=1e4, w0=3, w_pretrained=8)
+    q, k, v = make_qkv(1, 26, 4, 2, 8, seed=32)
+    qn, kn, vn = O.to_f64(q), O.to_f64(k), O.to_f64(v)
+    cache = O.cache_keys(kn, params)
+    Gs = set()
+    for n in (8, 9, 16, 17, 24, 25, 26):
+        Gs.add(O.group_size(n, params.w_pretrained))
+        dec = O.decode(qn[:, n - 1], cache[:, :n], vn[:, :n], params)
+        pre = O.prefill(qn[:, :n], kn[:, :n], vn[:, :n], params, rows=[n - 1], stage_bf16=False)
+        assert np.allclose(dec[0], pre[0][:, 0], atol=1e-12)
+        assert np.allclose(dec[1], pre[1][:, :, 0], atol=1e-12)
+    assert Gs == {1, 2, 3, 4}
