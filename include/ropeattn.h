@@ -162,6 +162,31 @@ int ropeattn_prefill_attend(const void* q, const void* k, const void* v, float* 
                             const ropeattn_params* params,
                             void* workspace, size_t workspace_bytes, void* stream);
 
+/* Prefill of a chunk of `count` new tokens, at positions start..L-1 with
+ * L = start + count, against a decode cache that already holds all L keys
+ * and values (rows 0..L-1 written by ropeattn_cache_write, the chunk's own
+ * tokens included): the last `count` rows of a prefill of length L, for
+ * chunked prefill and for extending a cached context. Keys are read as
+ * stored (Jet-Long §3.2 Eq. 4); for BIFOCAL a pre-pass writes the remote
+ * keys R(Delta s) k_cache[s], Delta s = f(s) - s with G = G(L) (Eq. 5-6),
+ * into `workspace`, and the remote pass reads them. Queries are rotated in
+ * the attention kernel as in ropeattn_prefill. Tensor-core operands are
+ * bf16 (the remote keys are rounded to bf16 after the correction).
+ *   q:      [B, count, Hq, D] bf16, unrotated
+ *   k_cache, v_cache: [B, L, Hkv, D] bf16 (contiguous, L rows)
+ *   out:    [B, count, Hq, D] fp32;  lse: [B, Hq, count] fp32 (natural log)
+ *   workspace: >= ropeattn_prefill_chunk_workspace_size bytes, 256-byte
+ *              aligned (may be NULL when that size is 0).
+ * count == 0 or B == 0 is a no-op. With start = 0 this is a whole prefill
+ * from a cache. Errors: INVALID_ARG, UNSUPPORTED_DEVICE, WORKSPACE, CUDA. */
+size_t ropeattn_prefill_chunk_workspace_size(const ropeattn_params* params, int64_t B, int64_t start,
+                                             int64_t count, int32_t Hq, int32_t Hkv, int32_t D);
+int ropeattn_prefill_chunk(const void* q, const void* k_cache, const void* v_cache,
+                           float* out, float* lse,
+                           int64_t B, int64_t start, int64_t count, int32_t Hq, int32_t Hkv, int32_t D,
+                           const ropeattn_params* params, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
 /* Bytes of device workspace ropeattn_decode needs (split-KV partials and
  * per-head arrival counters). Depends on the current device's SM count. */
 size_t ropeattn_decode_workspace_size(int64_t B, int64_t n, int32_t Hq,

@@ -53,7 +53,7 @@ __all__ = [
     "round_bf16", "rope_frequencies", "rotation_matrix", "rotate",
     "periodic_position", "endprompt_position", "group_size", "remote_position",
     "position_maps", "softmax_scale", "prefill", "prefill_three_call",
-    "decode", "cache_keys", "brute_prefill", "brute_decode", "to_f64",
+    "decode", "cache_keys", "prefill_from_cache", "brute_prefill", "brute_decode", "to_f64",
 ]
 
 
@@ -307,6 +307,53 @@ def cache_keys(k, params, start: int = 0):
         for h in range(k.shape[2]):
             out[b, :, h] = rotate(k[b, :, h], p_loc, freqs)
     return out
+
+
+def prefill_from_cache(q, k_cache, v_cache, params, start: int, stage_bf16: bool = True):
+    """Rows start..L-1 of a prefill of length L = k_cache.shape[1] whose keys
+    come from a decode cache (Eq. 4: k_cache[s] = RoPE(x_s, p(s))) instead of
+    raw keys: q [B,count,Hq,D] holds the unrotated queries of tokens
+    start..L-1 (count = L - start). Local scores read the cache as stored;
+    for BIFOCAL, remote scores read each cached key through the correction
+    rotation by Delta s = f(s) - s (Eq. 5-6, as in decode) against the query
+    rotated to f(t). ``stage_bf16`` rounds the rotated queries and the
+    corrected remote keys to bf16 (the cache itself is taken as given).
+    Returns out [B,count,Hq,D], lse [B,Hq,count]."""
+    q, kc, vc = to_f64(q), to_f64(k_cache), to_f64(v_cache)
+    B, count, Hq, D = q.shape
+    L, Hkv = kc.shape[1], kc.shape[2]
+    assert count == L - int(start)
+    grp = Hq // Hkv
+    scale = softmax_scale(D, params)
+    kind = int(params.kind)
+    freqs = _freqs(params, D)
+    p_loc, p_rem, G = position_maps(params, L)
+    stage = round_bf16 if stage_bf16 else (lambda a: a)
+    keys = np.arange(L)
+    rows = np.arange(int(start), L)
+    out = np.zeros((B, count, Hq, D))
+    lse = np.zeros((B, Hq, count))
+    for b in range(B):
+        for hk in range(Hkv):
+            kl = kc[b, :, hk]
+            kr = stage(rotate(kl, p_rem - keys, freqs)) if kind == BIFOCAL else None   # Eq. 6, keys
+            for h in range(hk * grp, (hk + 1) * grp):
+                for c0 in range(0, count, 64):
+                    rr = rows[c0:c0 + 64]
+                    nk = int(rr.max()) + 1
+                    ok = np.stack([_allowed(params, int(t), keys[:nk]) for t in rr])
+                    qq = q[b, rr - int(start), h, :]
+                    ql = qq if kind == NOPE else stage(rotate(qq, p_loc[rr], freqs))
+                    sc = (ql @ kl[:nk].T) * scale
+                    if kind == BIFOCAL:
+                        qr = stage(rotate(qq, p_rem[rr], freqs))
+                        sr = (qr @ kr[:nk].T) * scale
+                        local = (rr[:, None] - keys[None, :nk]) <= int(params.w0)
+                        sc = np.where(local, sc, sr)
+                    o, l = _softmax_rows(sc, ok, vc[b, :nk, hk, :])
+                    out[b, c0:c0 + 64, h, :] = o
+                    lse[b, h, c0:c0 + 64] = l
+    return out, lse
 
 
 def decode(q, k_cache, v_cache, params):

@@ -62,7 +62,9 @@ struct PrefillParams {
   float* lse;          // [B, Hq, S]
   const float2* tab0;  // [S][D/2] query (cos, sin) at map-0 positions (null for NoPE)
   const float2* tab1;  // [S][D/2] at remote positions (bifocal)
-  int B, S, Hq, Hkv;
+  int B, S, Hq, Hkv;   // S: query rows
+  int Sk;              // keys (rows of K and V); S for a whole prefill
+  int q_off;           // absolute position index of query row 0 (0 for a whole prefill)
   int nqb;             // 256-row query blocks per (b, h)
   int kind;
   int window;          // Periodic RoPE
@@ -90,12 +92,14 @@ __device__ __forceinline__ int make_passes(const PrefillParams& p, int q0, PassD
     bands[0][0] = kInf; bands[0][1] = 0; bands[0][2] = 0;
     nb = 1;
   }
-  const int q_last = min(p.S - 1, q0 + kBlockRows - 1);
+  // absolute positions of the block's first and last query rows
+  const int t_first = p.q_off + q0;
+  const int t_last = p.q_off + min(p.S - 1, q0 + kBlockRows - 1);
   int n = 0;
   for (int i = 0; i < nb; ++i) {
     const int lo_off = bands[i][0], hi_off = bands[i][1];
-    const int s_min = lo_off >= kInf ? 0 : max(0, q0 - lo_off);
-    const int s_max = min(p.S - 1, q_last - hi_off);
+    const int s_min = lo_off >= kInf ? 0 : max(0, t_first - lo_off);
+    const int s_max = min(p.Sk - 1, t_last - hi_off);
     if (s_max < s_min) continue;
     ps[n].j_lo = s_min / kBN;
     ps[n].j_hi = s_max / kBN;
@@ -369,9 +373,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         tc_fence_before();
         mbar_arrive(s_free);
         const int kv0 = j * kBN;
-        const bool full = (qa0 - kv0 - (kBN - 1) >= ps.hi_off) && (qa0 + kBM - 1 - kv0 <= ps.lo_off);
+        const int ta0 = p.q_off + qa0;   // absolute position of the tile's first row
+        const bool full = (ta0 - kv0 - (kBN - 1) >= ps.hi_off) && (ta0 + kBM - 1 - kv0 <= ps.lo_off);
         if (!full) {
-          const int dbase = t - kv0;  // t - s = dbase - c
+          const int dbase = p.q_off + t - kv0;  // t - s = dbase - c (absolute t)
 #pragma unroll
           for (int c = 0; c < kBN; ++c) {
             const int d = dbase - c;

@@ -56,4 +56,52 @@ __global__ void __launch_bounds__(256) rope_prep_kernel(const PrepArgs a) {
   }
 }
 
+// Prefill of a chunk of query rows against a decode cache (Jet-Long §3.2
+// Eq. 4: the cache holds every key rotated at its own position). The cache
+// is the local key tensor as it stands; for BIFOCAL this pass writes the
+// remote keys R(Delta s) k_cache[s], Delta s = f(s) - s (the correction of
+// Eq. 5-6), for every cached row, and the query angle tables of the chunk's
+// rows (absolute positions start + r). One thread per (token, pair).
+struct ChunkPrepArgs {
+  const uint32_t* k_cache;  // [B, L, Hkv, D] bf16 pairs
+  uint32_t* k_rem;          // [B, L, Hkv, D] remote keys (BIFOCAL), else null
+  float2* tab0;             // [count][D/2] (cos, sin) at primary positions, or null (NOPE)
+  float2* tab1;             // [count][D/2] at remote positions (BIFOCAL), else null
+  int B, L, Hkv, D, start;
+  PosMap m;
+  double theta[kMaxPairs];
+};
+
+__global__ void __launch_bounds__(256) chunk_prep_kernel(const ChunkPrepArgs a) {
+  const int P = a.D >> 1;
+  const int rows = blockDim.x / P;
+  const int t = blockIdx.x * rows + threadIdx.x / P;
+  const int i = threadIdx.x % P;
+  if (t >= a.L) return;
+  if (a.k_rem != nullptr) {
+    double sd, cd;
+    sincos(static_cast<double>(pos_remote(a.m, t) - t) * a.theta[i], &sd, &cd);
+    const float c = static_cast<float>(cd), s = static_cast<float>(sd);
+    for (int b = 0; b < a.B; ++b) {
+      for (int h = 0; h < a.Hkv; ++h) {
+        const size_t w = ((static_cast<size_t>(b) * a.L + t) * a.Hkv + h) * P + i;
+        const uint32_t x = __ldg(a.k_cache + w);
+        float y0, y1;
+        rot_pair(bf16lo(x), bf16hi(x), c, s, y0, y1);
+        a.k_rem[w] = pack_bf16x2(y0, y1);
+      }
+    }
+  }
+  if (t >= a.start && a.tab0 != nullptr) {
+    const size_t r = static_cast<size_t>(t - a.start) * P + i;
+    double sd, cd;
+    sincos(static_cast<double>(pos_primary(a.m, t)) * a.theta[i], &sd, &cd);
+    a.tab0[r] = make_float2(static_cast<float>(cd), static_cast<float>(sd));
+    if (a.tab1 != nullptr) {
+      sincos(static_cast<double>(pos_remote(a.m, t)) * a.theta[i], &sd, &cd);
+      a.tab1[r] = make_float2(static_cast<float>(cd), static_cast<float>(sd));
+    }
+  }
+}
+
 }  // namespace ropeattn

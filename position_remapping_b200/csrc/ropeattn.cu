@@ -440,6 +440,8 @@ int prefill_impl(int stages, const void* q, const void* k, const void* v, float*
   pp.lse = lse;
   pp.B = static_cast<int>(B);
   pp.S = static_cast<int>(S);
+  pp.Sk = static_cast<int>(S);
+  pp.q_off = 0;
   pp.Hq = Hq;
   pp.Hkv = Hkv;
   pp.nqb = static_cast<int>((S + kBlockRows - 1) / kBlockRows);
@@ -452,9 +454,117 @@ int prefill_impl(int stages, const void* q, const void* k, const void* v, float*
   return launch_prefill<64, 8>(tq, tk0, tk1, tv, pp, grid, st);
 }
 
+struct ChunkLayout {
+  size_t off_krem, off_tab0, off_tab1, total;
+  bool remote, tables;
+};
+
+ChunkLayout chunk_layout(int eff_kind, long long B, long long L, long long count, int Hkv, int D) {
+  ChunkLayout c{};
+  c.remote = eff_kind == ROPEATTN_BIFOCAL;
+  c.tables = eff_kind != ROPEATTN_NOPE;
+  size_t off = 0;
+  c.off_krem = off;
+  if (c.remote) off += align_up(static_cast<size_t>(B) * L * Hkv * D * 2, 256);
+  const size_t tab = align_up(static_cast<size_t>(count) * (D / 2) * sizeof(float2), 256);
+  c.off_tab0 = off;
+  if (c.tables) off += tab;
+  c.off_tab1 = off;
+  if (c.remote) off += tab;
+  c.total = off;
+  return c;
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t ropeattn_prefill_chunk_workspace_size(const ropeattn_params* params, int64_t B, int64_t start, int64_t count,
+                                             int32_t Hq, int32_t Hkv, int32_t D) {
+  PosMap m;
+  int eff;
+  if (start < 0 || count < 0 || check_params(params, start + count, D, &m, &eff) ||
+      check_shapes(B, start + count, Hq, Hkv, D))
+    return 0;
+  return chunk_layout(eff, B, start + count, count, Hkv, D).total;
+}
+
+int ropeattn_prefill_chunk(const void* q, const void* k_cache, const void* v_cache, float* out, float* lse,
+                           int64_t B, int64_t start, int64_t count, int32_t Hq, int32_t Hkv, int32_t D,
+                           const ropeattn_params* params, void* workspace, size_t workspace_bytes, void* stream) {
+  g_last_error.clear();
+  if (start < 0 || count < 0) return fail(ROPEATTN_ERR_INVALID_ARG, "start and count must be >= 0");
+  const long long L = start + count;
+  int rc = check_shapes(B, L, Hq, Hkv, D);
+  if (rc) return rc;
+  PosMap m;
+  int eff;
+  rc = check_params(params, L, D, &m, &eff);
+  if (rc) return rc;
+  if (B == 0 || count == 0) return ROPEATTN_OK;
+  if (!q || !k_cache || !v_cache || !out || !lse) return fail(ROPEATTN_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || !aligned16(lse))
+    return fail(ROPEATTN_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if ((static_cast<long long>((count + kBlockRows - 1) / kBlockRows)) * Hq * B > 0x7fffffffLL)
+    return fail(ROPEATTN_ERR_INVALID_ARG, "too many query tiles");
+  rc = check_device();
+  if (rc) return rc;
+  const ChunkLayout lay = chunk_layout(eff, B, L, count, Hkv, D);
+  if (lay.total > 0) {
+    if (!workspace || workspace_bytes < lay.total)
+      return fail(ROPEATTN_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", lay.total,
+                  workspace ? workspace_bytes : size_t(0));
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+      return fail(ROPEATTN_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  m.kind = eff;
+
+  PrefillParams pp{};
+  const void* kmap1 = k_cache;
+  if (lay.tables) {
+    ChunkPrepArgs a{};
+    a.k_cache = static_cast<const uint32_t*>(k_cache);
+    a.k_rem = lay.remote ? reinterpret_cast<uint32_t*>(ws + lay.off_krem) : nullptr;
+    a.tab0 = reinterpret_cast<float2*>(ws + lay.off_tab0);
+    a.tab1 = lay.remote ? reinterpret_cast<float2*>(ws + lay.off_tab1) : nullptr;
+    a.B = static_cast<int>(B);
+    a.L = static_cast<int>(L);
+    a.Hkv = Hkv;
+    a.D = D;
+    a.start = static_cast<int>(start);
+    a.m = m;
+    fill_theta(params, D, a.theta);
+    const int rows = 256 / (D / 2);
+    chunk_prep_kernel<<<static_cast<unsigned>((L + rows - 1) / rows), 256, 0, st>>>(a);
+    CUDA_TRY(cudaGetLastError(), "chunk_prep launch");
+    pp.tab0 = a.tab0;
+    pp.tab1 = a.tab1;
+    if (lay.remote) kmap1 = a.k_rem;
+  }
+  CUtensorMap tq, tk0, tk1, tv;
+  if ((rc = make_map(&tq, q, D, Hq, count, B, 64, kBM, true))) return rc;
+  if ((rc = make_map(&tk0, k_cache, D, Hkv, L, B, 64, kBN, true))) return rc;
+  if ((rc = make_map(&tk1, kmap1, D, Hkv, L, B, 64, kBN, true))) return rc;
+  if ((rc = make_map(&tv, v_cache, D, Hkv, L, B, 64, kBN, true))) return rc;
+  pp.out = out;
+  pp.lse = lse;
+  pp.B = static_cast<int>(B);
+  pp.S = static_cast<int>(count);
+  pp.Sk = static_cast<int>(L);
+  pp.q_off = static_cast<int>(start);
+  pp.Hq = Hq;
+  pp.Hkv = Hkv;
+  pp.nqb = static_cast<int>((count + kBlockRows - 1) / kBlockRows);
+  pp.kind = eff;
+  pp.window = m.window;
+  pp.w0 = m.w0;
+  pp.scale_log2 = scale_log2(params, D);
+  const int grid = pp.nqb * Hq * static_cast<int>(B);
+  if (D == 128) return launch_prefill<128, 4>(tq, tk0, tk1, tv, pp, grid, st);
+  return launch_prefill<64, 8>(tq, tk0, tk1, tv, pp, grid, st);
+}
 
 int ropeattn_prefill(const void* q, const void* k, const void* v, float* out, float* lse, int64_t B, int64_t S,
                      int32_t Hq, int32_t Hkv, int32_t D, const ropeattn_params* params, void* workspace,

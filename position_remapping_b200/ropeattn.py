@@ -23,6 +23,7 @@ ERR_INVALID_ARG, ERR_UNSUPPORTED_DEVICE, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = 
 # every symbol include/ropeattn.h declares
 EXPORTS = ("ropeattn_posmap", "ropeattn_cache_write", "ropeattn_prefill_workspace_size", "ropeattn_prefill",
            "ropeattn_prefill_prepare", "ropeattn_prefill_attend",
+           "ropeattn_prefill_chunk_workspace_size", "ropeattn_prefill_chunk",
            "ropeattn_decode_workspace_size", "ropeattn_decode", "ropeattn_decode_noalloc", "ropeattn_status",
            "ropeattn_last_error", "ropeattn_version")
 
@@ -77,6 +78,9 @@ def _load() -> ctypes.CDLL:
     lib.ropeattn_prefill.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, P, vp, sz, vp]
     lib.ropeattn_prefill_prepare.argtypes = [vp, i64, i64, i32, i32, i32, P, vp, sz, vp]
     lib.ropeattn_prefill_attend.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, P, vp, sz, vp]
+    lib.ropeattn_prefill_chunk_workspace_size.argtypes = [P, i64, i64, i64, i32, i32, i32]
+    lib.ropeattn_prefill_chunk_workspace_size.restype = sz
+    lib.ropeattn_prefill_chunk.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, i32, P, vp, sz, vp]
     lib.ropeattn_decode_workspace_size.argtypes = [i64, i64, i32, i32, i32]
     lib.ropeattn_decode_workspace_size.restype = sz
     lib.ropeattn_decode.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, P, vp, sz, vp]
@@ -86,7 +90,7 @@ def _load() -> ctypes.CDLL:
     lib.ropeattn_last_error.argtypes = []
     lib.ropeattn_last_error.restype = ctypes.c_char_p
     lib.ropeattn_version.argtypes = []
-    for name in ("ropeattn_posmap", "ropeattn_cache_write", "ropeattn_prefill", "ropeattn_prefill_prepare", "ropeattn_prefill_attend",
+    for name in ("ropeattn_posmap", "ropeattn_cache_write", "ropeattn_prefill", "ropeattn_prefill_chunk", "ropeattn_prefill_prepare", "ropeattn_prefill_attend",
                  "ropeattn_decode", "ropeattn_status", "ropeattn_version"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
@@ -193,6 +197,29 @@ def prefill_attend(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, params: Ma
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.ropeattn_prefill_attend(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, S, Hq, Hkv, D,
                                        ctypes.byref(cp), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def prefill_chunk(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, params: MapParams, start: int,
+                  out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, stream=None):
+    """q [B,count,Hq,D] (tokens start..start+count-1), caches [B,start+count,Hkv,D]
+    bf16 holding every key rotated at its own position. Returns
+    (out [B,count,Hq,D] fp32, lse [B,Hq,count] fp32)."""
+    B, count, Hq, D = q.shape
+    Hkv = k_cache.shape[2]
+    assert k_cache.shape[1] == start + count, "the cache must hold exactly start + count rows"
+    if out is None:
+        out = torch.empty((B, count, Hq, D), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, count), dtype=torch.float32, device=q.device)
+    cp = to_cparams(params)
+    if workspace is None:
+        workspace = _workspace(int(lib.ropeattn_prefill_chunk_workspace_size(ctypes.byref(cp), B, int(start), count,
+                                                                               Hq, Hkv, D)), q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.ropeattn_prefill_chunk(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse), B, int(start),
+                                      count, Hq, Hkv, D, ctypes.byref(cp), _ptr(workspace), ws_bytes, _stream(stream)))
+    return out, lse
 
 
 def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, params: MapParams,

@@ -434,3 +434,21 @@ def test_decode_over_growing_cache_crosses_group_changes():
         assert np.allclose(dec[0], pre[0][:, 0], atol=1e-12)
         assert np.allclose(dec[1], pre[1][:, :, 0], atol=1e-12)
     assert Gs == {1, 2, 3, 4}
+
+
+@pytest.mark.parametrize("kind", [O.STANDARD, O.ENDPROMPT, O.PERIODIC, O.NOPE, O.BIFOCAL])
+def test_prefill_from_cache_equals_prefill_rows(kind):
+    # a chunk of rows computed from the Eq. 4 cache (remote keys through the
+    # correction rotation of Eq. 6) equals the same rows of the plain prefill
+    params = {O.STANDARD: MapParams(O.STANDARD, rope_base=1e4),
+              O.ENDPROMPT: MapParams(O.ENDPROMPT, rope_base=5e5, interp=8.0, seg1_len=11, term_start=65500),
+              O.PERIODIC: MapParams(O.PERIODIC, window=5),
+              O.NOPE: MapParams(O.NOPE),
+              O.BIFOCAL: MapParams(O.BIFOCAL, rope_base=1e6, w0=3, w_pretrained=6)}[kind]
+    q, k, v = make_qkv(2, 27, 4, 2, 8, seed=33)
+    qn, kn, vn = O.to_f64(q), O.to_f64(k), O.to_f64(v)
+    cache = O.cache_keys(kn, params)
+    for start in (0, 1, 13, 26):
+        a = O.prefill_from_cache(qn[:, start:], cache, vn, params, start, stage_bf16=False)
+        b = O.prefill(qn, kn, vn, params, rows=list(range(start, 27)), stage_bf16=False)
+        assert np.allclose(a[0], b[0], atol=1e-12) and np.allclose(a[1], b[1], atol=1e-12)
