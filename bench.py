@@ -233,6 +233,58 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+CHUNK = 8192   # tokens of the chunked-prefill measurement (the last rows of the 131072 prefill)
+
+
+def _event_ms(fn, reps, stream):
+    fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def measure_cache_rows(ra, q, k, v, kd, vd, qd, stream):
+    """The decode-cache rows, timed with CUDA events after the main timed
+    region: writing the 131072-token prefill's cache (Eq. 4), the last 8192
+    rows of the same prefill computed from that cache, and one decode step
+    that appends its token to the cache before attending."""
+    P, Dd = PREFILL, DECODE
+    kc = torch.empty_like(k)
+    vc = torch.empty_like(v)
+    w_ms = _event_ms(lambda: ra.cache_write(k, v, kc, vc, P.params, 0, stream=stream), 5, stream)
+    w_bytes = 4 * k.numel() * k.element_size()            # read k, v; write both caches
+    start = P.S - CHUNK
+    qc = q[:, start:].contiguous()
+    ws = torch.empty(ra.prefill_chunk_workspace_size(P.params, P.B, start, CHUNK, P.Hq, P.Hkv, P.D),
+                     dtype=torch.uint8, device=q.device)
+    oc = torch.empty((P.B, CHUNK, P.Hq, P.D), dtype=torch.float32, device=q.device)
+    lc = torch.empty((P.B, P.Hq, CHUNK), dtype=torch.float32, device=q.device)
+    c_ms = _event_ms(lambda: ra.prefill_chunk(qc, kc, vc, P.params, start, out=oc, lse=lc, workspace=ws,
+                                              stream=stream), 3, stream)
+    c_flops = 4.0 * P.D * P.Hq * P.B * sum(range(start + 1, P.S + 1))
+    # decode step with append: the last cached token is rewritten, then attended
+    kn, vn = kd[:, -1:].contiguous(), vd[:, -1:].contiguous()
+    od = torch.empty((Dd.B, Dd.Hq, Dd.D), dtype=torch.float32, device=q.device)
+    ld = torch.empty((Dd.B, Dd.Hq), dtype=torch.float32, device=q.device)
+    wsd = torch.empty(ra.decode_workspace_size(Dd.B, Dd.S, Dd.Hq, Dd.Hkv, Dd.D), dtype=torch.uint8, device=q.device)
+
+    def step():
+        ra.cache_write(kn, vn, kd, vd, Dd.params, Dd.S - 1, stream=stream)
+        ra.decode(qd, kd, vd, Dd.params, out=od, lse=ld, workspace=wsd, stream=stream)
+    s_ms = _event_ms(step, 20, stream)
+    ra.status()
+    return {"cache_write_gbs": w_bytes / (w_ms / 1e3) / 1e9, "cache_write_ms": w_ms,
+            "cache_write_bytes": w_bytes,
+            "prefill_chunk_tflops": c_flops / (c_ms / 1e3) / 1e12, "prefill_chunk_ms": c_ms,
+            "prefill_chunk": f"rows {start}..{P.S - 1} of the {P.S}-token bifocal prefill from its cache",
+            "decode_append_us_per_token": s_ms * 1e3}
+
+
 def config_dict(n_gpus):
     return {"workload": f"{PREFILL.name} + {DECODE.name}",
             "prefill": {"B": PREFILL.B, "S": PREFILL.S, "Hq": PREFILL.Hq, "Hkv": PREFILL.Hkv, "D": PREFILL.D,
@@ -402,6 +454,7 @@ def main():
     e2e_pre_ms = sum(e[0].elapsed_time(e[1]) for e in e_evs)
     e2e_dec_ms = sum(e[1].elapsed_time(e[2]) for e in e_evs)
     ra.status()
+    cache_rows = measure_cache_rows(ra, q, k, v, kd, vd, qd, stream)
 
     total_ms, prep_ms, attn_ms, dec_ms, e2e_pre_ms, e2e_dec_ms = max_over_ranks(
         [total_ms, prep_ms, attn_ms, dec_ms, e2e_pre_ms, e2e_dec_ms], world, dev)
@@ -457,6 +510,7 @@ def main():
                             "algorithmic": f"{decode_bytes(Dd)} B per launch"},
         "clocks": clocks,
         "gpu_launches": 3 * K,
+        "cache_rows": cache_rows,
         "e2e": {"value": job_tflops(world, flops, K, e2e_pre_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "decode_us_per_token": e2e_dec_ms * 1e3 / K},

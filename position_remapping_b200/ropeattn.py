@@ -148,6 +148,11 @@ def prefill_workspace_size(params: MapParams, B, S, Hq, Hkv, D) -> int:
     return int(lib.ropeattn_prefill_workspace_size(ctypes.byref(cp), B, S, Hq, Hkv, D))
 
 
+def prefill_chunk_workspace_size(params: MapParams, B, start, count, Hq, Hkv, D) -> int:
+    cp = to_cparams(params)
+    return int(lib.ropeattn_prefill_chunk_workspace_size(ctypes.byref(cp), B, start, count, Hq, Hkv, D))
+
+
 def decode_workspace_size(B, n, Hq, Hkv, D) -> int:
     return int(lib.ropeattn_decode_workspace_size(B, n, Hq, Hkv, D))
 
@@ -214,8 +219,7 @@ def prefill_chunk(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
         lse = torch.empty((B, Hq, count), dtype=torch.float32, device=q.device)
     cp = to_cparams(params)
     if workspace is None:
-        workspace = _workspace(int(lib.ropeattn_prefill_chunk_workspace_size(ctypes.byref(cp), B, int(start), count,
-                                                                               Hq, Hkv, D)), q.device)
+        workspace = _workspace(prefill_chunk_workspace_size(params, B, int(start), count, Hq, Hkv, D), q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.ropeattn_prefill_chunk(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse), B, int(start),
                                       count, Hq, Hkv, D, ctypes.byref(cp), _ptr(workspace), ws_bytes, _stream(stream)))
