@@ -161,13 +161,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  // work item: longest (last) query blocks first; heads of one block adjacent
-  const int per_blk = p.Hq * p.B;
-  const int qb = p.nqb - 1 - static_cast<int>(blockIdx.x) / per_blk;
-  const int rem = static_cast<int>(blockIdx.x) % per_blk;
-  const int h = rem % p.Hq;
-  const int b = rem / p.Hq;
-  const int hk = h / (p.Hq / p.Hkv);
+  // work item, kv-head-major: all query blocks (longest first) and query
+  // heads of one (batch, kv head) before the next, so the CTAs resident at
+  // any time stream the keys and values of few kv heads and keep them in L2
+  const int grp = p.Hq / p.Hkv;
+  const int per_kv = p.nqb * grp;
+  const int bh = static_cast<int>(blockIdx.x) / per_kv;
+  const int r2 = static_cast<int>(blockIdx.x) % per_kv;
+  const int b = bh / p.Hkv;
+  const int hk = bh % p.Hkv;
+  const int qb = p.nqb - 1 - r2 / grp;
+  const int h = hk * grp + r2 % grp;
   const int q0 = qb * kBlockRows;
 
   PassDesc passes[2];
