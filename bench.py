@@ -19,6 +19,7 @@ oracle on a bounded sample of the same workload instead.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -285,6 +286,29 @@ def measure_cache_rows(ra, q, k, v, kd, vd, qd, stream):
             "decode_append_us_per_token": s_ms * 1e3}
 
 
+def measure_comparators(ra, q, k, v, out, lse, ws, stream):
+    """Same-box comparators of the fused bifocal prefill (CUDA events, after
+    the timed regions): the same attention kernel with standard RoPE on the
+    same shapes (the unmodified-model reference), and the literal three-call
+    bifocal route with a separate merge kernel. Ratios are throughput
+    relative to standard RoPE, as the pages report against their baseline."""
+    P = PREFILL
+    std = P.params.replace(kind=0)
+    std_ms = _event_ms(lambda: ra.prefill(q, k, v, std, out=out, lse=lse, workspace=ws, stream=stream), 2, stream)
+    fused_ms = _event_ms(lambda: ra.prefill(q, k, v, P.params, out=out, lse=lse, workspace=ws, stream=stream), 2,
+                         stream)
+    ws3 = torch.empty(int(ra.lib.ropeattn_prefill_three_call_workspace_size(
+        ctypes.byref(ra.to_cparams(P.params)), P.B, P.S, P.Hq, P.Hkv, P.D)), dtype=torch.uint8, device=q.device)
+    three_ms = _event_ms(lambda: ra.prefill_three_call(q, k, v, P.params, out=out, lse=lse, workspace=ws3,
+                                                       stream=stream), 2, stream)
+    del ws3
+    ra.status()
+    return {"standard_rope_prefill_ms": std_ms, "fused_bifocal_prefill_ms": fused_ms,
+            "three_call_bifocal_prefill_ms": three_ms,
+            "fused_vs_standard": std_ms / fused_ms, "three_call_vs_standard": std_ms / three_ms,
+            "note": "prepare + attend, 131072 tokens, 32/8 heads, D 128; ratio = standard time / time"}
+
+
 def config_dict(n_gpus):
     return {"workload": f"{PREFILL.name} + {DECODE.name}",
             "prefill": {"B": PREFILL.B, "S": PREFILL.S, "Hq": PREFILL.Hq, "Hkv": PREFILL.Hkv, "D": PREFILL.D,
@@ -455,6 +479,7 @@ def main():
     e2e_dec_ms = sum(e[1].elapsed_time(e[2]) for e in e_evs)
     ra.status()
     cache_rows = measure_cache_rows(ra, q, k, v, kd, vd, qd, stream)
+    comparators = measure_comparators(ra, q, k, v, out, lse, ws, stream)
 
     total_ms, prep_ms, attn_ms, dec_ms, e2e_pre_ms, e2e_dec_ms = max_over_ranks(
         [total_ms, prep_ms, attn_ms, dec_ms, e2e_pre_ms, e2e_dec_ms], world, dev)
@@ -511,6 +536,7 @@ def main():
         "clocks": clocks,
         "gpu_launches": 3 * K,
         "cache_rows": cache_rows,
+        "comparators": comparators,
         "e2e": {"value": job_tflops(world, flops, K, e2e_pre_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "decode_us_per_token": e2e_dec_ms * 1e3 / K},

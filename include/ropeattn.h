@@ -187,6 +187,24 @@ int ropeattn_prefill_chunk(const void* q, const void* k_cache, const void* v_cac
                            const ropeattn_params* params, void* workspace, size_t workspace_bytes,
                            void* stream);
 
+/* Comparator: the literal three-call bifocal prefill of Jet-Long §3.3 with a
+ * separate merge kernel, on the same attention kernel: (A) sliding window
+ * w0 at exact positions, (B) full causal at remote positions, (C) sliding
+ * window w0 at remote positions, each writing its normalised output and
+ * LSE, then O = (W_A O_A + W_B O_B - W_C O_C) / (W_A + W_B - W_C) with
+ * W_X = exp(l_X - M), M = max l_X (Eq. 7), in fp32. Same result as
+ * ropeattn_prefill up to rounding; exists to time the fused kernel against
+ * the unfused route on the same GPU. Needs an effective bifocal map (G > 1
+ * and w0 < S-1), else INVALID_ARG. Arguments and layouts as ropeattn_prefill;
+ * the workspace also holds O_A, O_C and their LSEs (2 (B S Hq D + B Hq S)
+ * floats more). Errors: INVALID_ARG, UNSUPPORTED_DEVICE, WORKSPACE, CUDA. */
+size_t ropeattn_prefill_three_call_workspace_size(const ropeattn_params* params, int64_t B, int64_t S,
+                                                  int32_t Hq, int32_t Hkv, int32_t D);
+int ropeattn_prefill_three_call(const void* q, const void* k, const void* v, float* out, float* lse,
+                                int64_t B, int64_t S, int32_t Hq, int32_t Hkv, int32_t D,
+                                const ropeattn_params* params, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
 /* Bytes of device workspace ropeattn_decode needs (split-KV partials and
  * per-head arrival counters). Depends on the current device's SM count. */
 size_t ropeattn_decode_workspace_size(int64_t B, int64_t n, int32_t Hq,

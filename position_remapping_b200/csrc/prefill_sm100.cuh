@@ -70,6 +70,9 @@ struct PrefillParams {
   int window;          // Periodic RoPE
   int w0;              // Jet-Long
   float scale_log2;    // softmax scale * log2(e)
+  // one forced pass (the separate calls of the literal three-call bifocal
+  // prefill): band hi <= t - s <= lo with query/key map sel; 0 = off
+  int forced, forced_lo, forced_hi, forced_sel;
 };
 
 struct PassDesc {
@@ -81,7 +84,10 @@ struct PassDesc {
 __device__ __forceinline__ int make_passes(const PrefillParams& p, int q0, PassDesc* ps) {
   int bands[2][3];  // lo_off, hi_off, sel
   int nb = 0;
-  if (p.kind == kBifocal) {
+  if (p.forced) {
+    bands[0][0] = p.forced_lo; bands[0][1] = p.forced_hi; bands[0][2] = p.forced_sel;
+    nb = 1;
+  } else if (p.kind == kBifocal) {
     bands[0][0] = kInf; bands[0][1] = p.w0 + 1; bands[0][2] = 1;
     bands[1][0] = p.w0; bands[1][1] = 0; bands[1][2] = 0;
     nb = 2;

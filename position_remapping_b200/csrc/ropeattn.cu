@@ -13,6 +13,7 @@
 #include "common.cuh"
 #include "cache.cuh"
 #include "decode_sm100.cuh"
+#include "merge.cuh"
 #include "posmap.cuh"
 #include "prefill_sm100.cuh"
 #include "prep.cuh"
@@ -564,6 +565,122 @@ int ropeattn_prefill_chunk(const void* q, const void* k_cache, const void* v_cac
   const int grid = pp.nqb * Hq * static_cast<int>(B);
   if (D == 128) return launch_prefill<128, 4>(tq, tk0, tk1, tv, pp, grid, st);
   return launch_prefill<64, 8>(tq, tk0, tk1, tv, pp, grid, st);
+}
+
+size_t ropeattn_prefill_three_call_workspace_size(const ropeattn_params* params, int64_t B, int64_t S, int32_t Hq,
+                                                  int32_t Hkv, int32_t D) {
+  PosMap m;
+  int eff;
+  if (check_params(params, S, D, &m, &eff) || check_shapes(B, S, Hq, Hkv, D) || eff != ROPEATTN_BIFOCAL) return 0;
+  const size_t o = align_up(static_cast<size_t>(B) * S * Hq * D * sizeof(float), 256);
+  const size_t l = align_up(static_cast<size_t>(B) * Hq * S * sizeof(float), 256);
+  return prefill_layout(eff, B, S, Hkv, D).total + 2 * o + 2 * l;
+}
+
+int ropeattn_prefill_three_call(const void* q, const void* k, const void* v, float* out, float* lse, int64_t B,
+                                int64_t S, int32_t Hq, int32_t Hkv, int32_t D, const ropeattn_params* params,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  g_last_error.clear();
+  int rc = check_shapes(B, S, Hq, Hkv, D);
+  if (rc) return rc;
+  PosMap m;
+  int eff;
+  rc = check_params(params, S, D, &m, &eff);
+  if (rc) return rc;
+  if (eff != ROPEATTN_BIFOCAL)
+    return fail(ROPEATTN_ERR_INVALID_ARG, "the three-call prefill needs a bifocal map with G > 1 and w0 < S-1");
+  if (B == 0 || S == 0) return ROPEATTN_OK;
+  if (!q || !k || !v || !out || !lse) return fail(ROPEATTN_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return fail(ROPEATTN_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if ((static_cast<long long>((S + kBlockRows - 1) / kBlockRows)) * Hq * B > 0x7fffffffLL)
+    return fail(ROPEATTN_ERR_INVALID_ARG, "too many query tiles");
+  rc = check_device();
+  if (rc) return rc;
+  const PrefillLayout lay = prefill_layout(eff, B, S, Hkv, D);
+  const size_t obytes = align_up(static_cast<size_t>(B) * S * Hq * D * sizeof(float), 256);
+  const size_t lbytes = align_up(static_cast<size_t>(B) * Hq * S * sizeof(float), 256);
+  const size_t need = lay.total + 2 * obytes + 2 * lbytes;
+  if (!workspace || workspace_bytes < need)
+    return fail(ROPEATTN_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need,
+                workspace ? workspace_bytes : size_t(0));
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+    return fail(ROPEATTN_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  m.kind = eff;
+  float* oA = reinterpret_cast<float*>(ws + lay.total);
+  float* oC = reinterpret_cast<float*>(ws + lay.total + obytes);
+  float* lA = reinterpret_cast<float*>(ws + lay.total + 2 * obytes);
+  float* lC = reinterpret_cast<float*>(ws + lay.total + 2 * obytes + lbytes);
+
+  // keys rotated to both maps and the query angle tables, as in the fused prefill
+  PrepArgs a{};
+  a.k = static_cast<const uint32_t*>(k);
+  a.k_rot0 = reinterpret_cast<uint32_t*>(ws + lay.off_krot[0]);
+  a.k_rot1 = reinterpret_cast<uint32_t*>(ws + lay.off_krot[1]);
+  a.tab0 = reinterpret_cast<float2*>(ws + lay.off_tab[0]);
+  a.tab1 = reinterpret_cast<float2*>(ws + lay.off_tab[1]);
+  a.B = static_cast<int>(B);
+  a.S = static_cast<int>(S);
+  a.Hkv = Hkv;
+  a.D = D;
+  a.m = m;
+  fill_theta(params, D, a.theta);
+  const int prow = 256 / (D / 2);
+  rope_prep_kernel<<<static_cast<unsigned>((S + prow - 1) / prow), 256, 0, st>>>(a);
+  CUDA_TRY(cudaGetLastError(), "rope_prep launch");
+
+  CUtensorMap tq, tk0, tk1, tv;
+  if ((rc = make_map(&tq, q, D, Hq, S, B, 64, kBM, true))) return rc;
+  if ((rc = make_map(&tk0, a.k_rot0, D, Hkv, S, B, 64, kBN, true))) return rc;
+  if ((rc = make_map(&tk1, a.k_rot1, D, Hkv, S, B, 64, kBN, true))) return rc;
+  if ((rc = make_map(&tv, v, D, Hkv, S, B, 64, kBN, true))) return rc;
+  PrefillParams pp{};
+  pp.tab0 = a.tab0;
+  pp.tab1 = a.tab1;
+  pp.B = static_cast<int>(B);
+  pp.S = static_cast<int>(S);
+  pp.Sk = static_cast<int>(S);
+  pp.q_off = 0;
+  pp.Hq = Hq;
+  pp.Hkv = Hkv;
+  pp.nqb = static_cast<int>((S + kBlockRows - 1) / kBlockRows);
+  pp.kind = ROPEATTN_STANDARD;   // each call writes its own normalised output and LSE
+  pp.window = m.window;
+  pp.w0 = m.w0;
+  pp.scale_log2 = scale_log2(params, D);
+  pp.forced = 1;
+  const int grid = pp.nqb * Hq * static_cast<int>(B);
+  // (A) sliding window w0, exact positions; (B) full causal, remote positions;
+  // (C) sliding window w0, remote positions (Jet-Long §3.3)
+  const int calls[3][3] = {{m.w0, 0, 0}, {kInf, 0, 1}, {m.w0, 0, 1}};
+  float* outs[3] = {oA, out, oC};
+  float* lses[3] = {lA, lse, lC};
+  for (int c = 0; c < 3; ++c) {
+    pp.forced_lo = calls[c][0];
+    pp.forced_hi = calls[c][1];
+    pp.forced_sel = calls[c][2];
+    pp.out = outs[c];
+    pp.lse = lses[c];
+    rc = D == 128 ? launch_prefill<128, 4>(tq, tk0, tk1, tv, pp, grid, st)
+                  : launch_prefill<64, 8>(tq, tk0, tk1, tv, pp, grid, st);
+    if (rc) return rc;
+  }
+  MergeArgs ma{};
+  ma.oA = oA;
+  ma.oC = oC;
+  ma.out = out;
+  ma.lA = lA;
+  ma.lC = lC;
+  ma.lse = lse;
+  ma.rows = static_cast<long long>(B) * S * Hq;
+  ma.S = static_cast<int>(S);
+  ma.Hq = Hq;
+  ma.D = D;
+  three_call_merge_kernel<<<static_cast<unsigned>((ma.rows * 32 + 255) / 256), 256, 0, st>>>(ma);
+  CUDA_TRY(cudaGetLastError(), "merge launch");
+  return ROPEATTN_OK;
 }
 
 int ropeattn_prefill(const void* q, const void* k, const void* v, float* out, float* lse, int64_t B, int64_t S,

@@ -24,6 +24,7 @@ ERR_INVALID_ARG, ERR_UNSUPPORTED_DEVICE, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = 
 EXPORTS = ("ropeattn_posmap", "ropeattn_cache_write", "ropeattn_prefill_workspace_size", "ropeattn_prefill",
            "ropeattn_prefill_prepare", "ropeattn_prefill_attend",
            "ropeattn_prefill_chunk_workspace_size", "ropeattn_prefill_chunk",
+           "ropeattn_prefill_three_call_workspace_size", "ropeattn_prefill_three_call",
            "ropeattn_decode_workspace_size", "ropeattn_decode", "ropeattn_decode_noalloc", "ropeattn_status",
            "ropeattn_last_error", "ropeattn_version")
 
@@ -81,6 +82,9 @@ def _load() -> ctypes.CDLL:
     lib.ropeattn_prefill_chunk_workspace_size.argtypes = [P, i64, i64, i64, i32, i32, i32]
     lib.ropeattn_prefill_chunk_workspace_size.restype = sz
     lib.ropeattn_prefill_chunk.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, i32, P, vp, sz, vp]
+    lib.ropeattn_prefill_three_call_workspace_size.argtypes = [P, i64, i64, i32, i32, i32]
+    lib.ropeattn_prefill_three_call_workspace_size.restype = sz
+    lib.ropeattn_prefill_three_call.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, P, vp, sz, vp]
     lib.ropeattn_decode_workspace_size.argtypes = [i64, i64, i32, i32, i32]
     lib.ropeattn_decode_workspace_size.restype = sz
     lib.ropeattn_decode.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, P, vp, sz, vp]
@@ -90,7 +94,8 @@ def _load() -> ctypes.CDLL:
     lib.ropeattn_last_error.argtypes = []
     lib.ropeattn_last_error.restype = ctypes.c_char_p
     lib.ropeattn_version.argtypes = []
-    for name in ("ropeattn_posmap", "ropeattn_cache_write", "ropeattn_prefill", "ropeattn_prefill_chunk", "ropeattn_prefill_prepare", "ropeattn_prefill_attend",
+    for name in ("ropeattn_posmap", "ropeattn_cache_write", "ropeattn_prefill", "ropeattn_prefill_chunk",
+                 "ropeattn_prefill_three_call", "ropeattn_prefill_prepare", "ropeattn_prefill_attend",
                  "ropeattn_decode", "ropeattn_status", "ropeattn_version"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
@@ -181,6 +186,27 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, params: MapParams
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.ropeattn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, S, Hq, Hkv, D,
                                 ctypes.byref(cp), _ptr(workspace), ws_bytes, _stream(stream)))
+    return out, lse
+
+
+def prefill_three_call(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, params: MapParams,
+                       out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None, stream=None):
+    """Comparator: the literal three-call bifocal prefill with a separate
+    merge kernel (same layouts as prefill)."""
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if out is None:
+        out = torch.empty((B, S, Hq, D), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
+    cp = to_cparams(params)
+    if workspace is None:
+        workspace = _workspace(int(lib.ropeattn_prefill_three_call_workspace_size(ctypes.byref(cp), B, S, Hq, Hkv, D)),
+                               q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.ropeattn_prefill_three_call(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, S, Hq, Hkv, D,
+                                           ctypes.byref(cp), _ptr(workspace), ws_bytes, _stream(stream)))
     return out, lse
 
 
