@@ -73,14 +73,17 @@ typedef enum {
  * except the reserved ones, which must be zero. */
 typedef struct ropeattn_params {
   int32_t kind;           /* ropeattn_kind */
-  int32_t reserved0;      /* must be 0 */
+  int32_t fixed_group;    /* BIFOCAL: 0 -> G = max(1, ceil(L / w_pretrained)) (Jet-Long
+                             Eq. 2, the dynamic schedule); > 0 -> this G for every L (a
+                             single group size fixed up front, as the grouped-window
+                             baselines Jet-Long contrasts itself with). Others: 0. */
   double  rope_base;      /* Theta > 1 (e.g. 1e4, 5e5, 1e6) */
   double  interp;         /* ENDPROMPT: interpolation factor s >= 1 (others: ignored) */
   int64_t seg1_len;       /* ENDPROMPT: n1 >= 0, length of the intact first segment */
   int64_t term_start;     /* ENDPROMPT: first position of the terminal segment, >= 0 */
   int64_t window;         /* PERIODIC: W >= 1 (window length = period) */
   int64_t w0;             /* BIFOCAL: local window, >= 0 (0 = the token itself only) */
-  int64_t w_pretrained;   /* BIFOCAL: pretrained context window, >= 1 */
+  int64_t w_pretrained;   /* BIFOCAL: pretrained context window, >= 1 (unused with fixed_group) */
   float   softmax_scale;  /* > 0 to override; 0 -> 1/sqrt(D) */
   int32_t reserved[3];    /* must be 0 */
 } ropeattn_params;

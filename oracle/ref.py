@@ -51,7 +51,7 @@ STANDARD, ENDPROMPT, PERIODIC, NOPE, BIFOCAL = 0, 1, 2, 3, 4
 __all__ = [
     "STANDARD", "ENDPROMPT", "PERIODIC", "NOPE", "BIFOCAL",
     "round_bf16", "rope_frequencies", "rotation_matrix", "rotate",
-    "periodic_position", "endprompt_position", "group_size", "remote_position",
+    "periodic_position", "endprompt_position", "group_size", "bifocal_group", "remote_position",
     "position_maps", "softmax_scale", "prefill", "prefill_three_call",
     "decode", "cache_keys", "prefill_from_cache", "brute_prefill", "brute_decode", "to_f64",
 ]
@@ -143,6 +143,14 @@ def group_size(L: int, w_pretrained: int) -> int:
     return max(1, -(-int(L) // int(w_pretrained)))
 
 
+def bifocal_group(params, L: int) -> int:
+    """G of a BIFOCAL map for length L: the dynamic schedule of Eq. 2, or a
+    single group size fixed up front (``fixed_group`` > 0), the grouping the
+    baselines Jet-Long compares against use (Jet-Long §2.2)."""
+    fixed = int(getattr(params, "fixed_group", 0) or 0)
+    return fixed if fixed > 0 else group_size(L, params.w_pretrained)
+
+
 def remote_position(t, G: int):
     """Jet-Long §3.1 Eq. 3: f(x) = floor(x / G)."""
     return np.asarray(t, dtype=np.int64) // int(G)
@@ -165,7 +173,7 @@ def position_maps(params, L: int):
     if k == NOPE:
         return np.zeros_like(t), None, 1
     if k == BIFOCAL:
-        G = group_size(L, params.w_pretrained)
+        G = bifocal_group(params, L)
         return t, remote_position(t, G), G
     raise ValueError(f"unknown kind {k}")
 
@@ -260,7 +268,7 @@ def prefill_three_call(q, k, v, params, stage_bf16: bool = True):
     grp = Hq // Hkv
     scale = softmax_scale(D, params)
     freqs = _freqs(params, D)
-    G = group_size(S, params.w_pretrained)
+    G = bifocal_group(params, S)
     t = np.arange(S)
     f = remote_position(t, G)
     stage = round_bf16 if stage_bf16 else (lambda a: a)
@@ -415,7 +423,8 @@ def _brute_positions(params, t: int, s: int, L: int, D: int):
         return pos(t), pos(s)
     if kind == PERIODIC:
         return t % params.window, s % params.window
-    G = max(1, math.ceil(L / params.w_pretrained))
+    fixed = int(getattr(params, "fixed_group", 0) or 0)
+    G = fixed if fixed > 0 else max(1, math.ceil(L / params.w_pretrained))
     if t - s <= params.w0:
         return t, s
     return t // G, s // G

@@ -114,8 +114,10 @@ constexpr long long kMaxPos = 0x7fffffffLL;
 // "reduces to the unmodified base model").
 int check_params(const ropeattn_params* p, long long L, int D, PosMap* m, int* eff_kind) {
   if (!p) return fail(ROPEATTN_ERR_INVALID_ARG, "params is NULL");
-  if (p->reserved0 != 0 || p->reserved[0] != 0 || p->reserved[1] != 0 || p->reserved[2] != 0)
+  if (p->reserved[0] != 0 || p->reserved[1] != 0 || p->reserved[2] != 0)
     return fail(ROPEATTN_ERR_INVALID_ARG, "reserved fields must be 0");
+  if (p->fixed_group < 0 || p->fixed_group > (1 << 30) || (p->fixed_group != 0 && p->kind != ROPEATTN_BIFOCAL))
+    return fail(ROPEATTN_ERR_INVALID_ARG, "fixed_group must be 0, or in [1, 2^30] for BIFOCAL");
   if (p->kind < ROPEATTN_STANDARD || p->kind > ROPEATTN_BIFOCAL)
     return fail(ROPEATTN_ERR_INVALID_ARG, "unknown kind %d", p->kind);
   if (p->kind != ROPEATTN_NOPE && !(p->rope_base > 1.0 && std::isfinite(p->rope_base)))
@@ -142,8 +144,9 @@ int check_params(const ropeattn_params* p, long long L, int D, PosMap* m, int* e
       break;
     case ROPEATTN_BIFOCAL: {
       if (p->w0 < 0) return fail(ROPEATTN_ERR_INVALID_ARG, "w0 must be >= 0");
-      if (p->w_pretrained < 1) return fail(ROPEATTN_ERR_INVALID_ARG, "w_pretrained must be >= 1");
-      m->G = group_size(L, p->w_pretrained);
+      if (p->fixed_group == 0 && p->w_pretrained < 1)
+        return fail(ROPEATTN_ERR_INVALID_ARG, "w_pretrained must be >= 1");
+      m->G = p->fixed_group > 0 ? p->fixed_group : group_size(L, p->w_pretrained);
       m->w0 = static_cast<int>(p->w0 < (1LL << 30) ? p->w0 : (1LL << 30));
       if (m->G == 1 || p->w0 >= L - 1) *eff_kind = ROPEATTN_STANDARD;
       break;

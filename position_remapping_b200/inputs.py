@@ -38,6 +38,7 @@ class MapParams:
     window: int = 0              # Periodic RoPE: window W (= period)
     w0: int = 0                  # Jet-Long: local window
     w_pretrained: int = 0        # Jet-Long: pretrained context window
+    fixed_group: int = 0         # bifocal with one fixed group size G (0: G from L, Eq. 2)
     softmax_scale: float = 0.0   # 0 -> 1/sqrt(D)
 
     def replace(self, **kw) -> "MapParams":

@@ -39,7 +39,7 @@ class CParams(ctypes.Structure):
     """Mirror of ``ropeattn_params``."""
     _fields_ = [
         ("kind", ctypes.c_int32),
-        ("reserved0", ctypes.c_int32),
+        ("fixed_group", ctypes.c_int32),
         ("rope_base", ctypes.c_double),
         ("interp", ctypes.c_double),
         ("seg1_len", ctypes.c_int64),
@@ -55,6 +55,7 @@ class CParams(ctypes.Structure):
 def to_cparams(p: MapParams) -> CParams:
     c = CParams()
     c.kind = int(p.kind)
+    c.fixed_group = int(p.fixed_group)
     c.rope_base = float(p.rope_base)
     c.interp = float(p.interp)
     c.seg1_len = int(p.seg1_len)

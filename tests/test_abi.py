@@ -50,8 +50,9 @@ def test_param_struct_layout_matches_c(ra):
 #include <stddef.h>
 #include "ropeattn.h"
 int main(void) {
-  printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(ropeattn_params),
-    offsetof(ropeattn_params, kind), offsetof(ropeattn_params, rope_base), offsetof(ropeattn_params, interp),
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(ropeattn_params),
+    offsetof(ropeattn_params, kind), offsetof(ropeattn_params, fixed_group),
+    offsetof(ropeattn_params, rope_base), offsetof(ropeattn_params, interp),
     offsetof(ropeattn_params, seg1_len), offsetof(ropeattn_params, term_start), offsetof(ropeattn_params, window),
     offsetof(ropeattn_params, w0), offsetof(ropeattn_params, w_pretrained), offsetof(ropeattn_params, softmax_scale),
     offsetof(ropeattn_params, reserved));
@@ -66,7 +67,7 @@ int main(void) {
         got = list(map(int, subprocess.run([exe], capture_output=True, text=True).stdout.split()))
     P = ra.CParams
     want = [ctypes.sizeof(P)] + [getattr(P, f).offset for f in
-            ("kind", "rope_base", "interp", "seg1_len", "term_start", "window", "w0", "w_pretrained",
+            ("kind", "fixed_group", "rope_base", "interp", "seg1_len", "term_start", "window", "w0", "w_pretrained",
              "softmax_scale", "reserved")]
     assert got == want
 

@@ -26,6 +26,8 @@ SMALL = [
     ("bifocal_g4_d64_grp4", 2, 4097, 8, 2, 64, MapParams(O.BIFOCAL, rope_base=1e4, w0=300, w_pretrained=1100)),
     ("bifocal_g8_d128", 1, 8000, 4, 4, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=2048, w_pretrained=1000)),
     ("bifocal_g2_edge_local", 1, 3000, 2, 1, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=2900, w_pretrained=1500)),
+    ("bifocal_fixed_g5_phasor", 1, 3000, 4, 2, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=200, fixed_group=5)),
+    ("bifocal_fixed_g4_table", 1, 5000, 8, 4, 128, MapParams(O.BIFOCAL, rope_base=1e4, w0=300, fixed_group=4)),
 ]
 
 

@@ -452,3 +452,23 @@ def test_prefill_from_cache_equals_prefill_rows(kind):
         a = O.prefill_from_cache(qn[:, start:], cache, vn, params, start, stage_bf16=False)
         b = O.prefill(qn, kn, vn, params, rows=list(range(start, 27)), stage_bf16=False)
         assert np.allclose(a[0], b[0], atol=1e-12) and np.allclose(a[1], b[1], atol=1e-12)
+
+
+def test_fixed_group_positions_and_brute_force():
+    # a single group size fixed up front: G does not follow L (Jet-Long §2.2
+    # contrasts its dynamic G with this); f(t) = floor(t / G) as in Eq. 3
+    for L in (5, 100, 10000):
+        p = MapParams(O.BIFOCAL, rope_base=1e4, w0=3, fixed_group=3)
+        loc, rem, G = O.position_maps(p, L)
+        assert G == 3 and np.array_equal(rem, np.arange(L) // 3) and np.array_equal(loc, np.arange(L))
+    assert O.bifocal_group(MapParams(O.BIFOCAL, w_pretrained=8), 20) == O.group_size(20, 8) == 3
+    params = MapParams(O.BIFOCAL, rope_base=1e4, w0=2, fixed_group=5)
+    q, k, v = make_qkv(1, 17, 2, 1, 8, seed=34)
+    a = O.prefill(q, k, v, params, stage_bf16=False)
+    b = O.brute_prefill(q, k, v, params)
+    assert np.allclose(a[0], b[0], atol=1e-12) and np.allclose(a[1], b[1], atol=1e-12)
+    qd, kd, vd = make_qkv(1, 17, 2, 1, 8, seed=35, q_len=1)
+    qn, kn, vn = O.to_f64(qd), O.to_f64(kd), O.to_f64(vd)
+    c = O.decode(qn, _cache(kn, params, 8), vn, params)
+    d = O.brute_decode(qn, kn, vn, params)
+    assert np.allclose(c[0], d[0], atol=1e-12) and np.allclose(c[1], d[1], atol=1e-12)

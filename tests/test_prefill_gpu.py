@@ -19,6 +19,8 @@ pytestmark = pytest.mark.gpu
 
 SMALL = [
     # (id, B, S, Hq, Hkv, D, params)
+    ("bifocal_fixed_g5", 1, 1000, 4, 2, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=100, fixed_group=5)),
+    ("bifocal_fixed_g2_d64", 2, 700, 2, 1, 64, MapParams(O.BIFOCAL, rope_base=1e4, w0=30, fixed_group=2)),
     ("standard_s512_d64", 1, 512, 1, 1, 64, MapParams(O.STANDARD, rope_base=1e4)),
     ("standard_ragged_gqa", 2, 300, 4, 2, 128, MapParams(O.STANDARD, rope_base=1e4)),
     ("standard_s1", 1, 1, 2, 1, 64, MapParams(O.STANDARD)),
