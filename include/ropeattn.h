@@ -256,6 +256,15 @@ int ropeattn_decode_noalloc(const void* q, const void* k_cache, const void* v_ca
                             int64_t B, int64_t n, int32_t Hq, int32_t Hkv, int32_t D,
                             const ropeattn_params* params, void* stream);
 
+/* Failure-detection self-test: launches one CTA whose mbarrier wait nothing
+ * completes, bounded by limit_ns (1e3..1e9 ns), through the same bounded
+ * wait every kernel uses. When the wait runs out the kernel sets the device
+ * status word and returns; *d_result (device int32) receives 0 (gave up) or
+ * 1 (completed, which cannot happen). The next ropeattn_status() reports
+ * ROPEATTN_ERR_TIMEOUT; the context stays usable. No fault is involved.
+ * Errors: INVALID_ARG, UNSUPPORTED_DEVICE, CUDA. */
+int ropeattn_wait_selftest(int64_t limit_ns, int32_t* d_result, void* stream);
+
 /* Reads and clears the device status word of the current device (waits for
  * the device to be idle first). Returns ROPEATTN_OK, or ROPEATTN_ERR_TIMEOUT
  * if any kernel since the last call gave up on a bounded wait (its outputs

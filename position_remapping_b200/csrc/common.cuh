@@ -63,10 +63,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase of `bar` with the given parity to complete. Gives up
-// after kWaitLimitNs, or as soon as *abort is set by another thread of the
-// CTA; on giving up it records the timeout in g_status and sets *abort.
-// Returns true when the phase completed.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// after limit_ns, or as soon as *abort is set by another thread of the CTA;
+// on giving up it records the timeout in g_status and sets *abort. Returns
+// true when the phase completed.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   unsigned long long t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
@@ -76,7 +77,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       const unsigned long long dt = globaltimer_ns() - t0;
       // after 10 ms also give up if another CTA has already timed out, so a
       // failing launch ends after one wait limit instead of one per wave
-      if (dt > kWaitLimitNs || (dt > 10000000ull && *reinterpret_cast<volatile int*>(&g_status) != 0)) {
+      if (dt > limit_ns || (dt > 10000000ull && *reinterpret_cast<volatile int*>(&g_status) != 0)) {
         atomicOr(&g_status, kStatusTimeout);
         *abort = 1;
         return false;

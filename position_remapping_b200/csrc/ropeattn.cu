@@ -14,6 +14,7 @@
 #include "cache.cuh"
 #include "decode_sm100.cuh"
 #include "merge.cuh"
+#include "selftest.cuh"
 #include "posmap.cuh"
 #include "prefill_sm100.cuh"
 #include "prep.cuh"
@@ -283,6 +284,19 @@ extern "C" {
 const char* ropeattn_last_error(void) { return g_last_error.c_str(); }
 
 int ropeattn_version(void) { return kVersion; }
+
+int ropeattn_wait_selftest(int64_t limit_ns, int32_t* d_result, void* stream) {
+  g_last_error.clear();
+  if (limit_ns < 1000 || limit_ns > 1000000000LL)
+    return fail(ROPEATTN_ERR_INVALID_ARG, "limit_ns must be in [1e3, 1e9]");
+  if (!d_result) return fail(ROPEATTN_ERR_INVALID_ARG, "d_result is NULL");
+  int rc = check_device();
+  if (rc) return rc;
+  wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<unsigned long long>(limit_ns),
+                                                                      d_result);
+  CUDA_TRY(cudaGetLastError(), "selftest launch");
+  return ROPEATTN_OK;
+}
 
 int ropeattn_status(void) {
   g_last_error.clear();

@@ -26,6 +26,7 @@ EXPORTS = ("ropeattn_posmap", "ropeattn_cache_write", "ropeattn_prefill_workspac
            "ropeattn_prefill_chunk_workspace_size", "ropeattn_prefill_chunk",
            "ropeattn_prefill_three_call_workspace_size", "ropeattn_prefill_three_call",
            "ropeattn_decode_workspace_size", "ropeattn_decode", "ropeattn_decode_noalloc", "ropeattn_status",
+           "ropeattn_wait_selftest",
            "ropeattn_last_error", "ropeattn_version")
 
 
@@ -92,6 +93,8 @@ def _load() -> ctypes.CDLL:
     lib.ropeattn_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, P, vp]
     lib.ropeattn_decode_noalloc.restype = ctypes.c_int
     lib.ropeattn_status.argtypes = []
+    lib.ropeattn_wait_selftest.argtypes = [i64, vp, vp]
+    lib.ropeattn_wait_selftest.restype = ctypes.c_int
     lib.ropeattn_last_error.argtypes = []
     lib.ropeattn_last_error.restype = ctypes.c_char_p
     lib.ropeattn_version.argtypes = []
@@ -122,6 +125,14 @@ def _ptr(t: Optional[torch.Tensor]):
 
 def version() -> int:
     return lib.ropeattn_version()
+
+
+def wait_selftest(limit_ns: int = 1_000_000, stream=None) -> int:
+    """Runs the bounded-wait self-test; returns the device result (0: the
+    wait gave up, as it must). Follow with status() to read the timeout."""
+    res = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    _check(lib.ropeattn_wait_selftest(int(limit_ns), _ptr(res), _stream(stream)))
+    return int(res.item())
 
 
 def status() -> None:
