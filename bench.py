@@ -309,6 +309,30 @@ def measure_comparators(ra, q, k, v, out, lse, ws, stream):
             "note": "prepare + attend, 131072 tokens, 32/8 heads, D 128; ratio = standard time / time"}
 
 
+def measure_decode_comparators(ra, qd, kd, vd, stream):
+    """Decode comparators on the 131072-key cache (CUDA events, after the
+    timed regions): the fused bifocal decode, the same decode with the
+    correction rotation as a separate pass over the cache, and standard RoPE
+    on the same cache (the unmodified-model reference)."""
+    Dd = DECODE
+    od = torch.empty((Dd.B, Dd.Hq, Dd.D), dtype=torch.float32, device=qd.device)
+    ld = torch.empty((Dd.B, Dd.Hq), dtype=torch.float32, device=qd.device)
+    wsd = torch.empty(ra.decode_workspace_size(Dd.B, Dd.S, Dd.Hq, Dd.Hkv, Dd.D), dtype=torch.uint8, device=qd.device)
+    wsu = torch.empty(int(ra.lib.ropeattn_decode_unfused_workspace_size(Dd.B, Dd.S, Dd.Hq, Dd.Hkv, Dd.D)),
+                      dtype=torch.uint8, device=qd.device)
+    std = Dd.params.replace(kind=0)
+    fused_us = 1e3 * _event_ms(lambda: ra.decode(qd, kd, vd, Dd.params, out=od, lse=ld, workspace=wsd,
+                                                 stream=stream), 20, stream)
+    unfused_us = 1e3 * _event_ms(lambda: ra.decode_unfused(qd, kd, vd, Dd.params, out=od, lse=ld, workspace=wsu,
+                                                           stream=stream), 20, stream)
+    std_us = 1e3 * _event_ms(lambda: ra.decode(qd, kd, vd, std, out=od, lse=ld, workspace=wsd, stream=stream), 20,
+                             stream)
+    ra.status()
+    return {"standard_rope_decode_us": std_us, "fused_bifocal_decode_us": fused_us,
+            "unfused_bifocal_decode_us": unfused_us,
+            "decode_fused_vs_standard": std_us / fused_us, "decode_unfused_vs_standard": std_us / unfused_us}
+
+
 def config_dict(n_gpus):
     return {"workload": f"{PREFILL.name} + {DECODE.name}",
             "prefill": {"B": PREFILL.B, "S": PREFILL.S, "Hq": PREFILL.Hq, "Hkv": PREFILL.Hkv, "D": PREFILL.D,
@@ -480,6 +504,7 @@ def main():
     ra.status()
     cache_rows = measure_cache_rows(ra, q, k, v, kd, vd, qd, stream)
     comparators = measure_comparators(ra, q, k, v, out, lse, ws, stream)
+    comparators.update(measure_decode_comparators(ra, qd, kd, vd, stream))
 
     total_ms, prep_ms, attn_ms, dec_ms, e2e_pre_ms, e2e_dec_ms = max_over_ranks(
         [total_ms, prep_ms, attn_ms, dec_ms, e2e_pre_ms, e2e_dec_ms], world, dev)

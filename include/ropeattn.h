@@ -265,6 +265,23 @@ int ropeattn_decode_noalloc(const void* q, const void* k_cache, const void* v_ca
  * Errors: INVALID_ARG, UNSUPPORTED_DEVICE, CUDA. */
 int ropeattn_wait_selftest(int64_t limit_ns, int32_t* d_result, void* stream);
 
+/* Comparator: decode with the correction rotation unfused. A separate pass
+ * writes a copy of the key cache in `workspace` in which every remote key
+ * (t - s > w0) is turned by Delta s - Delta q (Jet-Long Eq. 5-6; then
+ * q_local . copy[s] = q_remote . R(Delta s) k_cache[s]) and every local key
+ * is copied as is, then a standard-RoPE ropeattn_decode reads the copy. Same
+ * result as ropeattn_decode up to rounding (the copy is rounded to bf16); it
+ * exists to time the fused decode against the unfused route. Needs an
+ * effective bifocal map, else INVALID_ARG. Arguments and layouts as
+ * ropeattn_decode; workspace >= ropeattn_decode_unfused_workspace_size.
+ * Errors: INVALID_ARG, UNSUPPORTED_DEVICE, WORKSPACE, CUDA. */
+size_t ropeattn_decode_unfused_workspace_size(int64_t B, int64_t n, int32_t Hq, int32_t Hkv, int32_t D);
+int ropeattn_decode_unfused(const void* q, const void* k_cache, const void* v_cache,
+                            float* out, float* lse,
+                            int64_t B, int64_t n, int32_t Hq, int32_t Hkv, int32_t D,
+                            const ropeattn_params* params, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
 /* Reads and clears the device status word of the current device (waits for
  * the device to be idle first). Returns ROPEATTN_OK, or ROPEATTN_ERR_TIMEOUT
  * if any kernel since the last call gave up on a bounded wait (its outputs

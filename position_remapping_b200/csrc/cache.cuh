@@ -57,4 +57,50 @@ __global__ void __launch_bounds__(256) cache_write_kernel(const CacheArgs a) {
   }
 }
 
+// Unfused decode (comparator): the correction rotation of Jet-Long Eq. 5-6
+// done as a separate pass over the cache instead of in the attention kernel.
+// For a query at t, a remote key s (t - s > w0) scores
+//   q_remote . R(Delta s) k_cache[s] = q_local . R(Delta s - Delta q) k_cache[s]
+// (R_a R_b = R_{a+b}), so writing every remote key turned by
+// Delta s - Delta q, and every local key unchanged, into a copy lets a
+// standard-RoPE decode (query at p(t) = t, keys read as stored) give the
+// bifocal scores. One thread per (key, pair), angles in double, fp32
+// rotation, bf16 result.
+struct UnfusedRotArgs {
+  const uint32_t* k_cache;  // [B, n, Hkv, D]
+  uint32_t* k_out;          // [B, n, Hkv, D]
+  int B, n, Hkv, D, k_local, dq;
+  PosMap m;
+  double theta[kMaxPairs];
+};
+
+__global__ void __launch_bounds__(256) unfused_rotate_kernel(const UnfusedRotArgs a) {
+  const int P = a.D >> 1;
+  const int rows = blockDim.x / P;
+  const int s = blockIdx.x * rows + threadIdx.x / P;
+  const int i = threadIdx.x % P;
+  if (s >= a.n) return;
+  const bool remote = s < a.k_local;
+  float c = 1.f, sn = 0.f;
+  if (remote) {
+    double sd, cd;
+    sincos(static_cast<double>(pos_remote(a.m, s) - s - a.dq) * a.theta[i], &sd, &cd);
+    c = static_cast<float>(cd);
+    sn = static_cast<float>(sd);
+  }
+  for (int b = 0; b < a.B; ++b) {
+    for (int h = 0; h < a.Hkv; ++h) {
+      const size_t w = ((static_cast<size_t>(b) * a.n + s) * a.Hkv + h) * P + i;
+      const uint32_t x = __ldg(a.k_cache + w);
+      if (remote) {
+        float y0, y1;
+        rot_pair(bf16lo(x), bf16hi(x), c, sn, y0, y1);
+        a.k_out[w] = pack_bf16x2(y0, y1);
+      } else {
+        a.k_out[w] = x;
+      }
+    }
+  }
+}
+
 }  // namespace ropeattn

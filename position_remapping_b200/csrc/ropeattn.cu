@@ -827,7 +827,60 @@ int noalloc_scratch_ptr(void** out) {
 
 }  // namespace
 
-extern "C" int ropeattn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, float* out,
+extern "C" size_t ropeattn_decode_unfused_workspace_size(int64_t B, int64_t n, int32_t Hq, int32_t Hkv, int32_t D) {
+  if (check_shapes(B, n, Hq, Hkv, D) || B == 0 || n == 0) return 0;
+  return align_up(static_cast<size_t>(B) * n * Hkv * D * 2, 256) + decode_layout(B, n, Hq, Hkv, D).total;
+}
+
+int ropeattn_decode_unfused(const void* q, const void* k_cache, const void* v_cache, float* out, float* lse,
+                            int64_t B, int64_t n, int32_t Hq, int32_t Hkv, int32_t D, const ropeattn_params* params,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  g_last_error.clear();
+  int rc = check_shapes(B, n, Hq, Hkv, D);
+  if (rc) return rc;
+  PosMap m;
+  int eff;
+  rc = check_params(params, n, D, &m, &eff);
+  if (rc) return rc;
+  if (eff != ROPEATTN_BIFOCAL)
+    return fail(ROPEATTN_ERR_INVALID_ARG, "the unfused decode needs a bifocal map with G > 1 and w0 < n-1");
+  if (B == 0 || n == 0) return ROPEATTN_OK;
+  if (!q || !k_cache || !v_cache || !out || !lse) return fail(ROPEATTN_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(k_cache)) return fail(ROPEATTN_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  const size_t kbytes = align_up(static_cast<size_t>(B) * n * Hkv * D * 2, 256);
+  const size_t need = kbytes + decode_layout(B, n, Hq, Hkv, D).total;
+  if (!workspace || workspace_bytes < need)
+    return fail(ROPEATTN_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need,
+                workspace ? workspace_bytes : size_t(0));
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+    return fail(ROPEATTN_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  rc = check_device();
+  if (rc) return rc;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const long long t = n - 1;
+  UnfusedRotArgs a{};
+  a.k_cache = static_cast<const uint32_t*>(k_cache);
+  a.k_out = reinterpret_cast<uint32_t*>(ws);
+  a.B = static_cast<int>(B);
+  a.n = static_cast<int>(n);
+  a.Hkv = Hkv;
+  a.D = D;
+  a.k_local = static_cast<int>(t - m.w0 > 0 ? t - m.w0 : 0);
+  m.kind = eff;
+  a.m = m;
+  a.dq = pos_remote(m, static_cast<int>(t)) - static_cast<int>(t);
+  fill_theta(params, D, a.theta);
+  const int rows = 256 / (D / 2);
+  unfused_rotate_kernel<<<static_cast<unsigned>((n + rows - 1) / rows), 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
+  CUDA_TRY(cudaGetLastError(), "unfused rotate launch");
+  // standard RoPE decode over the rotated copy: query at p(t) = t, keys as stored
+  ropeattn_params sp = *params;
+  sp.kind = ROPEATTN_STANDARD;
+  sp.fixed_group = 0;
+  return ropeattn_decode(q, ws, v_cache, out, lse, B, n, Hq, Hkv, D, &sp, ws + kbytes, workspace_bytes - kbytes, stream);
+}
+
+int ropeattn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, float* out,
                                        float* lse, int64_t B, int64_t n, int32_t Hq, int32_t Hkv, int32_t D,
                                        const ropeattn_params* params, void* stream) {
   g_last_error.clear();

@@ -41,3 +41,27 @@ def test_three_call_rejects_non_bifocal():
     with pytest.raises(ra.RopeAttnError) as e:
         ra.prefill_three_call(q, k, v, MapParams(O.BIFOCAL, rope_base=1e4, w0=10, w_pretrained=1000))  # G = 1
     assert e.value.code == ra.ERR_INVALID_ARG
+
+
+UNFUSED = [
+    ("g4_table", 1, 5000, 4, 2, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=300, w_pretrained=1250)),
+    ("g3_phasor_d64", 2, 3001, 4, 1, 64, MapParams(O.BIFOCAL, rope_base=1e4, w0=100, w_pretrained=1001)),
+    ("fixed_g7", 1, 4000, 8, 4, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=50, fixed_group=7)),
+]
+
+
+@pytest.mark.parametrize("case", UNFUSED, ids=[c[0] for c in UNFUSED])
+def test_unfused_decode_matches_oracle_and_fused(case):
+    """Comparator: the correction rotation as a separate pass over the cache
+    followed by a standard-RoPE decode (Jet-Long Eq. 5-6)."""
+    from position_remapping_b200 import ropeattn as ra
+    name, B, n, Hq, Hkv, D, params = case
+    q, kc, vc = make_qkv(B, n, Hq, Hkv, D, seed=zlib.crc32(f"unfused-{name}".encode()) % 10000, q_len=1)
+    qd, kd, vd = q.cuda(), kc.cuda(), vc.cuda()
+    ou, lu = ra.decode_unfused(qd, kd, vd, params)
+    of, lf = ra.decode(qd, kd, vd, params)
+    torch.cuda.synchronize()
+    ra.status()
+    ref_o, ref_l = O.decode(q, kc, vc, params)
+    assert_close(ou.cpu().numpy(), lu.cpu().numpy(), ref_o, ref_l, name + " unfused")
+    assert_close(of.cpu().numpy(), lf.cpu().numpy(), ref_o, ref_l, name + " fused")
