@@ -315,14 +315,15 @@ __global__ void __launch_bounds__(DecodeShape<D, GRP>::kThreads, 1)
   bool ok = true;
   int slot = 0, tslot = 0;
   uint32_t phase = 0;
-  for (int st = 0; st < nstage; ++st) {
-    ok = __all_sync(0xffffffffu, mbar_wait(full + slot, phase, abort_flag));
-    if (!ok) break;
+  // one stage of 64 keys; all_remote: every key of the stage is a remote key
+  // (the stage-table path then rotates unconditionally)
+  auto stage_step = [&](const int st, const bool all_remote) -> bool {
+    if (!__all_sync(0xffffffffu, mbar_wait(full + slot, phase, abort_flag))) return false;
     const int k0 = kb + st * kDecKeys + ks;
     const uint8_t* rows = smem + slot * L::kStageBytes + ks * L::kRowBytes;
     uint4 kr[KPG][NV], vr[KPG][NV];
     float4 tb[NJ];
-    const bool rem_t = ROT == kRotTable && k0 < p.k_local;
+    const bool rem_t = ROT == kRotTable && (all_remote || k0 < p.k_local);
 #pragma unroll
     for (int kk = 0; kk < KPG; ++kk)
 #pragma unroll
@@ -381,7 +382,7 @@ __global__ void __launch_bounds__(DecodeShape<D, GRP>::kThreads, 1)
             X0[j] = y0;
             X1[j] = y1;
           }
-        } else if (q_remote) {
+        } else if (!all_remote && q_remote) {
           // this stream's keys became local: exact-position query view
           load_local();
           q_remote = false;
@@ -498,7 +499,16 @@ __global__ void __launch_bounds__(DecodeShape<D, GRP>::kThreads, 1)
       slot = 0;
       phase ^= 1u;
     }
+    return true;
+  };
+  // stages whose 64 keys all lie before the local window first, without the
+  // per-key remote/local test, then the rest
+  int st = 0;
+  if constexpr (ROT == kRotTable) {
+    const int st_rem = min(nstage, p.k_local - kb >= kDecKeys ? (p.k_local - kb) / kDecKeys : 0);
+    for (; st < st_rem && ok; ++st) ok = stage_step(st, true);
   }
+  for (; st < nstage && ok; ++st) ok = stage_step(st, false);
 
   // --------------------------------------------- merge lane groups of a warp
 #pragma unroll
