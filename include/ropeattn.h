@@ -265,6 +265,17 @@ int ropeattn_decode_noalloc(const void* q, const void* k_cache, const void* v_ca
  * Errors: INVALID_ARG, UNSUPPORTED_DEVICE, CUDA. */
 int ropeattn_wait_selftest(int64_t limit_ns, int32_t* d_result, void* stream);
 
+/* ropeattn_decode over caches with spare rows: k_cache and v_cache are
+ * [B, cache_len, Hkv, D] (cache_len >= n, the rows of each batch entry
+ * allocated for the sequence to grow into, as ropeattn_cache_write fills
+ * them); the first n rows of each batch entry are attended. Otherwise
+ * identical to ropeattn_decode (which is this call with cache_len = n). */
+int ropeattn_decode_cache(const void* q, const void* k_cache, const void* v_cache,
+                          float* out, float* lse,
+                          int64_t B, int64_t n, int64_t cache_len, int32_t Hq, int32_t Hkv, int32_t D,
+                          const ropeattn_params* params, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
 /* Comparator: decode with the correction rotation unfused. A separate pass
  * writes a copy of the key cache in `workspace` in which every remote key
  * (t - s > w0) is turned by Delta s - Delta q (Jet-Long Eq. 5-6; then

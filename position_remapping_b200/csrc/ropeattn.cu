@@ -91,12 +91,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // 4-D bf16 tensor [d3][d2][d1][d0] (d0 contiguous) with box (b0, 1, b2, 1).
+// 4-D bf16 map (d0 innermost); d2_stride: rows of d2 between consecutive d3
+// indices (d2 when 0: a dense tensor; larger for a cache with spare rows).
 int make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3,
-             uint32_t b0, uint32_t b2, bool swizzle128) {
+             uint32_t b0, uint32_t b2, bool swizzle128, uint64_t d2_stride = 0) {
   auto fn = encode_fn();
   if (!fn) return fail(ROPEATTN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t dims[4] = {d0, d1, d2, d3};
-  cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
+  cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * (d2_stride ? d2_stride : d2) * 2};
   cuuint32_t box[4] = {b0, 1, b2, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
@@ -728,9 +730,18 @@ size_t ropeattn_decode_workspace_size(int64_t B, int64_t n, int32_t Hq, int32_t 
 int ropeattn_decode(const void* q, const void* k_cache, const void* v_cache, float* out, float* lse, int64_t B,
                     int64_t n, int32_t Hq, int32_t Hkv, int32_t D, const ropeattn_params* params, void* workspace,
                     size_t workspace_bytes, void* stream) {
+  return ropeattn_decode_cache(q, k_cache, v_cache, out, lse, B, n, n, Hq, Hkv, D, params, workspace, workspace_bytes,
+                               stream);
+}
+
+int ropeattn_decode_cache(const void* q, const void* k_cache, const void* v_cache, float* out, float* lse, int64_t B,
+                          int64_t n, int64_t cache_len, int32_t Hq, int32_t Hkv, int32_t D,
+                          const ropeattn_params* params, void* workspace, size_t workspace_bytes, void* stream) {
   g_last_error.clear();
   int rc = check_shapes(B, n, Hq, Hkv, D);
   if (rc) return rc;
+  if (cache_len < n || cache_len > kMaxPos)
+    return fail(ROPEATTN_ERR_INVALID_ARG, "cache_len (%lld) must be in [n, 2^31)", static_cast<long long>(cache_len));
   PosMap m;
   int eff;
   rc = check_params(params, n, D, &m, &eff);
@@ -779,8 +790,8 @@ int ropeattn_decode(const void* q, const void* k_cache, const void* v_cache, flo
   fill_turns(params, D, dp.turns);
 
   CUtensorMap tk, tv;
-  if ((rc = make_map(&tk, k_cache, D, Hkv, n, B, D, kDecKeys, false))) return rc;
-  if ((rc = make_map(&tv, v_cache, D, Hkv, n, B, D, kDecKeys, false))) return rc;
+  if ((rc = make_map(&tk, k_cache, D, Hkv, n, B, D, kDecKeys, false, cache_len))) return rc;
+  if ((rc = make_map(&tv, v_cache, D, Hkv, n, B, D, kDecKeys, false, cache_len))) return rc;
   CUDA_TRY(cudaMemsetAsync(dp.counters, 0, static_cast<size_t>(B) * Hkv * sizeof(int), st), "memset counters");
   dim3 grid(lay.nsplit, Hkv, static_cast<unsigned>(B));
   if (D == 128) {

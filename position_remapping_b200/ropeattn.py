@@ -25,7 +25,8 @@ EXPORTS = ("ropeattn_posmap", "ropeattn_cache_write", "ropeattn_prefill_workspac
            "ropeattn_prefill_prepare", "ropeattn_prefill_attend",
            "ropeattn_prefill_chunk_workspace_size", "ropeattn_prefill_chunk",
            "ropeattn_prefill_three_call_workspace_size", "ropeattn_prefill_three_call",
-           "ropeattn_decode_workspace_size", "ropeattn_decode", "ropeattn_decode_noalloc", "ropeattn_status",
+           "ropeattn_decode_workspace_size", "ropeattn_decode", "ropeattn_decode_cache", "ropeattn_decode_noalloc",
+           "ropeattn_status",
            "ropeattn_wait_selftest", "ropeattn_decode_unfused_workspace_size", "ropeattn_decode_unfused",
            "ropeattn_last_error", "ropeattn_version")
 
@@ -90,6 +91,8 @@ def _load() -> ctypes.CDLL:
     lib.ropeattn_decode_workspace_size.argtypes = [i64, i64, i32, i32, i32]
     lib.ropeattn_decode_workspace_size.restype = sz
     lib.ropeattn_decode.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, P, vp, sz, vp]
+    lib.ropeattn_decode_cache.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, i32, P, vp, sz, vp]
+    lib.ropeattn_decode_cache.restype = ctypes.c_int
     lib.ropeattn_decode_unfused_workspace_size.argtypes = [i64, i64, i32, i32, i32]
     lib.ropeattn_decode_unfused_workspace_size.restype = sz
     lib.ropeattn_decode_unfused.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, P, vp, sz, vp]
@@ -265,6 +268,26 @@ def prefill_chunk(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.ropeattn_prefill_chunk(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse), B, int(start),
                                       count, Hq, Hkv, D, ctypes.byref(cp), _ptr(workspace), ws_bytes, _stream(stream)))
+    return out, lse
+
+
+def decode_cache(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, n: int, params: MapParams,
+                 out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                 workspace: Optional[torch.Tensor] = None, stream=None):
+    """Decode over the first n rows of caches [B, cache_len, Hkv, D] with
+    spare rows (q [B,Hq,D], the token at position n-1)."""
+    B, Hq, D = q.shape
+    cache_len, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = _workspace(decode_workspace_size(B, n, Hq, Hkv, D), q.device)
+    cp = to_cparams(params)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.ropeattn_decode_cache(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse), B, int(n), cache_len,
+                                     Hq, Hkv, D, ctypes.byref(cp), _ptr(workspace), ws_bytes, _stream(stream)))
     return out, lse
 
 

@@ -110,3 +110,38 @@ def test_multistep_decode_across_group_changes():
         ref_o, ref_l = O.decode(q[:, n - 1], cache[:, :n], v[:, :n], params)
         assert_close(outs[i].cpu().numpy(), lses[i].cpu().numpy(), ref_o, ref_l, f"n={n}")
     assert seen_G == {2, 3, 4}
+
+
+def test_batched_decode_over_caches_with_spare_rows():
+    """B = 3 sequences share one [B, capacity, Hkv, D] cache allocation; each
+    step appends the token of every sequence (ropeattn_cache_write) and
+    decodes over the first n rows (ropeattn_decode_cache), across G = 3 -> 4
+    at n = 769."""
+    from position_remapping_b200 import ropeattn as ra
+    params = MapParams(O.BIFOCAL, rope_base=1e6, w0=100, w_pretrained=256)
+    B, cap, Hq, Hkv, D = 3, 1024, 4, 2, 128
+    S0, N = 740, 790
+    q, k, v = make_qkv(B, N, Hq, Hkv, D, seed=43)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    kc = torch.zeros((B, cap, Hkv, D), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    ra.cache_write(kd[:, :S0].contiguous(), vd[:, :S0].contiguous(), kc, vc, params, 0)
+    outs = []
+    for n in range(S0 + 1, N + 1):
+        ra.cache_write(kd[:, n - 1:n].contiguous(), vd[:, n - 1:n].contiguous(), kc, vc, params, n - 1)
+        o, l = ra.decode_cache(qd[:, n - 1].contiguous(), kc, vc, n, params)
+        outs.append((o.clone(), l.clone()))
+    torch.cuda.synchronize()
+    ra.status()
+    cache = kc.cpu()
+    for i, n in enumerate(range(S0 + 1, N + 1)):
+        if i % 7 and n not in (768, 769, 770, N):
+            continue   # a sample of the steps, and every step around the G change
+        ref_o, ref_l = O.decode(q[:, n - 1], cache[:, :n], v[:, :n], params)
+        assert_close(outs[i][0].cpu().numpy(), outs[i][1].cpu().numpy(), ref_o, ref_l, f"n={n}")
+    # the same call on a dense copy of the first n rows gives the same bits
+    n = N
+    dense = (kc[:, :n].contiguous(), vc[:, :n].contiguous())
+    a = ra.decode(qd[:, n - 1].contiguous(), dense[0], dense[1], params)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], outs[-1][0]) and torch.equal(a[1], outs[-1][1])
