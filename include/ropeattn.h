@@ -189,6 +189,17 @@ int ropeattn_prefill_chunk(const void* q, const void* k_cache, const void* v_cac
                            int64_t B, int64_t start, int64_t count, int32_t Hq, int32_t Hkv, int32_t D,
                            const ropeattn_params* params, void* workspace, size_t workspace_bytes,
                            void* stream);
+/* ropeattn_prefill_chunk over caches with spare rows: k_cache and v_cache
+ * are [B, cache_len, Hkv, D] with cache_len >= start + count (rows of each
+ * batch entry allocated for the sequence to grow into); the first
+ * start + count rows are used. ropeattn_prefill_chunk is this call with
+ * cache_len = start + count; the workspace size is the same. */
+int ropeattn_prefill_chunk_cache(const void* q, const void* k_cache, const void* v_cache,
+                                 float* out, float* lse,
+                                 int64_t B, int64_t start, int64_t count, int64_t cache_len,
+                                 int32_t Hq, int32_t Hkv, int32_t D,
+                                 const ropeattn_params* params, void* workspace, size_t workspace_bytes,
+                                 void* stream);
 
 /* Comparator: the literal three-call bifocal prefill of Jet-Long §3.3 with a
  * separate merge kernel, on the same attention kernel: (A) sliding window

@@ -68,6 +68,7 @@ struct ChunkPrepArgs {
   float2* tab0;             // [count][D/2] (cos, sin) at primary positions, or null (NOPE)
   float2* tab1;             // [count][D/2] at remote positions (BIFOCAL), else null
   int B, L, Hkv, D, start;
+  long long cache_rows;     // rows between batch entries of k_cache (>= L)
   PosMap m;
   double theta[kMaxPairs];
 };
@@ -85,7 +86,8 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const ChunkPrepArgs a) 
     for (int b = 0; b < a.B; ++b) {
       for (int h = 0; h < a.Hkv; ++h) {
         const size_t w = ((static_cast<size_t>(b) * a.L + t) * a.Hkv + h) * P + i;
-        const uint32_t x = __ldg(a.k_cache + w);
+        const size_t r = ((static_cast<size_t>(b) * a.cache_rows + t) * a.Hkv + h) * P + i;
+        const uint32_t x = __ldg(a.k_cache + r);
         float y0, y1;
         rot_pair(bf16lo(x), bf16hi(x), c, s, y0, y1);
         a.k_rem[w] = pack_bf16x2(y0, y1);

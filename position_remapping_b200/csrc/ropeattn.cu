@@ -512,9 +512,20 @@ size_t ropeattn_prefill_chunk_workspace_size(const ropeattn_params* params, int6
 int ropeattn_prefill_chunk(const void* q, const void* k_cache, const void* v_cache, float* out, float* lse,
                            int64_t B, int64_t start, int64_t count, int32_t Hq, int32_t Hkv, int32_t D,
                            const ropeattn_params* params, void* workspace, size_t workspace_bytes, void* stream) {
+  return ropeattn_prefill_chunk_cache(q, k_cache, v_cache, out, lse, B, start, count, start + count, Hq, Hkv, D,
+                                      params, workspace, workspace_bytes, stream);
+}
+
+int ropeattn_prefill_chunk_cache(const void* q, const void* k_cache, const void* v_cache, float* out, float* lse,
+                                 int64_t B, int64_t start, int64_t count, int64_t cache_len, int32_t Hq, int32_t Hkv,
+                                 int32_t D, const ropeattn_params* params, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
   g_last_error.clear();
   if (start < 0 || count < 0) return fail(ROPEATTN_ERR_INVALID_ARG, "start and count must be >= 0");
   const long long L = start + count;
+  if (cache_len < L || cache_len > kMaxPos)
+    return fail(ROPEATTN_ERR_INVALID_ARG, "cache_len (%lld) must be in [start + count, 2^31)",
+                static_cast<long long>(cache_len));
   int rc = check_shapes(B, L, Hq, Hkv, D);
   if (rc) return rc;
   PosMap m;
@@ -551,6 +562,7 @@ int ropeattn_prefill_chunk(const void* q, const void* k_cache, const void* v_cac
     a.tab1 = lay.remote ? reinterpret_cast<float2*>(ws + lay.off_tab1) : nullptr;
     a.B = static_cast<int>(B);
     a.L = static_cast<int>(L);
+    a.cache_rows = cache_len;
     a.Hkv = Hkv;
     a.D = D;
     a.start = static_cast<int>(start);
@@ -565,9 +577,9 @@ int ropeattn_prefill_chunk(const void* q, const void* k_cache, const void* v_cac
   }
   CUtensorMap tq, tk0, tk1, tv;
   if ((rc = make_map(&tq, q, D, Hq, count, B, 64, kBM, true))) return rc;
-  if ((rc = make_map(&tk0, k_cache, D, Hkv, L, B, 64, kBN, true))) return rc;
-  if ((rc = make_map(&tk1, kmap1, D, Hkv, L, B, 64, kBN, true))) return rc;
-  if ((rc = make_map(&tv, v_cache, D, Hkv, L, B, 64, kBN, true))) return rc;
+  if ((rc = make_map(&tk0, k_cache, D, Hkv, L, B, 64, kBN, true, cache_len))) return rc;
+  if ((rc = make_map(&tk1, kmap1, D, Hkv, L, B, 64, kBN, true, lay.remote ? 0 : cache_len))) return rc;
+  if ((rc = make_map(&tv, v_cache, D, Hkv, L, B, 64, kBN, true, cache_len))) return rc;
   pp.out = out;
   pp.lse = lse;
   pp.B = static_cast<int>(B);

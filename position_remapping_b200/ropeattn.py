@@ -23,7 +23,7 @@ ERR_INVALID_ARG, ERR_UNSUPPORTED_DEVICE, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = 
 # every symbol include/ropeattn.h declares
 EXPORTS = ("ropeattn_posmap", "ropeattn_cache_write", "ropeattn_prefill_workspace_size", "ropeattn_prefill",
            "ropeattn_prefill_prepare", "ropeattn_prefill_attend",
-           "ropeattn_prefill_chunk_workspace_size", "ropeattn_prefill_chunk",
+           "ropeattn_prefill_chunk_workspace_size", "ropeattn_prefill_chunk", "ropeattn_prefill_chunk_cache",
            "ropeattn_prefill_three_call_workspace_size", "ropeattn_prefill_three_call",
            "ropeattn_decode_workspace_size", "ropeattn_decode", "ropeattn_decode_cache", "ropeattn_decode_noalloc",
            "ropeattn_status",
@@ -85,6 +85,8 @@ def _load() -> ctypes.CDLL:
     lib.ropeattn_prefill_chunk_workspace_size.argtypes = [P, i64, i64, i64, i32, i32, i32]
     lib.ropeattn_prefill_chunk_workspace_size.restype = sz
     lib.ropeattn_prefill_chunk.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, i32, P, vp, sz, vp]
+    lib.ropeattn_prefill_chunk_cache.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, i32, i32, P, vp, sz, vp]
+    lib.ropeattn_prefill_chunk_cache.restype = ctypes.c_int
     lib.ropeattn_prefill_three_call_workspace_size.argtypes = [P, i64, i64, i32, i32, i32]
     lib.ropeattn_prefill_three_call_workspace_size.restype = sz
     lib.ropeattn_prefill_three_call.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, P, vp, sz, vp]
@@ -252,12 +254,14 @@ def prefill_attend(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, params: Ma
 def prefill_chunk(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, params: MapParams, start: int,
                   out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                   workspace: Optional[torch.Tensor] = None, stream=None):
-    """q [B,count,Hq,D] (tokens start..start+count-1), caches [B,start+count,Hkv,D]
-    bf16 holding every key rotated at its own position. Returns
+    """q [B,count,Hq,D] (tokens start..start+count-1), caches [B,cache_len,Hkv,D]
+    bf16 (cache_len >= start+count; the first start+count rows are used)
+    holding every key rotated at its own position. Returns
     (out [B,count,Hq,D] fp32, lse [B,Hq,count] fp32)."""
     B, count, Hq, D = q.shape
     Hkv = k_cache.shape[2]
-    assert k_cache.shape[1] == start + count, "the cache must hold exactly start + count rows"
+    cache_len = k_cache.shape[1]
+    assert cache_len >= start + count, "the cache must hold at least start + count rows"
     if out is None:
         out = torch.empty((B, count, Hq, D), dtype=torch.float32, device=q.device)
     if lse is None:
@@ -266,8 +270,9 @@ def prefill_chunk(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
     if workspace is None:
         workspace = _workspace(prefill_chunk_workspace_size(params, B, int(start), count, Hq, Hkv, D), q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib.ropeattn_prefill_chunk(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse), B, int(start),
-                                      count, Hq, Hkv, D, ctypes.byref(cp), _ptr(workspace), ws_bytes, _stream(stream)))
+    _check(lib.ropeattn_prefill_chunk_cache(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse), B,
+                                            int(start), count, cache_len, Hq, Hkv, D, ctypes.byref(cp),
+                                            _ptr(workspace), ws_bytes, _stream(stream)))
     return out, lse
 
 

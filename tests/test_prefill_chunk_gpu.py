@@ -62,3 +62,26 @@ def test_chunks_cover_a_whole_prefill():
     last_o, last_l = ra.prefill_chunk(q[:, s0:].contiguous(), kc, vc, params, s0)
     torch.cuda.synchronize()
     assert torch.equal(last_o, whole_o[:, s0:]) and torch.equal(last_l, whole_l[:, :, s0:])
+
+
+@pytest.mark.parametrize("kind", ["bifocal", "standard"])
+def test_chunk_over_caches_with_spare_rows(kind):
+    """B = 2 sequences in one [B, capacity, Hkv, D] allocation: a chunk over
+    the first start + count rows equals the chunk over dense copies of those
+    rows, bit for bit, and matches the oracle."""
+    from position_remapping_b200 import ropeattn as ra
+    params = (MapParams(O.BIFOCAL, rope_base=1e6, w0=150, w_pretrained=400) if kind == "bifocal"
+              else MapParams(O.STANDARD, rope_base=1e4))
+    B, cap, L, start, Hq, Hkv, D = 2, 1600, 1200, 900, 4, 2, 128
+    q, k, v = make_qkv(B, L, Hq, Hkv, D, seed=78)
+    kc = torch.zeros((B, cap, Hkv, D), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    ra.cache_write(k.cuda(), v.cuda(), kc, vc, params, 0)
+    qc = q[:, start:].contiguous().cuda()
+    a_o, a_l = ra.prefill_chunk(qc, kc, vc, params, start)
+    b_o, b_l = ra.prefill_chunk(qc, kc[:, :L].contiguous(), vc[:, :L].contiguous(), params, start)
+    torch.cuda.synchronize()
+    ra.status()
+    assert torch.equal(a_o, b_o) and torch.equal(a_l, b_l)
+    ref_o, ref_l = O.prefill_from_cache(q[:, start:], kc[:, :L].cpu(), v, params, start, stage_bf16=True)
+    assert_close(a_o.cpu().numpy(), a_l.cpu().numpy(), ref_o, ref_l, kind)
