@@ -410,6 +410,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const float m_new = need ? mx : m;
         const float alpha = need ? ex2(m - m_new) : 1.0f;
         l *= alpha;
+        m = m_new;
+        const float mu = (m == -INFINITY) ? 0.f : m;
+        const float2 sl2x2 = make_float2(sl2, sl2), nmu2 = make_float2(-mu, -mu);
+        float2 lsum[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        // P for the whole row in registers first: the exponentials overlap
+        // the previous PV of this tile, which still reads P_a and writes O_a
+        uint32_t pk[kBN / 2];
+#pragma unroll
+        for (int e = 0; e < kBN; e += 2) {
+          const float2 x = __ffma2_rn(make_float2(s[e], s[e + 1]), sl2x2, nmu2);
+          const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+          lsum[(e >> 1) & 1] = __fadd2_rn(lsum[(e >> 1) & 1], pp);
+          pk[e >> 1] = pack_bf16x2(pp.x, pp.y);
+        }
+        l += (lsum[0].x + lsum[0].y) + (lsum[1].x + lsum[1].y);
         // the previous PV of this tile must have completed before O_a is
         // rescaled or P_a is overwritten
         if (g > 0 && !wwait(o_done + a, (g - 1) & 1)) { ok = false; break; }
@@ -425,23 +440,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             tmem_st32(tOa + c * 32, r);
           }
         }
-        m = m_new;
-        const float mu = (m == -INFINITY) ? 0.f : m;
-        const float2 sl2x2 = make_float2(sl2, sl2), nmu2 = make_float2(-mu, -mu);
-        float2 lsum[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-        for (int c = 0; c < kBN / 32; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float2 x = __ffma2_rn(make_float2(s[c * 32 + e], s[c * 32 + e + 1]), sl2x2, nmu2);
-            const float2 pp = make_float2(ex2(x.x), ex2(x.y));
-            lsum[(e >> 1) & 1] = __fadd2_rn(lsum[(e >> 1) & 1], pp);
-            pk[e >> 1] = pack_bf16x2(pp.x, pp.y);
-          }
-          tmem_st16(tPa + c * 16, pk);
-        }
-        l += (lsum[0].x + lsum[0].y) + (lsum[1].x + lsum[1].y);
+        for (int c = 0; c < kBN / 32; ++c) tmem_st16(tPa + c * 16, *reinterpret_cast<const uint32_t(*)[16]>(pk + c * 16));
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(p_full + a);
