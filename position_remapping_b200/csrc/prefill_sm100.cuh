@@ -20,9 +20,10 @@
 //              Separate issuers split the barrier waits and commits (each
 //              costs the issuing thread about a hundred cycles, and the issue
 //              queue is about one MMA deep), so one keeps the tensor pipe fed
-//              while another waits. A softmax waits for its tile's previous
-//              PV (one barrier per tile, committed after each PV) before
-//              rescaling O or overwriting P.
+//              while another waits. A softmax computes its row of P into
+//              registers, then waits for its tile's previous PV (one barrier
+//              per tile, committed after each PV) before rescaling O or
+//              overwriting P, so its exponentials overlap that PV.
 //   Registers: warps 8-11 (the third warpgroup) hand theirs to the softmax
 //              warpgroups with setmaxnreg: 216 per softmax thread, 72 per
 //              thread of warps 8-11; 384 x 168 at launch = 256 x 216 + 128 x 72.
@@ -40,7 +41,11 @@
 // obtained by masking instead of subtraction. The remote partial (normalised)
 // is parked in the output rows, the query tiles are reloaded and rotated to
 // exact positions, and the local pass's epilogue merges the two by their
-// log-sum-exp weights in fp32.
+// log-sum-exp weights in fp32. A forced single pass (one band and map, own
+// output) serves the literal three-call route; a query-row offset and a key
+// count apart from the query rows serve chunked prefill from a cache.
+// CTAs are ordered kv-head-major, so the resident CTAs stream the keys and
+// values of about one kv head and keep them in L2.
 #pragma once
 
 #include "common.cuh"
