@@ -506,11 +506,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 o.z = fmaf(pr.z, wr, o.z);
                 o.w = fmaf(pr.w, wr, o.w);
               }
-              *reinterpret_cast<float4*>(orow + c * 32 + e) = o;
+              // final output: streaming store (evict first), so the 2 GiB of
+              // output does not leave L2 full of dirty lines for what runs next
+              __stcs(reinterpret_cast<float4*>(orow + c * 32 + e), o);
             }
           }
         }
-        if (row_ok) p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.S + t] = lse2 * 0.69314718055994530942f;
+        if (row_ok) __stcs(p.lse + (static_cast<size_t>(b) * p.Hq + h) * p.S + t, lse2 * 0.69314718055994530942f);
       }
     }
   }
