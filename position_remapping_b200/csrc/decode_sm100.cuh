@@ -15,14 +15,17 @@
 //   score = q_remote . R(-u(k)) k_cache,   q_remote = R(Delta q) q_local,
 // and a local key through q_local . k_cache. R(-u(k)) is applied one of two
 // ways (template parameter ROT):
-//  * stage table (G divides 64, one key per group): every stage starts at a
-//    multiple of G, so u(k0 + r) = u(k0) + d(r) with d(r) = r - floor(r/G)
-//    the same in every stage. The group of row r keeps R(d(r)) q_remote, and
-//    all keys of a stage share R(-u(k0)), whose (cos, sin) table is computed
-//    once per stage, NS stages ahead, by one warp (warp st mod 16 while it
-//    works on stage st); the slot's barrier counts that warp's arrival with
-//    the copy's. A group switches to q_local when its keys become local.
-//  * phasor recurrence (any G): each lane carries exp(i u theta) for its
+//  * stage table (one key per group, any G): with d(r) = r - floor(r/G)
+//    and phi = k0 mod G for the stage's first key k0,
+//      u(k0 + r) = u(k0) + d(r) - e,  e = 1 if (r mod G) + phi >= G else 0,
+//    so the group of row r keeps R(d(r)) q_remote, and the keys of a stage
+//    share R(-u(k0)) (e = 0) or R(-(u(k0) - 1)) (e = 1; never when G divides
+//    64, since every stage then starts at a multiple of G). Both (cos, sin)
+//    tables are computed once per stage, NS stages ahead, by one warp (warp
+//    st mod 16 while it works on stage st); the slot's barrier counts that
+//    warp's arrival with the copy's. A group switches to q_local when its
+//    keys become local.
+//  * phasor recurrence (two keys per group): each lane carries exp(i u theta) for its
 //    pairs and advances it by one complex multiply per stage, re-seeded
 //    exactly every 16 stages; local keys use u(n-1), which turns
 //    q_remote . R(Delta q) k_cache back into q_local . k_cache, so one query
@@ -92,8 +95,8 @@ struct DecodeSmem {
   static constexpr int kStageBytes = 2 * kDecKeys * kRowBytes;  // K then V
   static constexpr int kRing = kStages * kStageBytes;
   static constexpr int kMul = kRing;                             // [2][D/2] float2 phasor stage multipliers
-  static constexpr int kTab = kMul + D * 8;                      // [2 kStages][D/4] float4 stage tables
-  static constexpr int kQloc = kTab + 2 * kStages * D * 4;       // [GRP][D/4] float4 local query view
+  static constexpr int kTab = kMul + D * 8;                      // [2 kStages][2][D/4] float4 stage tables
+  static constexpr int kQloc = kTab + 4 * kStages * D * 4;       // [GRP][D/4] float4 local query view
   static constexpr int kBar = kQloc + 2048;                      // full[] mbarriers (GRP * D <= 512)
   static constexpr int kCnt = kBar + kStages * 8;                // release counters per slot
   static constexpr int kMisc = kCnt + kStages * 4;               // abort flag, last flag
@@ -145,21 +148,25 @@ __global__ void __launch_bounds__(DecodeShape<D, GRP>::kThreads, 1)
   const int stage_q = kDecKeys / G, stage_r = kDecKeys - stage_q * G;
   const int t = p.n - 1;                // query position index
 
-  // Stage table of stage st (table slot st mod 2 NS): (cos, sin) of
-  // u(k0) theta for every pair, k0 the stage's first key. The entry of
-  // pair-pair pp (pairs 2pp, 2pp+1) = (c0, c1, s0, s1) sits at
+  // Stage tables of stage st (table slot st mod 2 NS, variants e = 0, 1):
+  // (cos, sin) of (u(k0) - e) theta for every pair, k0 the stage's first key;
+  // variant 1 only when G does not divide 64. The entry of pair-pair pp
+  // (pairs 2pp, 2pp+1) = (c0, c1, s0, s1) sits at
   // 16 (pp / 16) + 8 (pp % 2) + (pp % 16) / 2, so the 8 lanes of a group read
-  // 128 consecutive bytes. One warp writes it, then arrives on the stage's
+  // 128 consecutive bytes. One warp writes them, then arrives on the stage's
   // ring barrier.
+  const bool two_tabs = (kDecKeys % G) != 0;
   auto tab_pos = [](int pp) { return 16 * (pp >> 4) + 8 * (pp & 1) + ((pp & 15) >> 1); };
   auto fill_table = [&](int st) {
     const int k0 = kb + st * kDecKeys;
     const int u0 = k0 - k0 / G;
-    float4* tab = stab + (st % (2 * NS)) * NPP;
-    for (int pp = lane; pp < NPP; pp += 32) {
-      const float2 x = turn_cs(u0, p.turns[2 * pp]);
-      const float2 y = turn_cs(u0, p.turns[2 * pp + 1]);
-      tab[tab_pos(pp)] = make_float4(x.x, y.x, x.y, y.y);
+    for (int e = 0; e < (two_tabs ? 2 : 1); ++e) {
+      float4* tab = stab + ((st % (2 * NS)) * 2 + e) * NPP;
+      for (int pp = lane; pp < NPP; pp += 32) {
+        const float2 x = turn_cs(u0 - e, p.turns[2 * pp]);
+        const float2 y = turn_cs(u0 - e, p.turns[2 * pp + 1]);
+        tab[tab_pos(pp)] = make_float4(x.x, y.x, x.y, y.y);
+      }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(full + st % NS);
@@ -315,6 +322,8 @@ __global__ void __launch_bounds__(DecodeShape<D, GRP>::kThreads, 1)
   bool ok = true;
   int slot = 0, tslot = 0;
   uint32_t phase = 0;
+  int phi = kb % G;                       // first key of the current stage, mod G
+  const int adv = kDecKeys % G, ks_mod = ks % G;
   // one stage of 64 keys; all_remote: every key of the stage is a remote key
   // (the stage-table path then rotates unconditionally)
   auto stage_step = [&](const int st, const bool all_remote) -> bool {
@@ -333,7 +342,7 @@ __global__ void __launch_bounds__(DecodeShape<D, GRP>::kThreads, 1)
       }
     if constexpr (ROT == kRotTable) {
       if (rem_t) {
-        const float4* tt = stab + tslot * NPP;
+        const float4* tt = stab + (tslot * 2 + (phi + ks_mod >= G ? 1 : 0)) * NPP;
 #pragma unroll
         for (int j = 0; j < NJ; ++j) tb[j] = tt[16 * (j >> 1) + 8 * (j & 1) + l8];
       }
@@ -495,6 +504,8 @@ __global__ void __launch_bounds__(DecodeShape<D, GRP>::kThreads, 1)
       if (warp == st % NW && st + NS < nstage) fill_table(st + NS);
     }
     if (++tslot == 2 * NS) tslot = 0;
+    phi += adv;
+    if (phi >= G) phi -= G;
     if (++slot == NS) {
       slot = 0;
       phase ^= 1u;

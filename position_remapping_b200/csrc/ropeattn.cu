@@ -267,14 +267,14 @@ int launch_decode_rot(const CUtensorMap& tk, const CUtensorMap& tv, const Decode
   return ROPEATTN_OK;
 }
 
-// Rotation of remote keys: none (no bifocal map), a shared per-stage table
-// when one key per lane group and G divides the 64-key stage, else the
-// per-lane phasor recurrence.
+// Rotation of remote keys: none (no bifocal map), shared per-stage tables
+// when one key per lane group, else (two keys per group) the per-lane
+// phasor recurrence.
 template <int D, int GRP>
 int launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& dp, dim3 grid, cudaStream_t st) {
   if (!dp.bifocal) return launch_decode_rot<D, GRP, kRotNone>(tk, tv, dp, grid, st);
   if constexpr (DecodeShape<D, GRP>::kKeysPerGroup == 1) {
-    if (kDecKeys % dp.m.G == 0) return launch_decode_rot<D, GRP, kRotTable>(tk, tv, dp, grid, st);
+    return launch_decode_rot<D, GRP, kRotTable>(tk, tv, dp, grid, st);
   }
   return launch_decode_rot<D, GRP, kRotPhasor>(tk, tv, dp, grid, st);
 }
