@@ -10,7 +10,7 @@
 
 namespace ropeattn {
 
-constexpr int kMaxPairs = 64;  // rotation pairs per head: D <= 128
+constexpr int kMaxPairs = 128;  // rotation pairs per head: D <= 256
 
 // Device status word: kernels OR in a code when a bounded wait gives up.
 // Read and cleared by the host (ropeattn_status).

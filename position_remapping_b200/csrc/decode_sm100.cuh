@@ -53,7 +53,7 @@ enum DecodeRot : int { kRotNone = 0, kRotTable = 1, kRotPhasor = 2 };
 
 template <int D, int GRP>
 struct DecodeShape {
-  static constexpr int kKeysPerGroup = (GRP * D <= 256) ? 1 : 2;
+  static constexpr int kKeysPerGroup = (GRP * D <= 256 && D <= 128) ? 1 : 2;
   static constexpr int kWarps = 16 / kKeysPerGroup;
   static constexpr int kThreads = kWarps * 32;
   static constexpr bool kMulInRegs = kKeysPerGroup == 2;   // phasor multipliers in registers
@@ -90,7 +90,7 @@ __device__ __forceinline__ float2 turn_cs(int u, unsigned long long turn) {
 
 template <int D>
 struct DecodeSmem {
-  static constexpr int kStages = D == 128 ? 6 : 10;             // ring depth
+  static constexpr int kStages = D == 256 ? 3 : (D == 128 ? 6 : 10);  // ring depth
   static constexpr int kRowBytes = D * 2;
   static constexpr int kStageBytes = 2 * kDecKeys * kRowBytes;  // K then V
   static constexpr int kRing = kStages * kStageBytes;

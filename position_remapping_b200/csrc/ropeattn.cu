@@ -185,9 +185,13 @@ float scale_log2(const ropeattn_params* p, int D) {
   return static_cast<float>(sc * 1.4426950408889634074);
 }
 
-int check_shapes(long long B, long long S, int Hq, int Hkv, int D) {
+// Shapes every entry point accepts; the attention kernels of prefill take
+// D = 64 or 128 (two O accumulators of D fp32 columns share TMEM with S and
+// P), the decode and cache kernels also D = 256 (allow256).
+int check_shapes(long long B, long long S, int Hq, int Hkv, int D, bool allow256 = false) {
   if (B < 0 || S < 0) return fail(ROPEATTN_ERR_INVALID_ARG, "B and S must be >= 0");
-  if (D != 64 && D != 128) return fail(ROPEATTN_ERR_INVALID_ARG, "D must be 64 or 128 (got %d)", D);
+  if (D != 64 && D != 128 && !(allow256 && D == 256))
+    return fail(ROPEATTN_ERR_INVALID_ARG, allow256 ? "D must be 64, 128 or 256 (got %d)" : "D must be 64 or 128 (got %d)", D);
   if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0)
     return fail(ROPEATTN_ERR_INVALID_ARG, "need Hq >= 1, Hkv >= 1 and Hq %% Hkv == 0 (Hq=%d Hkv=%d)", Hq, Hkv);
   if (S > kMaxPos || B > 65535 || Hq > 65535) return fail(ROPEATTN_ERR_INVALID_ARG, "shape too large");
@@ -339,7 +343,7 @@ int ropeattn_cache_write(const void* k, const void* v, void* k_cache, void* v_ca
   if (start + count > cache_len)
     return fail(ROPEATTN_ERR_INVALID_ARG, "start + count (%lld) exceeds cache_len (%lld)",
                 static_cast<long long>(start + count), static_cast<long long>(cache_len));
-  int rc = check_shapes(B, cache_len, Hkv, Hkv, D);
+  int rc = check_shapes(B, cache_len, Hkv, Hkv, D, true);
   if (rc) return rc;
   PosMap m;
   int eff;
@@ -735,7 +739,7 @@ int ropeattn_prefill_attend(const void* q, const void* k, const void* v, float* 
 }
 
 size_t ropeattn_decode_workspace_size(int64_t B, int64_t n, int32_t Hq, int32_t Hkv, int32_t D) {
-  if (check_shapes(B, n, Hq, Hkv, D) || B == 0 || n == 0) return 0;
+  if (check_shapes(B, n, Hq, Hkv, D, true) || B == 0 || n == 0) return 0;
   return decode_layout(B, n, Hq, Hkv, D).total;
 }
 
@@ -750,7 +754,7 @@ int ropeattn_decode_cache(const void* q, const void* k_cache, const void* v_cach
                           int64_t n, int64_t cache_len, int32_t Hq, int32_t Hkv, int32_t D,
                           const ropeattn_params* params, void* workspace, size_t workspace_bytes, void* stream) {
   g_last_error.clear();
-  int rc = check_shapes(B, n, Hq, Hkv, D);
+  int rc = check_shapes(B, n, Hq, Hkv, D, true);
   if (rc) return rc;
   if (cache_len < n || cache_len > kMaxPos)
     return fail(ROPEATTN_ERR_INVALID_ARG, "cache_len (%lld) must be in [n, 2^31)", static_cast<long long>(cache_len));
@@ -760,8 +764,10 @@ int ropeattn_decode_cache(const void* q, const void* k_cache, const void* v_cach
   if (rc) return rc;
   if (B == 0 || n == 0) return ROPEATTN_OK;
   const int grp = Hq / Hkv;
-  if (!((D == 128 && (grp == 1 || grp == 2 || grp == 4)) || (D == 64 && (grp == 1 || grp == 2 || grp == 4 || grp == 8))))
-    return fail(ROPEATTN_ERR_INVALID_ARG, "decode supports Hq/Hkv in {1,2,4} for D=128 and {1,2,4,8} for D=64");
+  if (!((D == 256 && (grp == 1 || grp == 2)) || (D == 128 && (grp == 1 || grp == 2 || grp == 4)) ||
+        (D == 64 && (grp == 1 || grp == 2 || grp == 4 || grp == 8))))
+    return fail(ROPEATTN_ERR_INVALID_ARG,
+                "decode supports Hq/Hkv in {1,2} for D=256, {1,2,4} for D=128 and {1,2,4,8} for D=64");
   if (!q || !k_cache || !v_cache || !out || !lse) return fail(ROPEATTN_ERR_INVALID_ARG, "null tensor pointer");
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || !aligned16(lse))
     return fail(ROPEATTN_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
@@ -806,6 +812,7 @@ int ropeattn_decode_cache(const void* q, const void* k_cache, const void* v_cach
   if ((rc = make_map(&tv, v_cache, D, Hkv, n, B, D, kDecKeys, false, cache_len))) return rc;
   CUDA_TRY(cudaMemsetAsync(dp.counters, 0, static_cast<size_t>(B) * Hkv * sizeof(int), st), "memset counters");
   dim3 grid(lay.nsplit, Hkv, static_cast<unsigned>(B));
+  if (D == 256) return grp == 1 ? launch_decode<256, 1>(tk, tv, dp, grid, st) : launch_decode<256, 2>(tk, tv, dp, grid, st);
   if (D == 128) {
     if (grp == 1) return launch_decode<128, 1>(tk, tv, dp, grid, st);
     if (grp == 2) return launch_decode<128, 2>(tk, tv, dp, grid, st);
@@ -851,7 +858,7 @@ int noalloc_scratch_ptr(void** out) {
 }  // namespace
 
 extern "C" size_t ropeattn_decode_unfused_workspace_size(int64_t B, int64_t n, int32_t Hq, int32_t Hkv, int32_t D) {
-  if (check_shapes(B, n, Hq, Hkv, D) || B == 0 || n == 0) return 0;
+  if (check_shapes(B, n, Hq, Hkv, D, true) || B == 0 || n == 0) return 0;
   return align_up(static_cast<size_t>(B) * n * Hkv * D * 2, 256) + decode_layout(B, n, Hq, Hkv, D).total;
 }
 
@@ -859,7 +866,7 @@ int ropeattn_decode_unfused(const void* q, const void* k_cache, const void* v_ca
                             int64_t B, int64_t n, int32_t Hq, int32_t Hkv, int32_t D, const ropeattn_params* params,
                             void* workspace, size_t workspace_bytes, void* stream) {
   g_last_error.clear();
-  int rc = check_shapes(B, n, Hq, Hkv, D);
+  int rc = check_shapes(B, n, Hq, Hkv, D, true);
   if (rc) return rc;
   PosMap m;
   int eff;

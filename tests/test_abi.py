@@ -88,6 +88,12 @@ def test_host_argument_checks(ra):
                                   ctypes.byref(cp(_p(kind=STANDARD))), nullp, 0, nullp)
         assert rc == ra.ERR_INVALID_ARG
         assert lib.ropeattn_last_error().decode()
+    # head_dim 256: decode and cache writes only (the prefill's TMEM holds D <= 128)
+    assert lib.ropeattn_prefill(nullp, nullp, nullp, nullp, nullp, 1, 16, 2, 1, 256,
+                                ctypes.byref(cp(_p(kind=STANDARD))), nullp, 0, nullp) == ra.ERR_INVALID_ARG
+    assert lib.ropeattn_decode_workspace_size(1, 1000, 2, 1, 256) > 0
+    assert lib.ropeattn_decode(nullp, nullp, nullp, nullp, nullp, 1, 1000, 8, 1, 256,
+                               ctypes.byref(cp(_p(kind=STANDARD))), nullp, 0, nullp) == ra.ERR_INVALID_ARG  # GQA 8
     bad = [_p(kind=9), _p(kind=PERIODIC, window=0), _p(kind=BIFOCAL, w0=-1, w_pretrained=8),
            _p(kind=BIFOCAL, w0=4, w_pretrained=0), _p(kind=ENDPROMPT, interp=0.5),
            _p(kind=STANDARD, rope_base=1.0), _p(kind=STANDARD, softmax_scale=-1.0)]

@@ -29,7 +29,7 @@ def _bf16_f64(t):
     return t.float().cpu().numpy().astype(np.float64)
 
 
-@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("D", [64, 128, 256])
 @pytest.mark.parametrize("case", KINDS, ids=[c[0] for c in KINDS])
 def test_cache_write_matches_oracle(case, D):
     from position_remapping_b200 import ropeattn as ra

@@ -28,6 +28,10 @@ SMALL = [
     ("bifocal_g2_edge_local", 1, 3000, 2, 1, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=2900, w_pretrained=1500)),
     ("bifocal_fixed_g5_phasor", 1, 3000, 4, 2, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=200, fixed_group=5)),
     ("bifocal_fixed_g4_table", 1, 5000, 8, 4, 128, MapParams(O.BIFOCAL, rope_base=1e4, w0=300, fixed_group=4)),
+    ("d256_standard", 1, 3000, 2, 1, 256, MapParams(O.STANDARD, rope_base=1e4)),
+    ("d256_bifocal_g3_grp2", 2, 5000, 4, 2, 256, MapParams(O.BIFOCAL, rope_base=1e6, w0=400, w_pretrained=2000)),
+    ("d256_periodic", 1, 2500, 2, 2, 256, MapParams(O.PERIODIC, rope_base=1e4, window=512)),
+    ("d256_bifocal_grp1", 1, 4097, 2, 2, 256, MapParams(O.BIFOCAL, rope_base=1e4, w0=100, w_pretrained=1024)),
 ]
 
 
