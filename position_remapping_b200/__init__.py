@@ -8,7 +8,8 @@ without it; any compute call without the library raises ImportError.
 from .inputs import (BIFOCAL, ENDPROMPT, NOPE, PERIODIC, STANDARD, MapParams,  # noqa: F401
                      Workload, WORKLOADS, make_qkv)
 
-_API = ("prefill", "prefill_chunk", "cache_write", "decode", "posmap", "status", "version", "prefill_workspace_size",
+_API = ("prefill", "prefill_chunk", "cache_write", "decode", "decode_cache", "prefill_three_call", "decode_unfused",
+        "wait_selftest", "posmap", "status", "version", "prefill_workspace_size", "prefill_chunk_workspace_size",
         "decode_workspace_size", "RopeAttnError")
 
 

@@ -104,10 +104,6 @@ __device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
-// Named barrier over `count` threads (a multiple of 32).
-__device__ __forceinline__ void named_barrier_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
 
 // Makes generic-proxy writes to shared memory visible to the async proxy
 // (tensor-core operand reads).
