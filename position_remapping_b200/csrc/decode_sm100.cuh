@@ -5,7 +5,7 @@
 // shared-memory ring by TMA, 64 keys per stage (no swizzle, no multicast).
 // A lane group of 8 lanes holds D/8 dimensions of one key and of the query:
 // 16 warps take one key per group per stage, or 8 warps two keys when the
-// GQA group is too large for 128 registers a thread. The last warp to
+// GQA group is too large for 128 registers a thread or D is 256. The last warp to
 // release a slot issues the copy of the stage that reuses it; no thread polls.
 //
 // Scores: the query is rotated once to its position p(n-1) in fp32 and
