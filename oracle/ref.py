@@ -8,7 +8,8 @@ What it computes, and where each step is defined:
 
 * RoPE frequencies theta_i = base^(-2i/d), i = 0..d/2-1, and the
   block-diagonal 2x2 rotation R_t acting on coordinate pairs (2i, 2i+1):
-  "Periodic RoPE for Infinite Context LLMs", §3.1 Eq. 1-2.
+  "Periodic RoPE for Infinite Context LLMs", §3.1 Eq. 1-2. The half-split
+  variant (``pairing`` = 1) turns the pairs (i, i + d/2) by the same angles.
 * Position interpolation divides every position by the factor s ("linearly
   compresses positions into the pretrained range"): "Jet-Long: Efficient
   Long-Context Extension with Dynamic Bifocal RoPE", §2.2; used by
@@ -47,10 +48,11 @@ import math
 import numpy as np
 
 STANDARD, ENDPROMPT, PERIODIC, NOPE, BIFOCAL = 0, 1, 2, 3, 4
+PAIR_ADJACENT, PAIR_HALF = 0, 1
 
 __all__ = [
-    "STANDARD", "ENDPROMPT", "PERIODIC", "NOPE", "BIFOCAL",
-    "round_bf16", "rope_frequencies", "rotation_matrix", "rotate",
+    "STANDARD", "ENDPROMPT", "PERIODIC", "NOPE", "BIFOCAL", "PAIR_ADJACENT", "PAIR_HALF",
+    "round_bf16", "rope_frequencies", "pair_index", "rotation_matrix", "rotate",
     "periodic_position", "endprompt_position", "group_size", "bifocal_group", "remote_position",
     "position_maps", "softmax_scale", "prefill", "prefill_three_call",
     "decode", "cache_keys", "prefill_from_cache", "brute_prefill", "brute_decode", "to_f64",
@@ -94,31 +96,41 @@ def rope_frequencies(D: int, base: float, interp: float = 1.0) -> np.ndarray:
     return (1.0 / np.power(float(base), 2.0 * i / D)) / float(interp)
 
 
-def rotation_matrix(p: float, freqs: np.ndarray) -> np.ndarray:
-    """The D x D block-diagonal R_p of Eq. 2: block i is
+def pair_index(i: int, D: int, pairing: int = PAIR_ADJACENT):
+    """The coordinates (a, b) that rotation pair i turns: (2i, 2i+1) as in
+    the block-diagonal Eq. 2, or (i, i + D/2) for half-split pairing."""
+    return (i, i + D // 2) if pairing == PAIR_HALF else (2 * i, 2 * i + 1)
+
+
+def rotation_matrix(p: float, freqs: np.ndarray, pairing: int = PAIR_ADJACENT) -> np.ndarray:
+    """The D x D rotation R_p of Eq. 2: pair i = (a, b) gets the block
     [[cos(p th_i), -sin(p th_i)], [sin(p th_i), cos(p th_i)]] on rows/cols
-    (2i, 2i+1)."""
+    (a, b) (block-diagonal for adjacent pairing)."""
     D = 2 * len(freqs)
     R = np.zeros((D, D), dtype=np.float64)
     for i, th in enumerate(freqs):
+        a, b = pair_index(i, D, pairing)
         c, s = math.cos(p * th), math.sin(p * th)
-        R[2 * i, 2 * i] = c
-        R[2 * i, 2 * i + 1] = -s
-        R[2 * i + 1, 2 * i] = s
-        R[2 * i + 1, 2 * i + 1] = c
+        R[a, a] = c
+        R[a, b] = -s
+        R[b, a] = s
+        R[b, b] = c
     return R
 
 
-def rotate(x: np.ndarray, pos: np.ndarray, freqs: np.ndarray) -> np.ndarray:
+def rotate(x: np.ndarray, pos: np.ndarray, freqs: np.ndarray, pairing: int = PAIR_ADJACENT) -> np.ndarray:
     """Apply R_{pos[n]} to x[..., n, :] (the action of Eq. 2 without forming
     the matrix). x: [..., N, D]; pos: [N] (integer-valued)."""
     x = np.asarray(x, dtype=np.float64)
     ang = np.asarray(pos, dtype=np.float64)[:, None] * freqs[None, :]   # [N, D/2]
     c, s = np.cos(ang), np.sin(ang)
-    x0, x1 = x[..., 0::2], x[..., 1::2]
+    P = len(freqs)
+    first = slice(0, P) if pairing == PAIR_HALF else slice(0, None, 2)
+    second = slice(P, None) if pairing == PAIR_HALF else slice(1, None, 2)
+    x0, x1 = x[..., first], x[..., second]
     out = np.empty_like(x)
-    out[..., 0::2] = x0 * c - x1 * s
-    out[..., 1::2] = x0 * s + x1 * c
+    out[..., first] = x0 * c - x1 * s
+    out[..., second] = x0 * s + x1 * c
     return out
 
 
@@ -178,6 +190,10 @@ def position_maps(params, L: int):
     raise ValueError(f"unknown kind {k}")
 
 
+def _pairing(params) -> int:
+    return int(getattr(params, "pairing", 0) or 0)
+
+
 def _freqs(params, D):
     interp = float(getattr(params, "interp", 1.0) or 1.0) if int(params.kind) == ENDPROMPT else 1.0
     return rope_frequencies(D, params.rope_base, interp)
@@ -224,6 +240,7 @@ def prefill(q, k, v, params, rows=None, stage_bf16: bool = True):
     scale = softmax_scale(D, params)
     kind = int(params.kind)
     freqs = _freqs(params, D)
+    pr = _pairing(params)
     p_loc, p_rem, _G = position_maps(params, S)
     stage = round_bf16 if stage_bf16 else (lambda a: a)
 
@@ -233,8 +250,8 @@ def prefill(q, k, v, params, rows=None, stage_bf16: bool = True):
     for b in range(B):
         for hk in range(Hkv):
             kk = k[b, :, hk, :]
-            kl = kk if kind == NOPE else stage(rotate(kk, p_loc, freqs))
-            kr = stage(rotate(kk, p_rem, freqs)) if kind == BIFOCAL else None
+            kl = kk if kind == NOPE else stage(rotate(kk, p_loc, freqs, pr))
+            kr = stage(rotate(kk, p_rem, freqs, pr)) if kind == BIFOCAL else None
             for h in range(hk * grp, (hk + 1) * grp):
                 # rows in chunks only to bound memory; each row is independent
                 for c0 in range(0, len(rows), 64):
@@ -242,10 +259,10 @@ def prefill(q, k, v, params, rows=None, stage_bf16: bool = True):
                     nk = int(rr.max()) + 1            # keys beyond the last row are masked
                     ok = np.stack([_allowed(params, int(t), keys[:nk]) for t in rr])
                     qq = q[b, rr, h, :]
-                    ql = qq if kind == NOPE else stage(rotate(qq, p_loc[rr], freqs))
+                    ql = qq if kind == NOPE else stage(rotate(qq, p_loc[rr], freqs, pr))
                     sc = (ql @ kl[:nk].T) * scale                         # [r, nk]
                     if kind == BIFOCAL:
-                        qr = stage(rotate(qq, p_rem[rr], freqs))
+                        qr = stage(rotate(qq, p_rem[rr], freqs, pr))
                         sr = (qr @ kr[:nk].T) * scale
                         local = (rr[:, None] - keys[None, :nk]) <= int(params.w0)
                         sc = np.where(local, sc, sr)
@@ -268,6 +285,7 @@ def prefill_three_call(q, k, v, params, stage_bf16: bool = True):
     grp = Hq // Hkv
     scale = softmax_scale(D, params)
     freqs = _freqs(params, D)
+    pr = _pairing(params)
     G = bifocal_group(params, S)
     t = np.arange(S)
     f = remote_position(t, G)
@@ -279,8 +297,8 @@ def prefill_three_call(q, k, v, params, stage_bf16: bool = True):
     for b in range(B):
         for h in range(Hq):
             hk = h // grp
-            qb, qr = stage(rotate(q[b, :, h], t, freqs)), stage(rotate(q[b, :, h], f, freqs))
-            kb, kr = stage(rotate(k[b, :, hk], t, freqs)), stage(rotate(k[b, :, hk], f, freqs))
+            qb, qr = stage(rotate(q[b, :, h], t, freqs, pr)), stage(rotate(q[b, :, h], f, freqs, pr))
+            kb, kr = stage(rotate(k[b, :, hk], t, freqs, pr)), stage(rotate(k[b, :, hk], f, freqs, pr))
             vv = v[b, :, hk]
             OA, lA = _softmax_rows((qb @ kb.T) * scale, swa, vv)
             OB, lB = _softmax_rows((qr @ kr.T) * scale, causal, vv)
@@ -310,10 +328,11 @@ def cache_keys(k, params, start: int = 0):
         return k.copy()
     p_loc = position_maps(params, int(start) + count)[0][int(start):]
     freqs = _freqs(params, D)
+    pr = _pairing(params)
     out = np.empty_like(k)
     for b in range(k.shape[0]):
         for h in range(k.shape[2]):
-            out[b, :, h] = rotate(k[b, :, h], p_loc, freqs)
+            out[b, :, h] = rotate(k[b, :, h], p_loc, freqs, pr)
     return out
 
 
@@ -335,6 +354,7 @@ def prefill_from_cache(q, k_cache, v_cache, params, start: int, stage_bf16: bool
     scale = softmax_scale(D, params)
     kind = int(params.kind)
     freqs = _freqs(params, D)
+    pr = _pairing(params)
     p_loc, p_rem, G = position_maps(params, L)
     stage = round_bf16 if stage_bf16 else (lambda a: a)
     keys = np.arange(L)
@@ -344,17 +364,17 @@ def prefill_from_cache(q, k_cache, v_cache, params, start: int, stage_bf16: bool
     for b in range(B):
         for hk in range(Hkv):
             kl = kc[b, :, hk]
-            kr = stage(rotate(kl, p_rem - keys, freqs)) if kind == BIFOCAL else None   # Eq. 6, keys
+            kr = stage(rotate(kl, p_rem - keys, freqs, pr)) if kind == BIFOCAL else None   # Eq. 6, keys
             for h in range(hk * grp, (hk + 1) * grp):
                 for c0 in range(0, count, 64):
                     rr = rows[c0:c0 + 64]
                     nk = int(rr.max()) + 1
                     ok = np.stack([_allowed(params, int(t), keys[:nk]) for t in rr])
                     qq = q[b, rr - int(start), h, :]
-                    ql = qq if kind == NOPE else stage(rotate(qq, p_loc[rr], freqs))
+                    ql = qq if kind == NOPE else stage(rotate(qq, p_loc[rr], freqs, pr))
                     sc = (ql @ kl[:nk].T) * scale
                     if kind == BIFOCAL:
-                        qr = stage(rotate(qq, p_rem[rr], freqs))
+                        qr = stage(rotate(qq, p_rem[rr], freqs, pr))
                         sr = (qr @ kr[:nk].T) * scale
                         local = (rr[:, None] - keys[None, :nk]) <= int(params.w0)
                         sc = np.where(local, sc, sr)
@@ -382,6 +402,7 @@ def decode(q, k_cache, v_cache, params):
     scale = softmax_scale(D, params)
     kind = int(params.kind)
     freqs = _freqs(params, D)
+    pr = _pairing(params)
     p_loc, _, G = position_maps(params, n)
     t = n - 1
     keys = np.arange(n)
@@ -392,13 +413,13 @@ def decode(q, k_cache, v_cache, params):
         for h in range(Hq):
             hk = h // grp
             qq = q[b, h][None, :]
-            ql = qq if kind == NOPE else rotate(qq, np.array([p_loc[t]]), freqs)
+            ql = qq if kind == NOPE else rotate(qq, np.array([p_loc[t]]), freqs, pr)
             sc = (ql @ kc[b, :, hk].T) * scale                     # [1, n]
             if kind == BIFOCAL:
                 dq = int(remote_position(t, G)) - t                # Eq. 5
-                qr = rotate(ql, np.array([dq]), freqs)             # Eq. 6, query
+                qr = rotate(ql, np.array([dq]), freqs, pr)             # Eq. 6, query
                 dk = remote_position(keys, G) - keys               # Eq. 5
-                kr = rotate(kc[b, :, hk], dk, freqs)               # Eq. 6, keys
+                kr = rotate(kc[b, :, hk], dk, freqs, pr)               # Eq. 6, keys
                 sr = (qr @ kr.T) * scale
                 local = (t - keys) <= int(params.w0)
                 sc = np.where(local[None, :], sc, sr)
@@ -439,6 +460,7 @@ def brute_prefill(q, k, v, params, stage_bf16: bool = False):
     grp = Hq // Hkv
     scale = softmax_scale(D, params)
     freqs = _freqs(params, D)
+    pr = _pairing(params)
     stage = round_bf16 if stage_bf16 else (lambda a: a)
     out = np.zeros((B, S, Hq, D))
     lse = np.zeros((B, Hq, S))
@@ -454,8 +476,8 @@ def brute_prefill(q, k, v, params, stage_bf16: bool = False):
                     if ab is None:
                         qa, kb = q[b, t, h], k[b, s, hk]
                     else:
-                        qa = stage(rotation_matrix(ab[0], freqs) @ q[b, t, h])
-                        kb = stage(rotation_matrix(ab[1], freqs) @ k[b, s, hk])
+                        qa = stage(rotation_matrix(ab[0], freqs, pr) @ q[b, t, h])
+                        kb = stage(rotation_matrix(ab[1], freqs, pr) @ k[b, s, hk])
                     scores.append(scale * float(qa @ kb))
                 m = max(scores)
                 w = [math.exp(x - m) for x in scores]
@@ -475,6 +497,7 @@ def brute_decode(q, k_raw, v, params):
     grp = Hq // Hkv
     scale = softmax_scale(D, params)
     freqs = _freqs(params, D)
+    pr = _pairing(params)
     t = n - 1
     out = np.zeros((B, Hq, D))
     lse = np.zeros((B, Hq))
@@ -488,7 +511,7 @@ def brute_decode(q, k_raw, v, params):
                 if ab is None:
                     sc = q[b, h] @ k_raw[b, s, hk]
                 else:
-                    sc = (rotation_matrix(ab[0], freqs) @ q[b, h]) @ (rotation_matrix(ab[1], freqs) @ k_raw[b, s, hk])
+                    sc = (rotation_matrix(ab[0], freqs, pr) @ q[b, h]) @ (rotation_matrix(ab[1], freqs, pr) @ k_raw[b, s, hk])
                 scores.append(scale * float(sc))
             m = max(scores)
             w = [math.exp(x - m) for x in scores]

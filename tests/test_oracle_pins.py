@@ -472,3 +472,100 @@ def test_fixed_group_positions_and_brute_force():
     c = O.decode(qn, _cache(kn, params, 8), vn, params)
     d = O.brute_decode(qn, kn, vn, params)
     assert np.allclose(c[0], d[0], atol=1e-12) and np.allclose(c[1], d[1], atol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# half-split pairing: coordinates (i, i + D/2) turned by p * theta_i
+# ----------------------------------------------------------------------------
+def _complex_rope_half(x, pos, base, interp=1.0):
+    """Independent half-split RoPE: the first and second halves of the head
+    are the real and imaginary parts, multiplied by exp(i * pos * theta_i)."""
+    D = x.shape[-1]
+    P = D // 2
+    th = np.array([base ** (-(2.0 * i) / D) for i in range(P)]) / interp
+    z = (x[..., :P] + 1j * x[..., P:]) * np.exp(1j * np.asarray(pos)[:, None, None] * th[None, None, :])
+    return np.concatenate([z.real, z.imag], axis=-1)
+
+
+def _interleave(x):
+    """(x_0, x_{D/2}, x_1, x_{D/2+1}, ...): half-split order to adjacent order."""
+    P = x.shape[-1] // 2
+    out = np.empty_like(x)
+    out[..., 0::2], out[..., 1::2] = x[..., :P], x[..., P:]
+    return out
+
+
+def test_half_split_rotation_basis_vectors():
+    # D = 8, theta = (1, 0.1, 0.01, 0.001): R e_i = cos e_i + sin e_{i+4},
+    # R e_{i+4} = -sin e_i + cos e_{i+4}
+    f = O.rope_frequencies(8, 1e4)
+    for t in (1, 3, 1000):
+        R = O.rotation_matrix(t, f, O.PAIR_HALF)
+        for i, th in enumerate((1.0, 0.1, 0.01, 0.001)):
+            c, s = math.cos(t * th), math.sin(t * th)
+            col_i = np.zeros(8)
+            col_i[i], col_i[i + 4] = c, s
+            col_j = np.zeros(8)
+            col_j[i], col_j[i + 4] = -s, c
+            assert np.allclose(R[:, i], col_i, atol=1e-13)
+            assert np.allclose(R[:, i + 4], col_j, atol=1e-13)
+    assert O.pair_index(3, 16, O.PAIR_HALF) == (3, 11) and O.pair_index(3, 16) == (6, 7)
+
+
+def test_half_split_group_properties_and_complex_form():
+    D = 32
+    f = O.rope_frequencies(D, 5e5, 4.0)
+    I = np.eye(D)
+    for a, b in [(3, 5), (70000, -17)]:
+        Ra, Rb = O.rotation_matrix(a, f, O.PAIR_HALF), O.rotation_matrix(b, f, O.PAIR_HALF)
+        assert np.allclose(Ra.T @ Ra, I, atol=1e-13)
+        assert np.allclose(Ra @ Rb, O.rotation_matrix(a + b, f, O.PAIR_HALF), atol=1e-9)
+        # the same rotation seen through the interleaving permutation
+        Pi = _interleave(I).T        # Pi @ x = interleave(x)
+        assert np.allclose(Ra, Pi.T @ O.rotation_matrix(a, f) @ Pi, atol=1e-13)
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((6, 1, D))
+    pos = np.array([0, 1, 9, 4096, 65535, 131071])
+    got = O.rotate(x[:, 0], pos, f, O.PAIR_HALF)
+    assert np.allclose(got, _complex_rope_half(x, pos, 5e5, 4.0)[:, 0], atol=1e-12)
+
+
+_HALF_PARAMS = {
+    O.STANDARD: MapParams(O.STANDARD, rope_base=1e4, pairing=1),
+    O.ENDPROMPT: MapParams(O.ENDPROMPT, rope_base=5e5, interp=8.0, seg1_len=11, term_start=65500, pairing=1),
+    O.PERIODIC: MapParams(O.PERIODIC, window=5, pairing=1),
+    O.BIFOCAL: MapParams(O.BIFOCAL, rope_base=1e6, w0=3, w_pretrained=6, pairing=1),
+}
+
+
+@pytest.mark.parametrize("kind", [O.STANDARD, O.ENDPROMPT, O.PERIODIC, O.BIFOCAL])
+def test_half_split_prefill_brute_and_permutation(kind):
+    params = _HALF_PARAMS[kind]
+    q, k, v = make_qkv(1, 19, 4, 2, 8, seed=41)
+    a = O.prefill(q, k, v, params, stage_bf16=False)
+    b = O.brute_prefill(q, k, v, params)
+    assert np.allclose(a[0], b[0], atol=1e-12) and np.allclose(a[1], b[1], atol=1e-12)
+    # scores are unchanged when q and k are permuted alike: half-split on
+    # (q, k) is adjacent pairing on the interleaved (q, k)
+    adj = params.replace(pairing=0)
+    qn, kn, vn = O.to_f64(q), O.to_f64(k), O.to_f64(v)
+    c = O.prefill(_interleave(qn), _interleave(kn), vn, adj, stage_bf16=False)
+    assert np.allclose(a[0], c[0], atol=1e-12) and np.allclose(a[1], c[1], atol=1e-12)
+    # and it is a different map from adjacent pairing on the same inputs
+    d = O.prefill(q, k, v, adj, stage_bf16=False)
+    assert not np.allclose(a[0], d[0], atol=1e-6)
+
+
+@pytest.mark.parametrize("kind", [O.STANDARD, O.PERIODIC, O.BIFOCAL])
+def test_half_split_cache_and_decode(kind):
+    params = _HALF_PARAMS[kind]
+    qf, kf, vf = make_qkv(2, 23, 4, 2, 8, seed=42, q_len=1)
+    qn, kn, vn = O.to_f64(qf), O.to_f64(kf), O.to_f64(vf)
+    t = np.arange(23)
+    pos = t % params.window if kind == O.PERIODIC else t
+    cache = O.cache_keys(kn, params)
+    want = np.stack([_complex_rope_half(kn[b], pos, params.rope_base) for b in range(2)])
+    assert np.allclose(cache, want, atol=1e-12)
+    a = O.decode(qn, cache, vn, params)
+    b = O.brute_decode(qn, kn, vn, params)
+    assert np.allclose(a[0], b[0], atol=1e-12) and np.allclose(a[1], b[1], atol=1e-12)
