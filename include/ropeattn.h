@@ -24,8 +24,15 @@
  *           position; v_cache [B, n, Hkv, D] bf16; out [B, Hq, D] fp32;
  *           lse [B, Hq] fp32.
  *   GQA: query head h reads key/value head h / (Hq / Hkv).
- *   Supported: D in {64, 128}; Hq % Hkv == 0; decode also needs
- *   Hq / Hkv <= 4 for D = 128 and <= 8 for D = 64.
+ *   Supported: D in {64, 128} (decode and cache writes also 256);
+ *   Hq % Hkv == 0; decode also needs Hq / Hkv <= 2 for D = 256, <= 4 for
+ *   D = 128 and <= 8 for D = 64.
+ *   Half-split pairing (params.pairing = ROPEATTN_PAIR_HALF): q, k and v are
+ *   given in their own order; the rotation pairs coordinates (i, i + D/2),
+ *   and key caches hold each rotated key in adjacent order instead (element
+ *   2i = coordinate i, element 2i+1 = coordinate i + D/2), as
+ *   ropeattn_cache_write stores them. Value caches and outputs keep the
+ *   values' order.
  *
  * Errors: every entry point returns ROPEATTN_OK (0) or a negative code and
  * sets a thread-local message readable with ropeattn_last_error(). Argument
@@ -69,6 +76,16 @@ typedef enum {
   ROPEATTN_BIFOCAL   = 4
 } ropeattn_kind;
 
+/* Which coordinates the rotation pairs. Periodic RoPE §3.1 Eq. 2 writes the
+ * rotation block-diagonally on (2i, 2i+1); the half-split form pairs
+ * (i, i + D/2) with the same angle p * theta_i. The two differ only by a
+ * fixed permutation of the head dimensions, applied to q and k alike. NOPE
+ * rotates nothing and ignores the field. */
+typedef enum {
+  ROPEATTN_PAIR_ADJACENT = 0,   /* (2i, 2i+1) */
+  ROPEATTN_PAIR_HALF     = 1    /* (i, i + D/2) */
+} ropeattn_pairing;
+
 /* Parameters of the position map. Fields a kind does not use are ignored,
  * except the reserved ones, which must be zero. */
 typedef struct ropeattn_params {
@@ -85,7 +102,8 @@ typedef struct ropeattn_params {
   int64_t w0;             /* BIFOCAL: local window, >= 0 (0 = the token itself only) */
   int64_t w_pretrained;   /* BIFOCAL: pretrained context window, >= 1 (unused with fixed_group) */
   float   softmax_scale;  /* > 0 to override; 0 -> 1/sqrt(D) */
-  int32_t reserved[3];    /* must be 0 */
+  int32_t pairing;        /* ropeattn_pairing (0 = adjacent) */
+  int32_t reserved[2];    /* must be 0 */
 } ropeattn_params;
 
 /* Position map of a sequence of length L (Periodic RoPE §3.2 Eq. 4; Jet-Long
@@ -110,7 +128,11 @@ int ropeattn_posmap(const ropeattn_params* params, int64_t L,
  * for i < count, p the kind's primary position of the absolute token index
  * (t for STANDARD and BIFOCAL, EndPrompt's two segments, t mod W for
  * PERIODIC; NOPE stores keys unrotated). Angles p * theta_i in double
- * precision, rotation in fp32, as the prefill's key pre-pass does.
+ * precision, rotation in fp32, as the prefill's key pre-pass does. With
+ * ROPEATTN_PAIR_HALF the key is rotated on pairs (i, i + D/2) and stored in
+ * adjacent order (element 2i = rotated coordinate i, 2i+1 = rotated
+ * coordinate i + D/2), the order every cache reader of this library expects
+ * for half-split params; values are copied as given.
  *   k, v:             [B, count, Hkv, D] bf16, device, 4-byte aligned
  *   k_cache, v_cache: [B, cache_len, Hkv, D] bf16, device; caller-owned
  *   v, v_cache:       both NULL to write keys only
@@ -124,8 +146,9 @@ int ropeattn_cache_write(const void* k, const void* v, void* k_cache, void* v_ca
                          int32_t Hkv, int32_t D, const ropeattn_params* params, void* stream);
 
 /* Bytes of device workspace ropeattn_prefill needs for these shapes:
- * rotated keys (one copy per position map the kind uses) and the query
- * angle tables. 0 for NOPE. */
+ * rotated keys (one copy per position map the kind uses), the query angle
+ * tables and, for half-split pairing, a copy of q in adjacent order. 0 for
+ * NOPE. */
 size_t ropeattn_prefill_workspace_size(const ropeattn_params* params, int64_t B,
                                        int64_t S, int32_t Hq, int32_t Hkv, int32_t D);
 
@@ -136,7 +159,10 @@ size_t ropeattn_prefill_workspace_size(const ropeattn_params* params, int64_t B,
  * keeps an online softmax per row, and for BIFOCAL merges the local and
  * remote partials by their log-sum-exp (Jet-Long §3.3 Eq. 7) before writing.
  * Tensor-core operands are bf16: the rotated q and k are rounded to bf16
- * (round to nearest even); scores, softmax and outputs are fp32.
+ * (round to nearest even); scores, softmax and outputs are fp32. With
+ * ROPEATTN_PAIR_HALF the key pre-pass reads k on pairs (i, i + D/2) and
+ * writes adjacent order, and one streaming pass first copies q into the
+ * workspace in adjacent order; the attention kernel is the same.
  *   workspace: device, 256-byte aligned, >= ropeattn_prefill_workspace_size
  *              bytes (may be NULL when that size is 0). Caller-owned; the
  *              call overwrites it; calls sharing it must be stream-ordered.
@@ -174,7 +200,10 @@ int ropeattn_prefill_attend(const void* q, const void* k, const void* v, float* 
  * keys R(Delta s) k_cache[s], Delta s = f(s) - s with G = G(L) (Eq. 5-6),
  * into `workspace`, and the remote pass reads them. Queries are rotated in
  * the attention kernel as in ropeattn_prefill. Tensor-core operands are
- * bf16 (the remote keys are rounded to bf16 after the correction).
+ * bf16 (the remote keys are rounded to bf16 after the correction). With
+ * ROPEATTN_PAIR_HALF the key cache is in adjacent order (as
+ * ropeattn_cache_write stores it) and q is copied into the workspace in
+ * adjacent order first.
  *   q:      [B, count, Hq, D] bf16, unrotated
  *   k_cache, v_cache: [B, L, Hkv, D] bf16 (contiguous, L rows)
  *   out:    [B, count, Hq, D] fp32;  lse: [B, Hq, count] fp32 (natural log)
@@ -231,12 +260,16 @@ size_t ropeattn_decode_workspace_size(int64_t B, int64_t n, int32_t Hq,
  * (n-1) - k > w0 is corrected on the fly by Delta k = f(k) - k, in fp32
  * registers. Other kinds: the query is rotated to its position p(n-1) and
  * the cache is read as stored (PERIODIC reads only the last `window` keys).
- * Split-KV: each CTA streams a contiguous key range of one KV head with
- * 128-bit loads, and the last CTA of each head merges the partials by their
- * log-sum-exp in a fixed order (deterministic).
- *   workspace: device, >= ropeattn_decode_workspace_size bytes. The call
- *              clears its counters with cudaMemsetAsync on `stream` first;
- *              calls sharing a workspace must be stream-ordered.
+ * Split-KV: each CTA streams a contiguous key range of one KV head through
+ * a shared-memory ring filled by TMA, and the last CTA of each head merges
+ * the partials by their log-sum-exp in a fixed order (deterministic). With
+ * ROPEATTN_PAIR_HALF the key cache is in adjacent order (as
+ * ropeattn_cache_write stores it) and the query is first copied into the
+ * workspace in adjacent order.
+ *   workspace: device, >= ropeattn_decode_workspace_size bytes (the size
+ *              covers either pairing). The call clears its counters with
+ *              cudaMemsetAsync on `stream` first; calls sharing a workspace
+ *              must be stream-ordered.
  * n == 0 or B == 0 is a no-op.
  * Errors: INVALID_ARG, UNSUPPORTED_DEVICE, WORKSPACE, CUDA. */
 int ropeattn_decode(const void* q, const void* k_cache, const void* v_cache,

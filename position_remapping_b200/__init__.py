@@ -5,8 +5,8 @@ The compute path is the C-ABI library ``libropeattn.so`` (include/ropeattn.h);
 library lazily so that ``position_remapping_b200.inputs`` stays importable
 without it; any compute call without the library raises ImportError.
 """
-from .inputs import (BIFOCAL, ENDPROMPT, NOPE, PERIODIC, STANDARD, MapParams,  # noqa: F401
-                     Workload, WORKLOADS, make_qkv)
+from .inputs import (BIFOCAL, ENDPROMPT, NOPE, PAIR_ADJACENT, PAIR_HALF, PERIODIC, STANDARD,  # noqa: F401
+                     MapParams, Workload, WORKLOADS, make_qkv)
 
 _API = ("prefill", "prefill_chunk", "cache_write", "decode", "decode_cache", "prefill_three_call", "decode_unfused",
         "wait_selftest", "posmap", "status", "version", "prefill_workspace_size", "prefill_chunk_workspace_size",

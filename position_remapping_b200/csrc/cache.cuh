@@ -7,10 +7,12 @@
 // position of the token's absolute index), sincos in double, rounded to fp32;
 // the pair is rotated in fp32 and rounded to bf16 (nearest even) for every
 // (batch, kv head) row of the token. The value pair is copied alongside.
-// Consecutive threads touch consecutive 4-byte words of a row.
+// Consecutive threads touch consecutive 4-byte words of a row. Half-split
+// keys are read pair (i, i + D/2) and stored in adjacent order (pairing.cuh).
 #pragma once
 
 #include "common.cuh"
+#include "pairing.cuh"
 #include "posmap.cuh"
 
 namespace ropeattn {
@@ -22,6 +24,7 @@ struct CacheArgs {
   uint32_t* v_cache;   // same layout, or null
   long long start, count, cache_len;
   int B, Hkv, D;
+  int half;            // 1: k pairs coordinates (i, i + D/2)
   PosMap m;
   double theta[kMaxPairs];
 };
@@ -42,14 +45,15 @@ __global__ void __launch_bounds__(256) cache_write_kernel(const CacheArgs a) {
   }
   for (int b = 0; b < a.B; ++b) {
     for (int h = 0; h < a.Hkv; ++h) {
-      const size_t src = ((static_cast<size_t>(b) * a.count + i_tok) * a.Hkv + h) * P + i;
+      const size_t src_row = ((static_cast<size_t>(b) * a.count + i_tok) * a.Hkv + h) * P;
+      const size_t src = src_row + i;
       const size_t dst = ((static_cast<size_t>(b) * a.cache_len + t) * a.Hkv + h) * P + i;
-      const uint32_t x = __ldg(a.k + src);
       if (a.m.kind == kNope) {
-        a.k_cache[dst] = x;
+        a.k_cache[dst] = __ldg(a.k + src);
       } else {
-        float y0, y1;
-        rot_pair(bf16lo(x), bf16hi(x), c, s, y0, y1);
+        float x0, x1, y0, y1;
+        load_rot_pair(a.k, src_row, i, P, a.half != 0, x0, x1);
+        rot_pair(x0, x1, c, s, y0, y1);
         a.k_cache[dst] = pack_bf16x2(y0, y1);
       }
       if (a.v != nullptr) a.v_cache[dst] = __ldg(a.v + src);

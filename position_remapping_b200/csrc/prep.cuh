@@ -10,10 +10,12 @@
 // interpolation, Jet-Long §2.2), phase = p * theta_i in double precision,
 // sincos in double, rounded to fp32. The rotation of a pair (Eq. 2) is done in
 // fp32 and the result rounded to bf16 (nearest even), the tensor-core operand
-// type.
+// type. Half-split keys are read pair (i, i + D/2) and written in adjacent
+// order (pairing.cuh).
 #pragma once
 
 #include "common.cuh"
+#include "pairing.cuh"
 #include "posmap.cuh"
 
 namespace ropeattn {
@@ -25,6 +27,7 @@ struct PrepArgs {
   float2* tab0;           // [S][D/2] (cos, sin) at map-0 positions
   float2* tab1;           // [S][D/2] at map-1 positions, or null
   int B, S, Hkv, D;
+  int half;               // 1: k pairs coordinates (i, i + D/2)
   PosMap m;
   double theta[kMaxPairs];
 };
@@ -46,11 +49,11 @@ __global__ void __launch_bounds__(256) rope_prep_kernel(const PrepArgs a) {
     uint32_t* dst = mi == 0 ? a.k_rot0 : a.k_rot1;
     for (int b = 0; b < a.B; ++b) {
       for (int h = 0; h < a.Hkv; ++h) {
-        const size_t w = ((static_cast<size_t>(b) * a.S + t) * a.Hkv + h) * P + i;
-        const uint32_t x = __ldg(a.k + w);
-        float y0, y1;
-        rot_pair(bf16lo(x), bf16hi(x), c, s, y0, y1);
-        dst[w] = pack_bf16x2(y0, y1);
+        const size_t row = ((static_cast<size_t>(b) * a.S + t) * a.Hkv + h) * P;
+        float x0, x1, y0, y1;
+        load_rot_pair(a.k, row, i, P, a.half != 0, x0, x1);
+        rot_pair(x0, x1, c, s, y0, y1);
+        dst[row + i] = pack_bf16x2(y0, y1);
       }
     }
   }

@@ -12,6 +12,7 @@
 #include "../../include/ropeattn.h"
 #include "common.cuh"
 #include "cache.cuh"
+#include "pairing.cuh"
 #include "decode_sm100.cuh"
 #include "merge.cuh"
 #include "selftest.cuh"
@@ -117,8 +118,10 @@ constexpr long long kMaxPos = 0x7fffffffLL;
 // "reduces to the unmodified base model").
 int check_params(const ropeattn_params* p, long long L, int D, PosMap* m, int* eff_kind) {
   if (!p) return fail(ROPEATTN_ERR_INVALID_ARG, "params is NULL");
-  if (p->reserved[0] != 0 || p->reserved[1] != 0 || p->reserved[2] != 0)
+  if (p->reserved[0] != 0 || p->reserved[1] != 0)
     return fail(ROPEATTN_ERR_INVALID_ARG, "reserved fields must be 0");
+  if (p->pairing != ROPEATTN_PAIR_ADJACENT && p->pairing != ROPEATTN_PAIR_HALF)
+    return fail(ROPEATTN_ERR_INVALID_ARG, "pairing must be ROPEATTN_PAIR_ADJACENT or ROPEATTN_PAIR_HALF");
   if (p->fixed_group < 0 || p->fixed_group > (1 << 30) || (p->fixed_group != 0 && p->kind != ROPEATTN_BIFOCAL))
     return fail(ROPEATTN_ERR_INVALID_ARG, "fixed_group must be 0, or in [1, 2^30] for BIFOCAL");
   if (p->kind < ROPEATTN_STANDARD || p->kind > ROPEATTN_BIFOCAL)
@@ -161,6 +164,25 @@ int check_params(const ropeattn_params* p, long long L, int D, PosMap* m, int* e
   return ROPEATTN_OK;
 }
 
+// True when the rotation pairs (i, i + D/2): the query is then permuted to
+// adjacent order on entry and keys where they are rotated (pairing.cuh).
+bool half_pairing(const ropeattn_params* p) {
+  return p->pairing == ROPEATTN_PAIR_HALF && p->kind != ROPEATTN_NOPE;
+}
+
+// rows x D bf16 from half-split to adjacent order (pairing.cuh).
+int launch_interleave(const void* in, void* out, long long rows, int D, cudaStream_t st) {
+  PairInterleaveArgs a{};
+  a.in = static_cast<const uint2*>(in);
+  a.out = static_cast<uint4*>(out);
+  a.rows = rows;
+  a.D = D;
+  const long long threads = rows * (D / 8);
+  pair_interleave_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, st>>>(a);
+  CUDA_TRY(cudaGetLastError(), "pair_interleave launch");
+  return ROPEATTN_OK;
+}
+
 void fill_theta(const ropeattn_params* p, int D, double* theta) {
   const double s = p->kind == ROPEATTN_ENDPROMPT ? p->interp : 1.0;
   for (int i = 0; i < D / 2; ++i) theta[i] = std::pow(p->rope_base, -2.0 * i / D) / s;
@@ -200,18 +222,24 @@ int check_shapes(long long B, long long S, int Hq, int Hkv, int D, bool allow256
 
 struct PrefillLayout {
   int nmaps;
+  bool half;
   size_t krot_bytes, tab_bytes, total;
-  size_t off_krot[2], off_tab[2];
+  size_t off_krot[2], off_tab[2], off_q;
 };
 
-PrefillLayout prefill_layout(int eff_kind, long long B, long long S, int Hkv, int D) {
+// Workspace of a prefill: rotated keys per map, query angle tables per map,
+// and for half-split pairing the query in adjacent order.
+PrefillLayout prefill_layout(int eff_kind, bool half, long long B, long long S, int Hq, int Hkv, int D) {
   PrefillLayout L{};
   L.nmaps = eff_kind == ROPEATTN_NOPE ? 0 : (eff_kind == ROPEATTN_BIFOCAL ? 2 : 1);
+  L.half = half;
   L.krot_bytes = align_up(static_cast<size_t>(B) * S * Hkv * D * 2, 256);
   L.tab_bytes = align_up(static_cast<size_t>(S) * (D / 2) * sizeof(float2), 256);
   size_t off = 0;
   for (int i = 0; i < L.nmaps; ++i) { L.off_krot[i] = off; off += L.krot_bytes; }
   for (int i = 0; i < L.nmaps; ++i) { L.off_tab[i] = off; off += L.tab_bytes; }
+  L.off_q = off;
+  if (half) off += align_up(static_cast<size_t>(B) * S * Hq * D * 2, 256);
   L.total = off;
   return L;
 }
@@ -233,7 +261,7 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk0, const CUtensor
 
 struct DecodeLayout {
   int nsplit;
-  size_t off_o, off_ml, off_cnt, total;
+  size_t off_q, off_o, off_ml, off_cnt, total;
 };
 
 // One CTA per SM is resident (shared-memory ring), so the grid is sized to
@@ -249,8 +277,9 @@ DecodeLayout decode_layout(long long B, long long keys, int Hq, int Hkv, int D) 
   DecodeLayout L{};
   L.nsplit = decode_nsplit(B, keys, Hkv);
   size_t slots = static_cast<size_t>(B) * Hq * L.nsplit;
-  L.off_o = 0;
-  L.off_ml = align_up(slots * D * sizeof(float), 256);
+  L.off_q = 0;   // the query in adjacent order (half-split pairing); kept for either pairing
+  L.off_o = align_up(static_cast<size_t>(B) * Hq * D * 2, 256);
+  L.off_ml = L.off_o + align_up(slots * D * sizeof(float), 256);
   L.off_cnt = L.off_ml + align_up(slots * sizeof(float2), 256);
   L.total = L.off_cnt + align_up(static_cast<size_t>(B) * Hkv * sizeof(int), 256);
   return L;
@@ -369,6 +398,7 @@ int ropeattn_cache_write(const void* k, const void* v, void* k_cache, void* v_ca
   a.B = static_cast<int>(B);
   a.Hkv = Hkv;
   a.D = D;
+  a.half = half_pairing(params) ? 1 : 0;
   m.kind = params->kind == ROPEATTN_BIFOCAL ? ROPEATTN_STANDARD : params->kind;  // primary position: t
   a.m = m;
   fill_theta(params, D, a.theta);
@@ -383,7 +413,7 @@ size_t ropeattn_prefill_workspace_size(const ropeattn_params* params, int64_t B,
   PosMap m;
   int eff;
   if (check_params(params, S, D, &m, &eff) || check_shapes(B, S, Hq, Hkv, D)) return 0;
-  return prefill_layout(eff, B, S, Hkv, D).total;
+  return prefill_layout(eff, half_pairing(params), B, S, Hq, Hkv, D).total;
 }
 
 }  // extern "C"
@@ -414,7 +444,7 @@ int prefill_impl(int stages, const void* q, const void* k, const void* v, float*
     return fail(ROPEATTN_ERR_INVALID_ARG, "too many query tiles");
   rc = check_device();
   if (rc) return rc;
-  const PrefillLayout lay = prefill_layout(eff, B, S, Hkv, D);
+  const PrefillLayout lay = prefill_layout(eff, half_pairing(params), B, S, Hq, Hkv, D);
   if (lay.total > 0) {
     if (!workspace || workspace_bytes < lay.total)
       return fail(ROPEATTN_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", lay.total,
@@ -441,6 +471,7 @@ int prefill_impl(int stages, const void* q, const void* k, const void* v, float*
     a.S = static_cast<int>(S);
     a.Hkv = Hkv;
     a.D = D;
+    a.half = lay.half ? 1 : 0;
     a.m = m;
     if (stages & kStagePrepare) {
       fill_theta(params, D, a.theta);
@@ -454,6 +485,10 @@ int prefill_impl(int stages, const void* q, const void* k, const void* v, float*
     pp.tab1 = a.tab1;
   }
   if (!(stages & kStageAttend)) return ROPEATTN_OK;
+  if (lay.half) {
+    if ((rc = launch_interleave(q, ws + lay.off_q, B * S * Hq, D, st))) return rc;
+    q = ws + lay.off_q;
+  }
 
   CUtensorMap tq, tk0, tk1, tv;
   if ((rc = make_map(&tq, q, D, Hq, S, B, 64, kBM, true))) return rc;
@@ -479,14 +514,15 @@ int prefill_impl(int stages, const void* q, const void* k, const void* v, float*
 }
 
 struct ChunkLayout {
-  size_t off_krem, off_tab0, off_tab1, total;
-  bool remote, tables;
+  size_t off_krem, off_tab0, off_tab1, off_q, total;
+  bool remote, tables, half;
 };
 
-ChunkLayout chunk_layout(int eff_kind, long long B, long long L, long long count, int Hkv, int D) {
+ChunkLayout chunk_layout(int eff_kind, bool half, long long B, long long L, long long count, int Hq, int Hkv, int D) {
   ChunkLayout c{};
   c.remote = eff_kind == ROPEATTN_BIFOCAL;
   c.tables = eff_kind != ROPEATTN_NOPE;
+  c.half = half;
   size_t off = 0;
   c.off_krem = off;
   if (c.remote) off += align_up(static_cast<size_t>(B) * L * Hkv * D * 2, 256);
@@ -495,6 +531,8 @@ ChunkLayout chunk_layout(int eff_kind, long long B, long long L, long long count
   if (c.tables) off += tab;
   c.off_tab1 = off;
   if (c.remote) off += tab;
+  c.off_q = off;
+  if (half) off += align_up(static_cast<size_t>(B) * count * Hq * D * 2, 256);
   c.total = off;
   return c;
 }
@@ -510,7 +548,7 @@ size_t ropeattn_prefill_chunk_workspace_size(const ropeattn_params* params, int6
   if (start < 0 || count < 0 || check_params(params, start + count, D, &m, &eff) ||
       check_shapes(B, start + count, Hq, Hkv, D))
     return 0;
-  return chunk_layout(eff, B, start + count, count, Hkv, D).total;
+  return chunk_layout(eff, half_pairing(params), B, start + count, count, Hq, Hkv, D).total;
 }
 
 int ropeattn_prefill_chunk(const void* q, const void* k_cache, const void* v_cache, float* out, float* lse,
@@ -544,7 +582,7 @@ int ropeattn_prefill_chunk_cache(const void* q, const void* k_cache, const void*
     return fail(ROPEATTN_ERR_INVALID_ARG, "too many query tiles");
   rc = check_device();
   if (rc) return rc;
-  const ChunkLayout lay = chunk_layout(eff, B, L, count, Hkv, D);
+  const ChunkLayout lay = chunk_layout(eff, half_pairing(params), B, L, count, Hq, Hkv, D);
   if (lay.total > 0) {
     if (!workspace || workspace_bytes < lay.total)
       return fail(ROPEATTN_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", lay.total,
@@ -579,6 +617,10 @@ int ropeattn_prefill_chunk_cache(const void* q, const void* k_cache, const void*
     pp.tab1 = a.tab1;
     if (lay.remote) kmap1 = a.k_rem;
   }
+  if (lay.half) {
+    if ((rc = launch_interleave(q, ws + lay.off_q, B * count * Hq, D, st))) return rc;
+    q = ws + lay.off_q;
+  }
   CUtensorMap tq, tk0, tk1, tv;
   if ((rc = make_map(&tq, q, D, Hq, count, B, 64, kBM, true))) return rc;
   if ((rc = make_map(&tk0, k_cache, D, Hkv, L, B, 64, kBN, true, cache_len))) return rc;
@@ -609,7 +651,7 @@ size_t ropeattn_prefill_three_call_workspace_size(const ropeattn_params* params,
   if (check_params(params, S, D, &m, &eff) || check_shapes(B, S, Hq, Hkv, D) || eff != ROPEATTN_BIFOCAL) return 0;
   const size_t o = align_up(static_cast<size_t>(B) * S * Hq * D * sizeof(float), 256);
   const size_t l = align_up(static_cast<size_t>(B) * Hq * S * sizeof(float), 256);
-  return prefill_layout(eff, B, S, Hkv, D).total + 2 * o + 2 * l;
+  return prefill_layout(eff, half_pairing(params), B, S, Hq, Hkv, D).total + 2 * o + 2 * l;
 }
 
 int ropeattn_prefill_three_call(const void* q, const void* k, const void* v, float* out, float* lse, int64_t B,
@@ -632,7 +674,7 @@ int ropeattn_prefill_three_call(const void* q, const void* k, const void* v, flo
     return fail(ROPEATTN_ERR_INVALID_ARG, "too many query tiles");
   rc = check_device();
   if (rc) return rc;
-  const PrefillLayout lay = prefill_layout(eff, B, S, Hkv, D);
+  const PrefillLayout lay = prefill_layout(eff, half_pairing(params), B, S, Hq, Hkv, D);
   const size_t obytes = align_up(static_cast<size_t>(B) * S * Hq * D * sizeof(float), 256);
   const size_t lbytes = align_up(static_cast<size_t>(B) * Hq * S * sizeof(float), 256);
   const size_t need = lay.total + 2 * obytes + 2 * lbytes;
@@ -660,11 +702,16 @@ int ropeattn_prefill_three_call(const void* q, const void* k, const void* v, flo
   a.S = static_cast<int>(S);
   a.Hkv = Hkv;
   a.D = D;
+  a.half = lay.half ? 1 : 0;
   a.m = m;
   fill_theta(params, D, a.theta);
   const int prow = 256 / (D / 2);
   rope_prep_kernel<<<static_cast<unsigned>((S + prow - 1) / prow), 256, 0, st>>>(a);
   CUDA_TRY(cudaGetLastError(), "rope_prep launch");
+  if (lay.half) {
+    if ((rc = launch_interleave(q, ws + lay.off_q, B * S * Hq, D, st))) return rc;
+    q = ws + lay.off_q;
+  }
 
   CUtensorMap tq, tk0, tk1, tv;
   if ((rc = make_map(&tq, q, D, Hq, S, B, 64, kBM, true))) return rc;
@@ -786,6 +833,10 @@ int ropeattn_decode_cache(const void* q, const void* k_cache, const void* v_cach
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
 
+  if (half_pairing(params)) {
+    if ((rc = launch_interleave(q, ws + lay.off_q, B * Hq, D, st))) return rc;
+    q = ws + lay.off_q;
+  }
   DecodeParams dp{};
   dp.q = static_cast<const __nv_bfloat16*>(q);
   dp.out = out;

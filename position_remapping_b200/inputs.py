@@ -25,6 +25,8 @@ import torch
 STANDARD, ENDPROMPT, PERIODIC, NOPE, BIFOCAL = 0, 1, 2, 3, 4
 KIND_NAMES = {STANDARD: "standard", ENDPROMPT: "endprompt", PERIODIC: "periodic",
               NOPE: "nope", BIFOCAL: "bifocal"}
+# coordinate pairing codes, identical to the C header's enum
+PAIR_ADJACENT, PAIR_HALF = 0, 1
 
 
 @dataclasses.dataclass(frozen=True)
@@ -40,6 +42,7 @@ class MapParams:
     w_pretrained: int = 0        # Jet-Long: pretrained context window
     fixed_group: int = 0         # bifocal with one fixed group size G (0: G from L, Eq. 2)
     softmax_scale: float = 0.0   # 0 -> 1/sqrt(D)
+    pairing: int = 0             # PAIR_ADJACENT (2i, 2i+1) or PAIR_HALF (i, i + D/2)
 
     def replace(self, **kw) -> "MapParams":
         return dataclasses.replace(self, **kw)

@@ -50,7 +50,8 @@ class CParams(ctypes.Structure):
         ("w0", ctypes.c_int64),
         ("w_pretrained", ctypes.c_int64),
         ("softmax_scale", ctypes.c_float),
-        ("reserved", ctypes.c_int32 * 3),
+        ("pairing", ctypes.c_int32),
+        ("reserved", ctypes.c_int32 * 2),
     ]
 
 
@@ -66,6 +67,7 @@ def to_cparams(p: MapParams) -> CParams:
     c.w0 = int(p.w0)
     c.w_pretrained = int(p.w_pretrained)
     c.softmax_scale = float(p.softmax_scale)
+    c.pairing = int(p.pairing)
     return c
 
 

@@ -50,12 +50,12 @@ def test_param_struct_layout_matches_c(ra):
 #include <stddef.h>
 #include "ropeattn.h"
 int main(void) {
-  printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(ropeattn_params),
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(ropeattn_params),
     offsetof(ropeattn_params, kind), offsetof(ropeattn_params, fixed_group),
     offsetof(ropeattn_params, rope_base), offsetof(ropeattn_params, interp),
     offsetof(ropeattn_params, seg1_len), offsetof(ropeattn_params, term_start), offsetof(ropeattn_params, window),
     offsetof(ropeattn_params, w0), offsetof(ropeattn_params, w_pretrained), offsetof(ropeattn_params, softmax_scale),
-    offsetof(ropeattn_params, reserved));
+    offsetof(ropeattn_params, pairing), offsetof(ropeattn_params, reserved));
   return 0;
 }
 '''
@@ -68,7 +68,7 @@ int main(void) {
     P = ra.CParams
     want = [ctypes.sizeof(P)] + [getattr(P, f).offset for f in
             ("kind", "fixed_group", "rope_base", "interp", "seg1_len", "term_start", "window", "w0", "w_pretrained",
-             "softmax_scale", "reserved")]
+             "softmax_scale", "pairing", "reserved")]
     assert got == want
 
 
@@ -96,7 +96,8 @@ def test_host_argument_checks(ra):
                                ctypes.byref(cp(_p(kind=STANDARD))), nullp, 0, nullp) == ra.ERR_INVALID_ARG  # GQA 8
     bad = [_p(kind=9), _p(kind=PERIODIC, window=0), _p(kind=BIFOCAL, w0=-1, w_pretrained=8),
            _p(kind=BIFOCAL, w0=4, w_pretrained=0), _p(kind=ENDPROMPT, interp=0.5),
-           _p(kind=STANDARD, rope_base=1.0), _p(kind=STANDARD, softmax_scale=-1.0)]
+           _p(kind=STANDARD, rope_base=1.0), _p(kind=STANDARD, softmax_scale=-1.0),
+           _p(kind=STANDARD, pairing=2), _p(kind=BIFOCAL, w0=4, w_pretrained=8, pairing=-1)]
     for p in bad:
         rc = lib.ropeattn_prefill(nullp, nullp, nullp, nullp, nullp, 1, 16, 2, 1, 64,
                                   ctypes.byref(cp(p)), nullp, 0, nullp)
@@ -158,3 +159,9 @@ def test_workspace_sizes(ra):
     short = w.params.replace(w_pretrained=1 << 20)
     assert ra.prefill_workspace_size(short, 1, 4096, 32, 8, 128) == 4096 * 8 * 128 * 2 + 4096 * 64 * 8
     assert ra.decode_workspace_size(1, 131072, 16, 8, 128) > 0
+    # half-split pairing adds a copy of q in adjacent order (not for NOPE, which rotates nothing)
+    half = w.params.replace(pairing=1)
+    assert ra.prefill_workspace_size(half, w.B, w.S, w.Hq, w.Hkv, w.D) == n + w.B * w.S * w.Hq * w.D * 2
+    assert ra.prefill_workspace_size(nope.params.replace(pairing=1), nope.B, nope.S, nope.Hq, nope.Hkv, nope.D) == 0
+    assert (ra.prefill_chunk_workspace_size(half, 1, 4096, 1000, 32, 8, 128) ==
+            ra.prefill_chunk_workspace_size(w.params, 1, 4096, 1000, 32, 8, 128) + 1000 * 32 * 128 * 2)
