@@ -54,7 +54,7 @@ __all__ = [
     "STANDARD", "ENDPROMPT", "PERIODIC", "NOPE", "BIFOCAL", "PAIR_ADJACENT", "PAIR_HALF",
     "round_bf16", "rope_frequencies", "pair_index", "rotation_matrix", "rotate",
     "periodic_position", "endprompt_position", "group_size", "bifocal_group", "remote_position",
-    "position_maps", "softmax_scale", "prefill", "prefill_three_call",
+    "position_maps", "softmax_scale", "prefill", "prefill_three_call", "prefill_backward",
     "decode", "cache_keys", "prefill_from_cache", "brute_prefill", "brute_decode", "to_f64",
 ]
 
@@ -309,6 +309,70 @@ def prefill_three_call(q, k, v, params, stage_bf16: bool = True):
             out[b, :, h] = (WA[:, None] * OA + WB[:, None] * OB - WC[:, None] * OC) / den[:, None]
             lse[b, h] = M + np.log(den)
     return out, lse
+
+
+# ----------------------------------------------------------------------------
+# backward of the prefill: gradients of a scalar loss through the routed
+# softmax (the fine-tuning pass EndPrompt's method needs)
+# ----------------------------------------------------------------------------
+def prefill_backward(q, k, v, dout, params):
+    """(dq, dk, dv) of the prefill (unstaged, float64) for an upstream
+    gradient ``dout`` of ``out`` [B,S,Hq,D]; shapes of q, k, v.
+
+    With P the row softmax of scale * score(t,s) over the allowed keys and
+    score(t,s) = <R_a q_t, R_b k_s> ((a, b) the positions the kind assigns
+    to the pair; for BIFOCAL (t, s) inside the local window, (f(t), f(s))
+    outside it), the chain rule gives
+      dv_s  = sum_t P(t,s) dout_t
+      dP    = dout_t . v_s,     dS(t,s) = P(t,s) (dP(t,s) - sum_s' P(t,s') dP(t,s'))
+      dq_t  = scale * sum_s dS(t,s) R_a^T R_b k_s
+      dk_s  = scale * sum_t dS(t,s) R_b^T R_a q_t
+    (R^T = R of the negated position). For BIFOCAL the sums split by the
+    window into a local part (map t) and a remote part (map f). dk and dv of
+    a KV head collect the heads of its GQA group."""
+    q, k, v, dout = to_f64(q), to_f64(k), to_f64(v), to_f64(dout)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    grp = Hq // Hkv
+    scale = softmax_scale(D, params)
+    kind = int(params.kind)
+    freqs = _freqs(params, D)
+    pr = _pairing(params)
+    p_loc, p_rem, _G = position_maps(params, S)
+    t = np.arange(S)
+    ok = np.stack([_allowed(params, int(r), t) for r in t])          # [S, S]
+    local = (t[:, None] - t[None, :]) <= int(params.w0)
+
+    def rot(x, pos):
+        return x if kind == NOPE else rotate(x, pos, freqs, pr)
+
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // grp
+            ql, kl = rot(q[b, :, h], p_loc), rot(k[b, :, hk], p_loc)
+            sc = ql @ kl.T
+            if kind == BIFOCAL:
+                qr, kr = rot(q[b, :, h], p_rem), rot(k[b, :, hk], p_rem)
+                sc = np.where(local, sc, qr @ kr.T)
+            sc = np.where(ok, sc * scale, -np.inf)
+            m = sc.max(axis=1, keepdims=True)
+            e = np.where(ok, np.exp(sc - m), 0.0)
+            P = e / e.sum(axis=1, keepdims=True)
+            do = dout[b, :, h]
+            dv[b, :, hk] += P.T @ do
+            dP = do @ v[b, :, hk].T
+            dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))
+            if kind == BIFOCAL:
+                dSl, dSr = np.where(local, dS, 0.0), np.where(local, 0.0, dS)
+                dq[b, :, h] += scale * (rot(dSl @ kl, -p_loc) + rot(dSr @ kr, -p_rem))
+                dk[b, :, hk] += scale * (rot(dSl.T @ ql, -p_loc) + rot(dSr.T @ qr, -p_rem))
+            else:
+                dq[b, :, h] += scale * rot(dS @ kl, -p_loc)
+                dk[b, :, hk] += scale * rot(dS.T @ ql, -p_loc)
+    return dq, dk, dv
 
 
 # ----------------------------------------------------------------------------

@@ -569,3 +569,71 @@ def test_half_split_cache_and_decode(kind):
     a = O.decode(qn, cache, vn, params)
     b = O.brute_decode(qn, kn, vn, params)
     assert np.allclose(a[0], b[0], atol=1e-12) and np.allclose(a[1], b[1], atol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# backward of the prefill
+# ----------------------------------------------------------------------------
+_BWD_PARAMS = [
+    ("standard", MapParams(O.STANDARD, rope_base=1e2)),
+    ("endprompt", MapParams(O.ENDPROMPT, rope_base=1e3, interp=2.0, seg1_len=4, term_start=40)),
+    ("periodic", MapParams(O.PERIODIC, rope_base=1e2, window=4)),
+    ("nope", MapParams(O.NOPE)),
+    ("bifocal", MapParams(O.BIFOCAL, rope_base=1e2, w0=2, w_pretrained=4)),
+    ("bifocal_half", MapParams(O.BIFOCAL, rope_base=1e2, w0=1, w_pretrained=3, pairing=1)),
+    ("bifocal_fixed", MapParams(O.BIFOCAL, rope_base=1e2, w0=3, fixed_group=2)),
+]
+
+
+@pytest.mark.parametrize("case", _BWD_PARAMS, ids=[c[0] for c in _BWD_PARAMS])
+def test_backward_matches_finite_differences(case):
+    # d/dx of sum(dout * out) by central differences of the forward oracle,
+    # every element of q, k and v (GQA group of 2 so dk, dv collect heads)
+    _, params = case
+    rng = np.random.default_rng(61)
+    B, S, Hq, Hkv, D = 1, 9, 2, 1, 4
+    q, k, v = (rng.standard_normal(s) for s in ((B, S, Hq, D), (B, S, Hkv, D), (B, S, Hkv, D)))
+    dout = rng.standard_normal((B, S, Hq, D))
+    dq, dk, dv = O.prefill_backward(q, k, v, dout, params)
+
+    def loss(qq, kk, vv):
+        return float((O.prefill(qq, kk, vv, params, stage_bf16=False)[0] * dout).sum())
+
+    h = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args = {"q": (q, k, v), "k": (q, k, v), "v": (q, k, v)}[name]
+            ap = [xp if a is x else a for a in args]
+            am = [xm if a is x else a for a in args]
+            fd[idx] = (loss(*ap) - loss(*am)) / (2 * h)
+        assert np.allclose(g, fd, rtol=1e-6, atol=1e-8), (name, np.abs(g - fd).max())
+
+
+def test_backward_closed_forms():
+    rng = np.random.default_rng(62)
+    params = MapParams(O.BIFOCAL, rope_base=1e4, w0=2, w_pretrained=4)
+    # one token: out = v_0, so dv = dout summed over the group, dq = dk = 0
+    q, k, v = rng.standard_normal((1, 1, 4, 8)), rng.standard_normal((1, 1, 2, 8)), rng.standard_normal((1, 1, 2, 8))
+    dout = rng.standard_normal((1, 1, 4, 8))
+    dq, dk, dv = O.prefill_backward(q, k, v, dout, params)
+    assert np.array_equal(dq, np.zeros_like(dq)) and np.array_equal(dk, np.zeros_like(dk))
+    assert np.allclose(dv[0, 0, 0], dout[0, 0, 0] + dout[0, 0, 1]) and np.allclose(dv[0, 0, 1], dout[0, 0, 2] + dout[0, 0, 3])
+    # zero queries: uniform attention over the allowed keys, so dk = 0 and
+    # dv_s = sum over rows t that allow s of dout_t / (number of keys of t)
+    S = 11
+    for p in (params, MapParams(O.PERIODIC, window=3)):
+        q = np.zeros((1, S, 1, 8))
+        k, v = rng.standard_normal((1, S, 1, 8)), rng.standard_normal((1, S, 1, 8))
+        dout = rng.standard_normal((1, S, 1, 8))
+        _, dk, dv = O.prefill_backward(q, k, v, dout, p)
+        assert np.allclose(dk, 0.0, atol=1e-15)
+        want = np.zeros((S, 8))
+        for t in range(S):
+            keys = [s for s in range(S) if s <= t and (p.kind != O.PERIODIC or s > t - p.window)]
+            for s in keys:
+                want[s] += dout[0, t, 0] / len(keys)
+        assert np.allclose(dv[0, :, 0], want, atol=1e-13)
