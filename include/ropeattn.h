@@ -24,7 +24,8 @@
  *           position; v_cache [B, n, Hkv, D] bf16; out [B, Hq, D] fp32;
  *           lse [B, Hq] fp32.
  *   GQA: query head h reads key/value head h / (Hq / Hkv).
- *   Supported: D in {64, 128} (decode and cache writes also 256);
+ *   Supported: D in {64, 128, 256} (the prefill runs D = 256 with one
+ *   128-row query tile per CTA and 64-key tiles);
  *   Hq % Hkv == 0; decode also needs Hq / Hkv <= 2 for D = 256, <= 4 for
  *   D = 128 and <= 8 for D = 64.
  *   Half-split pairing (params.pairing = ROPEATTN_PAIR_HALF): q, k and v are

@@ -1,7 +1,8 @@
 // Causal prefill attention with RoPE at remapped positions, sm_100a.
 //
 // One CTA computes two 128-row query tiles (256 consecutive rows) of one
-// (batch, query head) against the key tiles of its passes:
+// (batch, query head) against the 128-key tiles of its passes (D = 64, 128;
+// at D = 256 one query tile against 64-key tiles, see PrefillShape):
 //   warps 0-3, 4-7  softmax warpgroups, one per query tile (one TMEM lane =
 //              one query row per thread): rotate the staged query tile in
 //              shared memory, then per key tile copy S from TMEM into
@@ -28,7 +29,11 @@
 //              warpgroups with setmaxnreg: 216 per softmax thread, 72 per
 //              thread of warps 8-11; 384 x 168 at launch = 256 x 216 + 128 x 72.
 // TMEM (512 columns): S [0,128), P0 [128,192), P1 [192,256) (bf16 pairs),
-// O0 [256,256+D), O1 [256+D, 256+2D).
+// O0 [256,256+D), O1 [256+D, 256+2D). At D = 256 the single tile's S, P and
+// O take [0,64), [128,160) and [256,512); the warp roles shift down by the
+// missing softmax warpgroup (TMA warp 4, QK warp 5, PV warp 6), and every
+// thread keeps its launch registers (seven warps are not whole warpgroups,
+// and 224 threads x 255 registers fit the register file).
 //
 // A pass is a sweep over key tiles with one query rotation, one key tensor
 // and one distance band hi_off <= t - s <= lo_off:
@@ -54,13 +59,24 @@
 namespace ropeattn {
 
 constexpr int kBM = 128;               // rows per query tile (TMEM lanes)
-constexpr int kQT = 2;                 // query tiles per CTA
-constexpr int kBlockRows = kBM * kQT;  // query rows per CTA
-constexpr int kBN = 128;               // keys per tile
-constexpr int kPrefillThreads = 384;
-constexpr int kSoftmaxRegs = 216;      // per thread of warps 0-7 after setmaxnreg
-constexpr int kProducerRegs = 72;      // per thread of warps 8-11 after setmaxnreg
+constexpr int kSoftmaxRegs = 216;      // per thread of warps 0-7 after setmaxnreg (two tiles)
+constexpr int kProducerRegs = 72;      // per thread of warps 8-11 after setmaxnreg (two tiles)
 constexpr int kInf = 0x3fffffff;
+
+// Tile schedule per head dimension. D <= 128: two query tiles per CTA, 128
+// keys per tile. D = 256: one query tile per CTA (its O accumulator takes 256
+// TMEM columns) and 64 keys per tile (a 64 KiB query tile and four 32 KiB
+// K/V slots fit shared memory).
+template <int D>
+struct PrefillShape {
+  static constexpr int kQT = D == 256 ? 1 : 2;          // query tiles per CTA
+  static constexpr int kBN = D == 256 ? 64 : 128;       // keys per tile
+  static constexpr int kBlockRows = kBM * kQT;          // query rows per CTA
+  static constexpr int kWarpTMA = 4 * kQT;              // warp roles after the softmax warps
+  static constexpr int kWarpQK = kWarpTMA + 1;
+  static constexpr int kWarpPV = kWarpTMA + 2;          // kQT PV issuers
+  static constexpr int kThreads = 32 * (kWarpPV + kQT);
+};
 
 struct PrefillParams {
   float* out;          // [B, S, Hq, D]
@@ -70,7 +86,7 @@ struct PrefillParams {
   int B, S, Hq, Hkv;   // S: query rows
   int Sk;              // keys (rows of K and V); S for a whole prefill
   int q_off;           // absolute position index of query row 0 (0 for a whole prefill)
-  int nqb;             // 256-row query blocks per (b, h)
+  int nqb;             // query blocks (PrefillShape::kBlockRows rows) per (b, h)
   int kind;
   int window;          // Periodic RoPE
   int w0;              // Jet-Long
@@ -86,7 +102,7 @@ struct PassDesc {
   int sel;             // 0: main or local map, 1: remote map
 };
 
-__device__ __forceinline__ int make_passes(const PrefillParams& p, int q0, PassDesc* ps) {
+__device__ __forceinline__ int make_passes(const PrefillParams& p, int q0, int block_rows, int bn, PassDesc* ps) {
   int bands[2][3];  // lo_off, hi_off, sel
   int nb = 0;
   if (p.forced) {
@@ -105,15 +121,15 @@ __device__ __forceinline__ int make_passes(const PrefillParams& p, int q0, PassD
   }
   // absolute positions of the block's first and last query rows
   const int t_first = p.q_off + q0;
-  const int t_last = p.q_off + min(p.S - 1, q0 + kBlockRows - 1);
+  const int t_last = p.q_off + min(p.S - 1, q0 + block_rows - 1);
   int n = 0;
   for (int i = 0; i < nb; ++i) {
     const int lo_off = bands[i][0], hi_off = bands[i][1];
     const int s_min = lo_off >= kInf ? 0 : max(0, t_first - lo_off);
     const int s_max = min(p.Sk - 1, t_last - hi_off);
     if (s_max < s_min) continue;
-    ps[n].j_lo = s_min / kBN;
-    ps[n].j_hi = s_max / kBN;
+    ps[n].j_lo = s_min / bn;
+    ps[n].j_hi = s_max / bn;
     ps[n].lo_off = lo_off;
     ps[n].hi_off = hi_off;
     ps[n].sel = bands[i][2];
@@ -124,10 +140,10 @@ __device__ __forceinline__ int make_passes(const PrefillParams& p, int q0, PassD
 
 template <int D, int NSLOT>
 struct PrefillSmem {
-  static constexpr int kQBytes = kBM * D * 2;     // one query tile
-  static constexpr int kTileBytes = kBN * D * 2;  // one K or V tile
+  static constexpr int kQBytes = kBM * D * 2;                       // one query tile
+  static constexpr int kTileBytes = PrefillShape<D>::kBN * D * 2;   // one K or V tile
   static constexpr int kQ = 0;
-  static constexpr int kRing = kQ + kQT * kQBytes;
+  static constexpr int kRing = kQ + PrefillShape<D>::kQT * kQBytes;
   static constexpr int kBar = kRing + NSLOT * kTileBytes;
   // barriers: q_full, q_ready[2], q_free, ring_full[NSLOT], ring_empty[NSLOT],
   // s_full[2], s_free, p_full[2], o_done[2], o_free[2]
@@ -138,14 +154,19 @@ struct PrefillSmem {
 };
 
 template <int D, int NSLOT>
-__global__ void __launch_bounds__(kPrefillThreads, 1)
+__global__ void __launch_bounds__(PrefillShape<D>::kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK0,
                    const __grid_constant__ CUtensorMap tmK1, const __grid_constant__ CUtensorMap tmV,
                    const PrefillParams p) {
   using L = PrefillSmem<D, NSLOT>;
+  using SH = PrefillShape<D>;
+  constexpr int kQT = SH::kQT;
+  constexpr int kBN = SH::kBN;
+  constexpr int kBlockRows = SH::kBlockRows;
   static_assert(NSLOT % 2 == 0, "K and V tiles alternate over an even number of ring slots");
   constexpr int kCB = D / 64;              // 64-column (128-byte) swizzle blocks per row
-  constexpr int kBlockBytes = kBM * 128;   // one swizzle block of a 128-row tile
+  constexpr int kBlockBytes = kBM * 128;   // one swizzle block of a query tile
+  constexpr int kKVBlockBytes = kBN * 128; // one swizzle block of a K or V tile
   constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, false);
   constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, true);
   constexpr uint32_t kTmemCols = 512;
@@ -186,7 +207,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const int q0 = qb * kBlockRows;
 
   PassDesc passes[2];
-  const int npass = make_passes(p, q0, passes);
+  const int npass = make_passes(p, q0, kBlockRows, kBN, passes);
 
   if (tid == 0) {
     mbar_init(q_full, 1);
@@ -194,10 +215,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     mbar_init(q_ready + 1, kBM);
     mbar_init(q_free, 1);
     // K tiles sit at even ring positions (released by the QK issuer), V tiles
-    // at odd ones (released by both PV issuers); NSLOT is even
+    // at odd ones (released by every PV issuer); NSLOT is even
     for (int i = 0; i < NSLOT; ++i) {
       mbar_init(ring_full + i, 1);
-      mbar_init(ring_empty + i, (i & 1) ? 2 : 1);
+      mbar_init(ring_empty + i, (i & 1) ? kQT : 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(s_full + a, 1);
@@ -213,7 +234,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == SH::kWarpTMA && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK0);
     tma_prefetch_desc(&tmK1);
@@ -227,9 +248,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const uint32_t tP = tmem + 128;      // P_a at 128 + 64 a
   const uint32_t tO = tmem + 256;      // O_a at 256 + a D
 
-  if (warp == 8) {
+  if (warp == SH::kWarpTMA) {
     // ------------------------------------------------------------------ TMA
-    reg_dealloc<kProducerRegs>();
+    if constexpr (kQT == 2) reg_dealloc<kProducerRegs>();
     if (lane == 0) {
       int pos = 0;
       bool ok = true;
@@ -248,19 +269,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             mbar_arrive_expect_tx(ring_full + slot, L::kTileBytes);
             uint8_t* dst = sRing + slot * L::kTileBytes;
             for (int cb = 0; cb < kCB; ++cb)
-              tma_load_4d(dst + cb * kBlockBytes, kv ? &tmV : tk, ring_full + slot, cb * 64, hk, j * kBN, b);
+              tma_load_4d(dst + cb * kKVBlockBytes, kv ? &tmV : tk, ring_full + slot, cb * 64, hk, j * kBN, b);
           }
         }
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == SH::kWarpQK) {
     // ---------------------------------------------------------- MMA: QK^T
-    reg_dealloc<kProducerRegs>();
+    if constexpr (kQT == 2) reg_dealloc<kProducerRegs>();
     if (lane == 0) {
       int pos = 0, nqk = 0;
       bool ok = true;
       for (int pi = 0; pi < npass && ok; ++pi) {
-        if (!mbar_wait(q_ready + 0, pi & 1, abort_flag) || !mbar_wait(q_ready + 1, pi & 1, abort_flag)) break;
+        if (!mbar_wait(q_ready + 0, pi & 1, abort_flag) ||
+            (kQT == 2 && !mbar_wait(q_ready + 1, pi & 1, abort_flag)))
+          break;
         const int T = passes[pi].j_hi - passes[pi].j_lo + 1;
         for (int i = 0; i < T && ok; ++i, pos += 2) {
           const int kslot = pos % NSLOT;
@@ -273,9 +296,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             const uint32_t qaddr = smem_u32(sQ + a * L::kQBytes);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * kBlockBytes + (kk & 3) * 32;
-              umma_ss(tS, sdesc_sw128(qaddr + off, 16, 1024), sdesc_sw128(kaddr + off, 16, 1024), kIdescQK,
-                      kk > 0 ? 1u : 0u);
+              const uint32_t kin = (kk & 3) * 32;   // K step inside a 64-column swizzle block
+              umma_ss(tS, sdesc_sw128(qaddr + (kk >> 2) * kBlockBytes + kin, 16, 1024),
+                      sdesc_sw128(kaddr + (kk >> 2) * kKVBlockBytes + kin, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
             }
             umma_commit(s_full + a);
             ++nqk;
@@ -286,11 +309,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
       }
     }
-  } else if (warp == 10 || warp == 11) {
-    // --------------------------------------------- MMA: PV of tile warp - 10
-    reg_dealloc<kProducerRegs>();
+  } else if (warp >= SH::kWarpPV) {
+    // ------------------------------------- MMA: PV of tile warp - kWarpPV
+    if constexpr (kQT == 2) reg_dealloc<kProducerRegs>();
     if (lane == 0) {
-      const int a = warp - 10;
+      const int a = warp - SH::kWarpPV;
       int pos = 0, g = 0;
       bool ok = true;
       for (int pi = 0; pi < npass && ok; ++pi) {
@@ -306,7 +329,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           const uint32_t vaddr = smem_u32(sRing + vslot * L::kTileBytes);
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk) {
-            const uint64_t bdesc = sdesc_sw128(vaddr + kk * 2048, kBlockBytes, 1024);
+            const uint64_t bdesc = sdesc_sw128(vaddr + kk * 2048, kKVBlockBytes, 1024);
             umma_ts(tO + a * D, tP + a * 64 + kk * 8, bdesc, kIdescPV, (kk > 0 || i > 0) ? 1u : 0u);
           }
           umma_commit(o_done + a);
@@ -316,7 +339,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
   } else {
     // -------------------------------------------------------------- softmax
-    reg_alloc<kSoftmaxRegs>();
+    if constexpr (kQT == 2) reg_alloc<kSoftmaxRegs>();
     const int a = warp >> 2;                 // query tile of this warpgroup
     const int row = tid & (kBM - 1);         // TMEM lane == row in the tile
     const int qa0 = q0 + a * kBM;

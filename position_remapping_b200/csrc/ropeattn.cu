@@ -207,13 +207,12 @@ float scale_log2(const ropeattn_params* p, int D) {
   return static_cast<float>(sc * 1.4426950408889634074);
 }
 
-// Shapes every entry point accepts; the attention kernels of prefill take
-// D = 64 or 128 (two O accumulators of D fp32 columns share TMEM with S and
-// P), the decode and cache kernels also D = 256 (allow256).
-int check_shapes(long long B, long long S, int Hq, int Hkv, int D, bool allow256 = false) {
+// Shapes every entry point accepts: D = 64, 128 or 256 (the prefill runs
+// D = 256 with one query tile per CTA, PrefillShape).
+int check_shapes(long long B, long long S, int Hq, int Hkv, int D) {
   if (B < 0 || S < 0) return fail(ROPEATTN_ERR_INVALID_ARG, "B and S must be >= 0");
-  if (D != 64 && D != 128 && !(allow256 && D == 256))
-    return fail(ROPEATTN_ERR_INVALID_ARG, allow256 ? "D must be 64, 128 or 256 (got %d)" : "D must be 64 or 128 (got %d)", D);
+  if (D != 64 && D != 128 && D != 256)
+    return fail(ROPEATTN_ERR_INVALID_ARG, "D must be 64, 128 or 256 (got %d)", D);
   if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0)
     return fail(ROPEATTN_ERR_INVALID_ARG, "need Hq >= 1, Hkv >= 1 and Hq %% Hkv == 0 (Hq=%d Hkv=%d)", Hq, Hkv);
   if (S > kMaxPos || B > 65535 || Hq > 65535) return fail(ROPEATTN_ERR_INVALID_ARG, "shape too large");
@@ -254,9 +253,21 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk0, const CUtensor
     attr_err = cudaFuncSetAttribute(prefill_kernel<D, NST>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(prefill)");
-  prefill_kernel<D, NST><<<grid, kPrefillThreads, L::kAlloc, st>>>(tq, tk0, tk1, tv, pp);
+  prefill_kernel<D, NST><<<grid, PrefillShape<D>::kThreads, L::kAlloc, st>>>(tq, tk0, tk1, tv, pp);
   CUDA_TRY(cudaGetLastError(), "prefill launch");
   return ROPEATTN_OK;
+}
+
+// Query rows per CTA and keys per K/V tile of the prefill kernel (PrefillShape).
+int prefill_block_rows(int D) { return D == 256 ? PrefillShape<256>::kBlockRows : PrefillShape<128>::kBlockRows; }
+int prefill_bn(int D) { return D == 256 ? PrefillShape<256>::kBN : PrefillShape<128>::kBN; }
+
+// One prefill attention launch for the head dimension.
+int launch_prefill_d(int D, const CUtensorMap& tq, const CUtensorMap& tk0, const CUtensorMap& tk1,
+                     const CUtensorMap& tv, const PrefillParams& pp, int grid, cudaStream_t st) {
+  if (D == 256) return launch_prefill<256, 4>(tq, tk0, tk1, tv, pp, grid, st);
+  if (D == 128) return launch_prefill<128, 4>(tq, tk0, tk1, tv, pp, grid, st);
+  return launch_prefill<64, 8>(tq, tk0, tk1, tv, pp, grid, st);
 }
 
 struct DecodeLayout {
@@ -372,7 +383,7 @@ int ropeattn_cache_write(const void* k, const void* v, void* k_cache, void* v_ca
   if (start + count > cache_len)
     return fail(ROPEATTN_ERR_INVALID_ARG, "start + count (%lld) exceeds cache_len (%lld)",
                 static_cast<long long>(start + count), static_cast<long long>(cache_len));
-  int rc = check_shapes(B, cache_len, Hkv, Hkv, D, true);
+  int rc = check_shapes(B, cache_len, Hkv, Hkv, D);
   if (rc) return rc;
   PosMap m;
   int eff;
@@ -440,7 +451,7 @@ int prefill_impl(int stages, const void* q, const void* k, const void* v, float*
     if (!aligned16(q) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
       return fail(ROPEATTN_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
   }
-  if ((static_cast<long long>((S + kBlockRows - 1) / kBlockRows)) * Hq * B > 0x7fffffffLL)
+  if ((static_cast<long long>((S + prefill_block_rows(D) - 1) / prefill_block_rows(D))) * Hq * B > 0x7fffffffLL)
     return fail(ROPEATTN_ERR_INVALID_ARG, "too many query tiles");
   rc = check_device();
   if (rc) return rc;
@@ -492,9 +503,9 @@ int prefill_impl(int stages, const void* q, const void* k, const void* v, float*
 
   CUtensorMap tq, tk0, tk1, tv;
   if ((rc = make_map(&tq, q, D, Hq, S, B, 64, kBM, true))) return rc;
-  if ((rc = make_map(&tk0, kmap0, D, Hkv, S, B, 64, kBN, true))) return rc;
-  if ((rc = make_map(&tk1, kmap1, D, Hkv, S, B, 64, kBN, true))) return rc;
-  if ((rc = make_map(&tv, v, D, Hkv, S, B, 64, kBN, true))) return rc;
+  if ((rc = make_map(&tk0, kmap0, D, Hkv, S, B, 64, prefill_bn(D), true))) return rc;
+  if ((rc = make_map(&tk1, kmap1, D, Hkv, S, B, 64, prefill_bn(D), true))) return rc;
+  if ((rc = make_map(&tv, v, D, Hkv, S, B, 64, prefill_bn(D), true))) return rc;
   pp.out = out;
   pp.lse = lse;
   pp.B = static_cast<int>(B);
@@ -503,14 +514,13 @@ int prefill_impl(int stages, const void* q, const void* k, const void* v, float*
   pp.q_off = 0;
   pp.Hq = Hq;
   pp.Hkv = Hkv;
-  pp.nqb = static_cast<int>((S + kBlockRows - 1) / kBlockRows);
+  pp.nqb = static_cast<int>((S + prefill_block_rows(D) - 1) / prefill_block_rows(D));
   pp.kind = eff;
   pp.window = m.window;
   pp.w0 = m.w0;
   pp.scale_log2 = scale_log2(params, D);
   const int grid = pp.nqb * Hq * static_cast<int>(B);
-  if (D == 128) return launch_prefill<128, 4>(tq, tk0, tk1, tv, pp, grid, st);
-  return launch_prefill<64, 8>(tq, tk0, tk1, tv, pp, grid, st);
+  return launch_prefill_d(D, tq, tk0, tk1, tv, pp, grid, st);
 }
 
 struct ChunkLayout {
@@ -578,7 +588,7 @@ int ropeattn_prefill_chunk_cache(const void* q, const void* k_cache, const void*
   if (!q || !k_cache || !v_cache || !out || !lse) return fail(ROPEATTN_ERR_INVALID_ARG, "null tensor pointer");
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || !aligned16(lse))
     return fail(ROPEATTN_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
-  if ((static_cast<long long>((count + kBlockRows - 1) / kBlockRows)) * Hq * B > 0x7fffffffLL)
+  if ((static_cast<long long>((count + prefill_block_rows(D) - 1) / prefill_block_rows(D))) * Hq * B > 0x7fffffffLL)
     return fail(ROPEATTN_ERR_INVALID_ARG, "too many query tiles");
   rc = check_device();
   if (rc) return rc;
@@ -623,9 +633,9 @@ int ropeattn_prefill_chunk_cache(const void* q, const void* k_cache, const void*
   }
   CUtensorMap tq, tk0, tk1, tv;
   if ((rc = make_map(&tq, q, D, Hq, count, B, 64, kBM, true))) return rc;
-  if ((rc = make_map(&tk0, k_cache, D, Hkv, L, B, 64, kBN, true, cache_len))) return rc;
-  if ((rc = make_map(&tk1, kmap1, D, Hkv, L, B, 64, kBN, true, lay.remote ? 0 : cache_len))) return rc;
-  if ((rc = make_map(&tv, v_cache, D, Hkv, L, B, 64, kBN, true, cache_len))) return rc;
+  if ((rc = make_map(&tk0, k_cache, D, Hkv, L, B, 64, prefill_bn(D), true, cache_len))) return rc;
+  if ((rc = make_map(&tk1, kmap1, D, Hkv, L, B, 64, prefill_bn(D), true, lay.remote ? 0 : cache_len))) return rc;
+  if ((rc = make_map(&tv, v_cache, D, Hkv, L, B, 64, prefill_bn(D), true, cache_len))) return rc;
   pp.out = out;
   pp.lse = lse;
   pp.B = static_cast<int>(B);
@@ -634,14 +644,13 @@ int ropeattn_prefill_chunk_cache(const void* q, const void* k_cache, const void*
   pp.q_off = static_cast<int>(start);
   pp.Hq = Hq;
   pp.Hkv = Hkv;
-  pp.nqb = static_cast<int>((count + kBlockRows - 1) / kBlockRows);
+  pp.nqb = static_cast<int>((count + prefill_block_rows(D) - 1) / prefill_block_rows(D));
   pp.kind = eff;
   pp.window = m.window;
   pp.w0 = m.w0;
   pp.scale_log2 = scale_log2(params, D);
   const int grid = pp.nqb * Hq * static_cast<int>(B);
-  if (D == 128) return launch_prefill<128, 4>(tq, tk0, tk1, tv, pp, grid, st);
-  return launch_prefill<64, 8>(tq, tk0, tk1, tv, pp, grid, st);
+  return launch_prefill_d(D, tq, tk0, tk1, tv, pp, grid, st);
 }
 
 size_t ropeattn_prefill_three_call_workspace_size(const ropeattn_params* params, int64_t B, int64_t S, int32_t Hq,
@@ -670,7 +679,7 @@ int ropeattn_prefill_three_call(const void* q, const void* k, const void* v, flo
   if (!q || !k || !v || !out || !lse) return fail(ROPEATTN_ERR_INVALID_ARG, "null tensor pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
     return fail(ROPEATTN_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
-  if ((static_cast<long long>((S + kBlockRows - 1) / kBlockRows)) * Hq * B > 0x7fffffffLL)
+  if ((static_cast<long long>((S + prefill_block_rows(D) - 1) / prefill_block_rows(D))) * Hq * B > 0x7fffffffLL)
     return fail(ROPEATTN_ERR_INVALID_ARG, "too many query tiles");
   rc = check_device();
   if (rc) return rc;
@@ -715,9 +724,9 @@ int ropeattn_prefill_three_call(const void* q, const void* k, const void* v, flo
 
   CUtensorMap tq, tk0, tk1, tv;
   if ((rc = make_map(&tq, q, D, Hq, S, B, 64, kBM, true))) return rc;
-  if ((rc = make_map(&tk0, a.k_rot0, D, Hkv, S, B, 64, kBN, true))) return rc;
-  if ((rc = make_map(&tk1, a.k_rot1, D, Hkv, S, B, 64, kBN, true))) return rc;
-  if ((rc = make_map(&tv, v, D, Hkv, S, B, 64, kBN, true))) return rc;
+  if ((rc = make_map(&tk0, a.k_rot0, D, Hkv, S, B, 64, prefill_bn(D), true))) return rc;
+  if ((rc = make_map(&tk1, a.k_rot1, D, Hkv, S, B, 64, prefill_bn(D), true))) return rc;
+  if ((rc = make_map(&tv, v, D, Hkv, S, B, 64, prefill_bn(D), true))) return rc;
   PrefillParams pp{};
   pp.tab0 = a.tab0;
   pp.tab1 = a.tab1;
@@ -727,7 +736,7 @@ int ropeattn_prefill_three_call(const void* q, const void* k, const void* v, flo
   pp.q_off = 0;
   pp.Hq = Hq;
   pp.Hkv = Hkv;
-  pp.nqb = static_cast<int>((S + kBlockRows - 1) / kBlockRows);
+  pp.nqb = static_cast<int>((S + prefill_block_rows(D) - 1) / prefill_block_rows(D));
   pp.kind = ROPEATTN_STANDARD;   // each call writes its own normalised output and LSE
   pp.window = m.window;
   pp.w0 = m.w0;
@@ -745,8 +754,7 @@ int ropeattn_prefill_three_call(const void* q, const void* k, const void* v, flo
     pp.forced_sel = calls[c][2];
     pp.out = outs[c];
     pp.lse = lses[c];
-    rc = D == 128 ? launch_prefill<128, 4>(tq, tk0, tk1, tv, pp, grid, st)
-                  : launch_prefill<64, 8>(tq, tk0, tk1, tv, pp, grid, st);
+    rc = launch_prefill_d(D, tq, tk0, tk1, tv, pp, grid, st);
     if (rc) return rc;
   }
   MergeArgs ma{};
@@ -786,7 +794,7 @@ int ropeattn_prefill_attend(const void* q, const void* k, const void* v, float* 
 }
 
 size_t ropeattn_decode_workspace_size(int64_t B, int64_t n, int32_t Hq, int32_t Hkv, int32_t D) {
-  if (check_shapes(B, n, Hq, Hkv, D, true) || B == 0 || n == 0) return 0;
+  if (check_shapes(B, n, Hq, Hkv, D) || B == 0 || n == 0) return 0;
   return decode_layout(B, n, Hq, Hkv, D).total;
 }
 
@@ -801,7 +809,7 @@ int ropeattn_decode_cache(const void* q, const void* k_cache, const void* v_cach
                           int64_t n, int64_t cache_len, int32_t Hq, int32_t Hkv, int32_t D,
                           const ropeattn_params* params, void* workspace, size_t workspace_bytes, void* stream) {
   g_last_error.clear();
-  int rc = check_shapes(B, n, Hq, Hkv, D, true);
+  int rc = check_shapes(B, n, Hq, Hkv, D);
   if (rc) return rc;
   if (cache_len < n || cache_len > kMaxPos)
     return fail(ROPEATTN_ERR_INVALID_ARG, "cache_len (%lld) must be in [n, 2^31)", static_cast<long long>(cache_len));
@@ -909,7 +917,7 @@ int noalloc_scratch_ptr(void** out) {
 }  // namespace
 
 extern "C" size_t ropeattn_decode_unfused_workspace_size(int64_t B, int64_t n, int32_t Hq, int32_t Hkv, int32_t D) {
-  if (check_shapes(B, n, Hq, Hkv, D, true) || B == 0 || n == 0) return 0;
+  if (check_shapes(B, n, Hq, Hkv, D) || B == 0 || n == 0) return 0;
   return align_up(static_cast<size_t>(B) * n * Hkv * D * 2, 256) + decode_layout(B, n, Hq, Hkv, D).total;
 }
 
@@ -917,7 +925,7 @@ int ropeattn_decode_unfused(const void* q, const void* k_cache, const void* v_ca
                             int64_t B, int64_t n, int32_t Hq, int32_t Hkv, int32_t D, const ropeattn_params* params,
                             void* workspace, size_t workspace_bytes, void* stream) {
   g_last_error.clear();
-  int rc = check_shapes(B, n, Hq, Hkv, D, true);
+  int rc = check_shapes(B, n, Hq, Hkv, D);
   if (rc) return rc;
   PosMap m;
   int eff;

@@ -88,9 +88,11 @@ def test_host_argument_checks(ra):
                                   ctypes.byref(cp(_p(kind=STANDARD))), nullp, 0, nullp)
         assert rc == ra.ERR_INVALID_ARG
         assert lib.ropeattn_last_error().decode()
-    # head_dim 256: decode and cache writes only (the prefill's TMEM holds D <= 128)
-    assert lib.ropeattn_prefill(nullp, nullp, nullp, nullp, nullp, 1, 16, 2, 1, 256,
-                                ctypes.byref(cp(_p(kind=STANDARD))), nullp, 0, nullp) == ra.ERR_INVALID_ARG
+    # head_dim 256 passes the shape checks of every entry point (the prefill
+    # runs it with one query tile per CTA)
+    assert lib.ropeattn_prefill_workspace_size(ctypes.byref(cp(_p(kind=STANDARD))), 1, 4096, 2, 1, 256) == \
+        4096 * 256 * 2 + 4096 * 128 * 8
+    assert lib.ropeattn_prefill_workspace_size(ctypes.byref(cp(_p(kind=STANDARD))), 1, 4096, 2, 1, 96) == 0
     assert lib.ropeattn_decode_workspace_size(1, 1000, 2, 1, 256) > 0
     assert lib.ropeattn_decode(nullp, nullp, nullp, nullp, nullp, 1, 1000, 8, 1, 256,
                                ctypes.byref(cp(_p(kind=STANDARD))), nullp, 0, nullp) == ra.ERR_INVALID_ARG  # GQA 8

@@ -47,6 +47,8 @@ PREFILL = [
                                                  pairing=PAIR_HALF)),
     ("bifocal_g3_d64", 1, 700, 2, 2, 64, MapParams(O.BIFOCAL, rope_base=1e4, w0=64, w_pretrained=300,
                                                    pairing=PAIR_HALF)),
+    ("bifocal_d256", 1, 600, 2, 1, 256, MapParams(O.BIFOCAL, rope_base=1e6, w0=100, w_pretrained=200,
+                                                  pairing=PAIR_HALF)),
 ]
 
 

@@ -26,6 +26,7 @@ CASES = [
     ("bifocal_small_chunk", 2, 2049, 2000, 4, 1, 64, MapParams(O.BIFOCAL, rope_base=1e4, w0=64, w_pretrained=512)),
     ("bifocal_one_row", 1, 3001, 3000, 4, 4, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=1000, w_pretrained=1000)),
     ("bifocal_in_window", 1, 400, 200, 4, 2, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=500, w_pretrained=100)),
+    ("bifocal_d256", 1, 900, 500, 2, 1, 256, MapParams(O.BIFOCAL, rope_base=1e6, w0=100, w_pretrained=300)),
 ]
 
 

@@ -40,6 +40,15 @@ SMALL = [
     ("bifocal_w0_300", 2, 1100, 4, 2, 128, MapParams(O.BIFOCAL, rope_base=1e4, w0=300, w_pretrained=300)),
     ("bifocal_g3_d64", 1, 700, 2, 2, 64, MapParams(O.BIFOCAL, rope_base=1e4, w0=64, w_pretrained=300)),
     ("bifocal_w0_127", 1, 640, 2, 1, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=127, w_pretrained=100)),
+    # head_dim 256: one 128-row query tile per CTA, 64-key tiles
+    ("standard_d256_ragged", 1, 300, 2, 1, 256, MapParams(O.STANDARD, rope_base=1e4)),
+    ("endprompt_d256", 1, 400, 2, 1, 256, MapParams(O.ENDPROMPT, rope_base=5e5, interp=8.0, seg1_len=300,
+                                                     term_start=65000)),
+    ("periodic_d256_w100", 1, 500, 2, 2, 256, MapParams(O.PERIODIC, window=100)),
+    ("nope_d256", 1, 333, 2, 1, 256, MapParams(O.NOPE)),
+    ("bifocal_d256_g4", 1, 700, 2, 1, 256, MapParams(O.BIFOCAL, rope_base=1e6, w0=100, w_pretrained=200)),
+    ("bifocal_d256_gqa4_w0_63", 2, 520, 4, 1, 256, MapParams(O.BIFOCAL, rope_base=1e4, w0=63, w_pretrained=150)),
+    ("standard_d256_s1", 1, 1, 2, 1, 256, MapParams(O.STANDARD)),
 ]
 
 
@@ -60,9 +69,10 @@ def test_prefill_small_all_rows(case):
     assert_close(out.cpu().numpy(), lse.cpu().numpy(), ref_o, ref_l, name)
 
 
-def test_bifocal_inside_window_is_bitwise_standard():
+@pytest.mark.parametrize("D", [128, 256])
+def test_bifocal_inside_window_is_bitwise_standard(D):
     # L <= w_pretrained: the bifocal map is the base model exactly (Jet-Long §3)
-    q, k, v = make_qkv(1, 700, 4, 2, 128, seed=5)
+    q, k, v = make_qkv(1, 700, 4, 2, D, seed=5)
     a = _run(q, k, v, MapParams(O.BIFOCAL, rope_base=1e6, w0=64, w_pretrained=700))
     b = _run(q, k, v, MapParams(O.STANDARD, rope_base=1e6))
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])

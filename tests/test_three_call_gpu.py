@@ -15,6 +15,7 @@ pytestmark = pytest.mark.gpu
 CASES = [
     ("g4_d128", 1, 1000, 4, 2, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=100, w_pretrained=300)),
     ("w0_0_d64", 2, 777, 2, 1, 64, MapParams(O.BIFOCAL, rope_base=1e4, w0=0, w_pretrained=256)),
+    ("g3_d256", 1, 600, 2, 1, 256, MapParams(O.BIFOCAL, rope_base=1e6, w0=100, w_pretrained=200)),
     ("g3_wide_window", 1, 3000, 4, 1, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=1000, w_pretrained=1000)),
 ]
 
