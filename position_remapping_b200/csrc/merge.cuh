@@ -4,8 +4,8 @@
 //   M = max(l_A, l_B, l_C),  W_X = exp(l_X - M),
 //   O = (W_A O_A + W_B O_B - W_C O_C) / (W_A + W_B - W_C),
 //   l = M + ln(W_A + W_B - W_C),
-// all in fp32. One warp per (batch, position, head) row, one float4 of O per
-// lane (D = 128; two rows per warp for D = 64 is not needed: D / 4 <= 32).
+// all in fp32. One warp per (batch, position, head) row; each lane merges the
+// float4 groups lane, lane + 32, ... of the row (D / 4 groups: 16, 32 or 64).
 // O_B and l_B live in the output buffers and are overwritten in place.
 #pragma once
 
@@ -39,16 +39,16 @@ __global__ void __launch_bounds__(256) three_call_merge_kernel(const MergeArgs a
   const float den = wa + wb - wc;
   const float inv = 1.0f / den;
   const size_t base = static_cast<size_t>(row) * a.D;
-  if (lane * 4 < a.D) {
-    const float4 xa = *reinterpret_cast<const float4*>(a.oA + base + lane * 4);
-    const float4 xb = *reinterpret_cast<const float4*>(a.out + base + lane * 4);
-    const float4 xc = *reinterpret_cast<const float4*>(a.oC + base + lane * 4);
+  for (int c = lane * 4; c < a.D; c += 128) {
+    const float4 xa = *reinterpret_cast<const float4*>(a.oA + base + c);
+    const float4 xb = *reinterpret_cast<const float4*>(a.out + base + c);
+    const float4 xc = *reinterpret_cast<const float4*>(a.oC + base + c);
     float4 o;
     o.x = (wa * xa.x + wb * xb.x - wc * xc.x) * inv;
     o.y = (wa * xa.y + wb * xb.y - wc * xc.y) * inv;
     o.z = (wa * xa.z + wb * xb.z - wc * xc.z) * inv;
     o.w = (wa * xa.w + wb * xb.w - wc * xc.w) * inv;
-    *reinterpret_cast<float4*>(a.out + base + lane * 4) = o;
+    *reinterpret_cast<float4*>(a.out + base + c) = o;
   }
   __syncwarp();
   if (lane == 0) a.lse[li] = M + logf(den);
