@@ -350,16 +350,18 @@ def run_profile_case(which: str):
     """Capture-sized cases for ncu (a few GB on the device at most, inputs
     still larger than L2). prefill: the 131072-token workload's kernel on a
     32768-token sequence with w_pretrained 8192, so G = 4 as in the full run;
-    decode: the full 131072-key decode (512 MiB of cache)."""
+    prefill256: the same case at head_dim 256; decode: the full 131072-key
+    decode (512 MiB of cache)."""
     from position_remapping_b200 import ropeattn as ra
     dev = torch.device("cuda", 0)
-    if which == "prefill":
+    if which in ("prefill", "prefill256"):
         P = PREFILL
         S = 32768
+        D = 256 if which == "prefill256" else P.D
         params = P.params.replace(w_pretrained=8192)
-        q, k, v = make_qkv(P.B, S, P.Hq, P.Hkv, P.D, P.seed, device=dev)
-        ws = torch.empty(ra.prefill_workspace_size(params, P.B, S, P.Hq, P.Hkv, P.D), dtype=torch.uint8, device=dev)
-        out = torch.empty((P.B, S, P.Hq, P.D), dtype=torch.float32, device=dev)
+        q, k, v = make_qkv(P.B, S, P.Hq, P.Hkv, D, P.seed, device=dev)
+        ws = torch.empty(ra.prefill_workspace_size(params, P.B, S, P.Hq, P.Hkv, D), dtype=torch.uint8, device=dev)
+        out = torch.empty((P.B, S, P.Hq, D), dtype=torch.float32, device=dev)
         lse = torch.empty((P.B, P.Hq, S), dtype=torch.float32, device=dev)
         for _ in range(3):
             ra.prefill(q, k, v, params, out=out, lse=lse, workspace=ws)
@@ -379,7 +381,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--profile", choices=["prefill", "prefill256", "decode"], default=None,
                     help="run a capture-sized case of one kernel three times (for ncu); no timing, no JSON")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
