@@ -24,7 +24,7 @@ using namespace ropeattn;
 
 namespace {
 
-constexpr int kVersion = 10000;  // 1.0.0
+constexpr int kVersion = 10100;  // 1.1.0: half-split pairing, head_dim 256 prefill
 thread_local std::string g_last_error;
 
 int fail(int code, const char* fmt, ...) {
@@ -91,9 +91,9 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 4-D bf16 tensor [d3][d2][d1][d0] (d0 contiguous) with box (b0, 1, b2, 1).
-// 4-D bf16 map (d0 innermost); d2_stride: rows of d2 between consecutive d3
-// indices (d2 when 0: a dense tensor; larger for a cache with spare rows).
+// TMA map of a 4-D bf16 tensor [d3][d2][d1][d0] (d0 contiguous) with box
+// (b0, 1, b2, 1); d2_stride: rows of d2 between consecutive d3 indices (d2
+// when 0: a dense tensor; larger for a cache with spare rows).
 int make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3,
              uint32_t b0, uint32_t b2, bool swizzle128, uint64_t d2_stride = 0) {
   auto fn = encode_fn();
