@@ -134,6 +134,52 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+# The C ABI sees only pointers and sizes: the dtype, layout and device of
+# every tensor are checked here, before the call.
+def _need(t, name: str, dtype, shape=None) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype} (got {t.dtype})")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)} (got {tuple(t.shape)})")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be on a CUDA device (got {t.device})")
+    return t
+
+
+def _need_ndim(t, name: str, dtype, ndim: int) -> torch.Tensor:
+    if isinstance(t, torch.Tensor) and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions (got shape {tuple(t.shape)})")
+    return _need(t, name, dtype)
+
+
+def _need_workspace(ws: Optional[torch.Tensor]) -> Optional[torch.Tensor]:
+    if ws is None:
+        return None
+    if not isinstance(ws, torch.Tensor) or not ws.is_contiguous() or ws.device.type != "cuda":
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return ws
+
+
+def _check_prefill_args(q, k, v):
+    _need_ndim(q, "q", torch.bfloat16, 4)
+    _need_ndim(k, "k", torch.bfloat16, 4)
+    B, S, _, D = q.shape
+    if k.shape[0] != B or k.shape[1] != S or k.shape[3] != D:
+        raise ValueError(f"k {tuple(k.shape)} does not match q {tuple(q.shape)} (B, S, D)")
+    _need(v, "v", torch.bfloat16, k.shape)
+
+
+def _check_cache_args(q, k_cache, v_cache):
+    _need_ndim(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, k_cache.shape)
+    if q.shape[0] != k_cache.shape[0] or q.shape[-1] != k_cache.shape[3]:
+        raise ValueError(f"q {tuple(q.shape)} does not match the cache {tuple(k_cache.shape)} (B, D)")
+
+
 def version() -> int:
     return lib.ropeattn_version()
 
@@ -164,7 +210,16 @@ def cache_write(k: torch.Tensor, v: Optional[torch.Tensor], k_cache: torch.Tenso
                 params: MapParams, start: int, stream=None) -> None:
     """Stores k [B,count,Hkv,D] rotated at positions start..start+count-1 (and
     v as is) into rows start.. of k_cache / v_cache [B,cache_len,Hkv,D]."""
+    _need_ndim(k, "k", torch.bfloat16, 4)
     B, count, Hkv, D = k.shape
+    _need_ndim(k_cache, "k_cache", torch.bfloat16, 4)
+    if k_cache.shape[0] != B or k_cache.shape[2] != Hkv or k_cache.shape[3] != D:
+        raise ValueError(f"k_cache {tuple(k_cache.shape)} does not match k {tuple(k.shape)} (B, Hkv, D)")
+    if (v is None) != (v_cache is None):
+        raise ValueError("v and v_cache must be both given or both None")
+    if v is not None:
+        _need(v, "v", torch.bfloat16, k.shape)
+        _need(v_cache, "v_cache", torch.bfloat16, k_cache.shape)
     cache_len = k_cache.shape[1]
     cp = to_cparams(params)
     _check(lib.ropeattn_cache_write(_ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), B, int(start), count, cache_len,
@@ -196,12 +251,16 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, params: MapParams
             workspace: Optional[torch.Tensor] = None, stream=None):
     """q [B,S,Hq,D], k/v [B,S,Hkv,D] bf16 contiguous on one CUDA device.
     Returns (out [B,S,Hq,D] fp32, lse [B,Hq,S] fp32)."""
+    _check_prefill_args(q, k, v)
     B, S, Hq, D = q.shape
     Hkv = k.shape[2]
     if out is None:
         out = torch.empty((B, S, Hq, D), dtype=torch.float32, device=q.device)
     if lse is None:
         lse = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32, (B, S, Hq, D))
+    _need(lse, "lse", torch.float32, (B, Hq, S))
+    _need_workspace(workspace)
     need = prefill_workspace_size(params, B, S, Hq, Hkv, D)
     if workspace is None:
         workspace = _workspace(need, q.device)
@@ -217,12 +276,16 @@ def prefill_three_call(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, params
                        workspace: Optional[torch.Tensor] = None, stream=None):
     """Comparator: the literal three-call bifocal prefill with a separate
     merge kernel (same layouts as prefill)."""
+    _check_prefill_args(q, k, v)
     B, S, Hq, D = q.shape
     Hkv = k.shape[2]
     if out is None:
         out = torch.empty((B, S, Hq, D), dtype=torch.float32, device=q.device)
     if lse is None:
         lse = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32, (B, S, Hq, D))
+    _need(lse, "lse", torch.float32, (B, Hq, S))
+    _need_workspace(workspace)
     cp = to_cparams(params)
     if workspace is None:
         workspace = _workspace(int(lib.ropeattn_prefill_three_call_workspace_size(ctypes.byref(cp), B, S, Hq, Hkv, D)),
@@ -235,6 +298,8 @@ def prefill_three_call(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, params
 
 def prefill_prepare(k: torch.Tensor, Hq: int, params: MapParams, workspace: torch.Tensor, stream=None) -> None:
     """First half of prefill: rotated keys and query angle tables into ``workspace``."""
+    _need_ndim(k, "k", torch.bfloat16, 4)
+    _need_workspace(workspace)
     B, S, Hkv, D = k.shape
     cp = to_cparams(params)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
@@ -245,8 +310,12 @@ def prefill_prepare(k: torch.Tensor, Hq: int, params: MapParams, workspace: torc
 def prefill_attend(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, params: MapParams,
                    out: torch.Tensor, lse: torch.Tensor, workspace: Optional[torch.Tensor], stream=None) -> None:
     """Second half of prefill: attention on a workspace filled by prefill_prepare."""
+    _check_prefill_args(q, k, v)
     B, S, Hq, D = q.shape
     Hkv = k.shape[2]
+    _need(out, "out", torch.float32, (B, S, Hq, D))
+    _need(lse, "lse", torch.float32, (B, Hq, S))
+    _need_workspace(workspace)
     cp = to_cparams(params)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.ropeattn_prefill_attend(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, S, Hq, Hkv, D,
@@ -260,14 +329,20 @@ def prefill_chunk(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
     bf16 (cache_len >= start+count; the first start+count rows are used)
     holding every key rotated at its own position. Returns
     (out [B,count,Hq,D] fp32, lse [B,Hq,count] fp32)."""
+    _need_ndim(q, "q", torch.bfloat16, 4)
+    _check_cache_args(q, k_cache, v_cache)
     B, count, Hq, D = q.shape
     Hkv = k_cache.shape[2]
     cache_len = k_cache.shape[1]
-    assert cache_len >= start + count, "the cache must hold at least start + count rows"
+    if cache_len < start + count:
+        raise ValueError(f"the cache holds {cache_len} rows; start + count = {start + count}")
     if out is None:
         out = torch.empty((B, count, Hq, D), dtype=torch.float32, device=q.device)
     if lse is None:
         lse = torch.empty((B, Hq, count), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32, (B, count, Hq, D))
+    _need(lse, "lse", torch.float32, (B, Hq, count))
+    _need_workspace(workspace)
     cp = to_cparams(params)
     if workspace is None:
         workspace = _workspace(prefill_chunk_workspace_size(params, B, int(start), count, Hq, Hkv, D), q.device)
@@ -283,12 +358,17 @@ def decode_cache(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, 
                  workspace: Optional[torch.Tensor] = None, stream=None):
     """Decode over the first n rows of caches [B, cache_len, Hkv, D] with
     spare rows (q [B,Hq,D], the token at position n-1)."""
+    _need_ndim(q, "q", torch.bfloat16, 3)
+    _check_cache_args(q, k_cache, v_cache)
     B, Hq, D = q.shape
     cache_len, Hkv = k_cache.shape[1], k_cache.shape[2]
     if out is None:
         out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
     if lse is None:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32, (B, Hq, D))
+    _need(lse, "lse", torch.float32, (B, Hq))
+    _need_workspace(workspace)
     if workspace is None:
         workspace = _workspace(decode_workspace_size(B, n, Hq, Hkv, D), q.device)
     cp = to_cparams(params)
@@ -303,12 +383,17 @@ def decode_unfused(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
                    workspace: Optional[torch.Tensor] = None, stream=None):
     """Comparator: decode with the correction rotation as a separate pass
     (same layouts as decode)."""
+    _need_ndim(q, "q", torch.bfloat16, 3)
+    _check_cache_args(q, k_cache, v_cache)
     B, Hq, D = q.shape
     n, Hkv = k_cache.shape[1], k_cache.shape[2]
     if out is None:
         out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
     if lse is None:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32, (B, Hq, D))
+    _need(lse, "lse", torch.float32, (B, Hq))
+    _need_workspace(workspace)
     if workspace is None:
         workspace = _workspace(int(lib.ropeattn_decode_unfused_workspace_size(B, n, Hq, Hkv, D)), q.device)
     cp = to_cparams(params)
@@ -323,12 +408,17 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, params
            workspace: Optional[torch.Tensor] = None, stream=None):
     """q [B,Hq,D] (unrotated, position n-1), caches [B,n,Hkv,D] bf16.
     Returns (out [B,Hq,D] fp32, lse [B,Hq] fp32)."""
+    _need_ndim(q, "q", torch.bfloat16, 3)
+    _check_cache_args(q, k_cache, v_cache)
     B, Hq, D = q.shape
     n, Hkv = k_cache.shape[1], k_cache.shape[2]
     if out is None:
         out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
     if lse is None:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32, (B, Hq, D))
+    _need(lse, "lse", torch.float32, (B, Hq))
+    _need_workspace(workspace)
     if workspace is None:
         workspace = _workspace(decode_workspace_size(B, n, Hq, Hkv, D), q.device)
     cp = to_cparams(params)

@@ -167,3 +167,28 @@ def test_workspace_sizes(ra):
     assert ra.prefill_workspace_size(nope.params.replace(pairing=1), nope.B, nope.S, nope.Hq, nope.Hkv, nope.D) == 0
     assert (ra.prefill_chunk_workspace_size(half, 1, 4096, 1000, 32, 8, 128) ==
             ra.prefill_chunk_workspace_size(w.params, 1, 4096, 1000, 32, 8, 128) + 1000 * 32 * 128 * 2)
+
+
+def test_binding_checks_tensors_before_the_call(ra):
+    # the C ABI sees only pointers: dtype, shape, layout and device are
+    # checked by the binding, before any library call (CPU tensors here)
+    import torch
+    from position_remapping_b200.inputs import BIFOCAL
+    p = _p(kind=BIFOCAL, w0=4, w_pretrained=8)
+    q = torch.zeros((1, 16, 2, 64), dtype=torch.bfloat16)
+    k = torch.zeros((1, 16, 1, 64), dtype=torch.bfloat16)
+    cases = [
+        lambda: ra.prefill(q.float(), k, k, p),                        # wrong dtype
+        lambda: ra.prefill(q[0], k, k, p),                             # wrong rank
+        lambda: ra.prefill(q, k, k[:, :8], p),                         # v does not match k
+        lambda: ra.prefill(q, k[:, :8], k[:, :8], p),                  # k rows do not match q
+        lambda: ra.prefill(q.transpose(1, 2), k, k, p),                # not contiguous
+        lambda: ra.prefill(q, k, k, p),                                # not on a CUDA device
+        lambda: ra.decode(q[:, 0], k, k.float(), p),                   # v_cache dtype
+        lambda: ra.decode(q[:, 0, :, :32].contiguous(), k, k, p),      # head_dim mismatch
+        lambda: ra.cache_write(k, k, k, None, p, 0),                   # v without v_cache
+        lambda: ra.prefill_chunk(q, k, k, p, 4),                       # cache shorter than start + count
+    ]
+    for i, fn in enumerate(cases):
+        with pytest.raises((ValueError, TypeError)):
+            fn()
