@@ -10,11 +10,11 @@ What it computes, and where each step is defined:
   block-diagonal 2x2 rotation R_t acting on coordinate pairs (2i, 2i+1):
   "Periodic RoPE for Infinite Context LLMs", §3.1 Eq. 1-2. The half-split
   variant (``pairing`` = 1) turns the pairs (i, i + d/2) by the same angles.
-* Position interpolation divides every position by the factor s ("linearly
-  compresses positions into the pretrained range"): "Jet-Long: Efficient
-  Long-Context Extension with Dynamic Bifocal RoPE", §2.2; used by
-  "EndPrompt: Efficient Long-Context Extension via Terminal Anchoring",
-  abstract and summary ("combined with RoPE interpolation").
+* Position interpolation divides every position by the factor s, a linear
+  squeeze of the positions into the range seen in pre-training: "Jet-Long:
+  Efficient Long-Context Extension with Dynamic Bifocal RoPE", §2.2; EndPrompt
+  pairs its positions with it: "EndPrompt: Efficient Long-Context Extension
+  via Terminal Anchoring", abstract and summary.
 * Periodic position phi(t) = t mod W inside causal sliding-window attention
   over the W keys {t-W+1 .. t}: Periodic RoPE, §3.2 Eq. 4-5.
 * NoPE causal attention A_ts = q.k / sqrt(d_h), s <= t: Periodic RoPE, §3.3

@@ -115,7 +115,7 @@ constexpr long long kMaxPos = 0x7fffffffLL;
 // Validates the parameter struct for a sequence of length L; fills the
 // position map. The kind may be simplified: a bifocal map with G = 1 or with
 // every key inside the local window is exactly the standard map (Jet-Long §3:
-// "reduces to the unmodified base model").
+// the method then gives the base model's attention unchanged).
 int check_params(const ropeattn_params* p, long long L, int D, PosMap* m, int* eff_kind) {
   if (!p) return fail(ROPEATTN_ERR_INVALID_ARG, "params is NULL");
   if (p->reserved[0] != 0 || p->reserved[1] != 0)
