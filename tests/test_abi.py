@@ -93,6 +93,10 @@ def test_host_argument_checks(ra):
     assert lib.ropeattn_prefill_workspace_size(ctypes.byref(cp(_p(kind=STANDARD))), 1, 4096, 2, 1, 256) == \
         4096 * 256 * 2 + 4096 * 128 * 8
     assert lib.ropeattn_prefill_workspace_size(ctypes.byref(cp(_p(kind=STANDARD))), 1, 4096, 2, 1, 96) == 0
+    bif = ctypes.byref(cp(_p(kind=BIFOCAL, w0=64, w_pretrained=1024)))
+    assert lib.ropeattn_prefill_chunk_workspace_size(bif, 1, 3000, 1096, 2, 1, 256) > 0
+    assert lib.ropeattn_prefill_three_call_workspace_size(bif, 1, 4096, 2, 1, 256) > \
+        lib.ropeattn_prefill_workspace_size(bif, 1, 4096, 2, 1, 256) > 0
     assert lib.ropeattn_decode_workspace_size(1, 1000, 2, 1, 256) > 0
     assert lib.ropeattn_decode(nullp, nullp, nullp, nullp, nullp, 1, 1000, 8, 1, 256,
                                ctypes.byref(cp(_p(kind=STANDARD))), nullp, 0, nullp) == ra.ERR_INVALID_ARG  # GQA 8
