@@ -317,10 +317,10 @@ def test_endprompt_degenerate_is_standard_and_shift_invariant():
     assert np.allclose(b[0], std[0], atol=1e-10) and np.allclose(b[1], std[1], atol=1e-10)
 
 
-@pytest.mark.parametrize("w0,wp", [(0, 5), (3, 5), (6, 4), (11, 8)])
-def test_three_call_merge_equals_routed(w0, wp):
+@pytest.mark.parametrize("w0,wp,pairing", [(0, 5, 0), (3, 5, 0), (6, 4, 0), (11, 8, 0), (3, 5, 1)])
+def test_three_call_merge_equals_routed(w0, wp, pairing):
     q, k, v = make_qkv(1, 33, 4, 2, 16, seed=16)
-    p = MapParams(O.BIFOCAL, rope_base=1e4, w0=w0, w_pretrained=wp)
+    p = MapParams(O.BIFOCAL, rope_base=1e4, w0=w0, w_pretrained=wp, pairing=pairing)
     a = O.prefill(q, k, v, p)
     b = O.prefill_three_call(q, k, v, p)
     assert np.allclose(a[0], b[0], atol=1e-10) and np.allclose(a[1], b[1], atol=1e-10)
