@@ -448,7 +448,7 @@ def prefill_from_cache(q, k_cache, v_cache, params, start: int, stage_bf16: bool
     return out, lse
 
 
-def decode(q, k_cache, v_cache, params):
+def decode(q, k_cache, v_cache, params, stage_bf16: bool = False):
     """One query token at position n-1 against a cache of n keys.
 
     q [B,Hq,D] unrotated; k_cache [B,n,Hkv,D] holds keys already rotated at
@@ -456,8 +456,11 @@ def decode(q, k_cache, v_cache, params):
     L = n. The query is rotated to its position; for BIFOCAL, keys with
     (n-1) - k > w0 are read through the correction rotation
     k_remote = RoPE(k_cache[k], Delta k), Delta k = f(k) - k, and the query
-    through q_remote = RoPE(q_local, Delta q) (Eq. 5-6). Rotations are kept in
-    float64 (no bf16 staging): the decode kernel keeps them in registers.
+    through q_remote = RoPE(q_local, Delta q) (Eq. 5-6). Rotations are in
+    float64. ``stage_bf16`` rounds the rotated query views and the corrected
+    remote keys to bf16 (round to nearest even) before the dot products: the
+    operand rounding of a decode on bf16 tensor cores, the same modelled input
+    rounding as the prefill's; the cache itself is taken as given.
     Returns out [B,Hq,D], lse [B,Hq]."""
     q, kc, vc = to_f64(q), to_f64(k_cache), to_f64(v_cache)
     B, Hq, D = q.shape
@@ -468,6 +471,7 @@ def decode(q, k_cache, v_cache, params):
     freqs = _freqs(params, D)
     pr = _pairing(params)
     p_loc, _, G = position_maps(params, n)
+    stage = round_bf16 if stage_bf16 else (lambda a: a)
     t = n - 1
     keys = np.arange(n)
     ok = _allowed(params, t, keys)[None, :]
@@ -478,12 +482,12 @@ def decode(q, k_cache, v_cache, params):
             hk = h // grp
             qq = q[b, h][None, :]
             ql = qq if kind == NOPE else rotate(qq, np.array([p_loc[t]]), freqs, pr)
-            sc = (ql @ kc[b, :, hk].T) * scale                     # [1, n]
+            sc = (stage(ql) @ kc[b, :, hk].T) * scale              # [1, n]
             if kind == BIFOCAL:
                 dq = int(remote_position(t, G)) - t                # Eq. 5
-                qr = rotate(ql, np.array([dq]), freqs, pr)             # Eq. 6, query
+                qr = stage(rotate(ql, np.array([dq]), freqs, pr))      # Eq. 6, query
                 dk = remote_position(keys, G) - keys               # Eq. 5
-                kr = rotate(kc[b, :, hk], dk, freqs, pr)               # Eq. 6, keys
+                kr = stage(rotate(kc[b, :, hk], dk, freqs, pr))        # Eq. 6, keys
                 sr = (qr @ kr.T) * scale
                 local = (t - keys) <= int(params.w0)
                 sc = np.where(local[None, :], sc, sr)

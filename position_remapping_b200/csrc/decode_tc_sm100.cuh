@@ -1,0 +1,570 @@
+// One decode step over an untouched RoPE key cache (Jet-Long §3.2) on the
+// fifth-generation tensor cores, sm_100a, for head_dim 64 and 128.
+//
+// Split-KV: CTA (split, kv head, batch) owns a contiguous key range of one kv
+// head; the grid is one wave. The range streams through shared memory by TMA
+// in 128-key tiles (128-byte swizzle, no multicast), K tiles and V tiles in
+// rings of their own. Per tile, with the GQA group's query heads as the MMA's N
+// dimension (the tensor cores see the keys as M = 128 rows):
+//   S^T = K' Q^T   tcgen05.mma, A = the K tile (K-major), B = the staged
+//                  query rows (K-major), fp32 into TMEM (lane = key);
+//   softmax        lane = key: the score of each head, the tile maximum per
+//                  head (warp shuffles, then an mbarrier exchange between the
+//                  four softmax warps), exp2 with a lazily moved reference
+//                  maximum, P^T (bf16) into shared memory;
+//   O^T += V^T P^T tcgen05.mma, A = the V tile read MN-major (the head_dim
+//                  axis as M), B = P^T, fp32 accumulator in TMEM (lane = one
+//                  output dimension).
+// The staged query rows are R(p(t)) q for the kind's own position of the query
+// token t = n - 1 (rows 0..GP-1) and, for the bifocal map, R(f(t)) q (rows
+// GP..2 GP-1), both rotated from the raw query with exact angles in fp32 and
+// rounded to bf16. Local keys use the first set as stored in the cache. Remote
+// keys k ((n-1) - k > w0) are read through the correction of Eq. 6: the
+// rotation warps turn each remote key of the staged K tile in place by
+// R(f(k) - k) = R(-u(k)), u(k) = k - floor(k/G), before the MMA reads it. A
+// thread of those warps owns one 16-byte chunk (four rotation pairs) of
+// every STEP-th row: the (cos, sin) of -u(k) theta_i is advanced row to row,
+// and on from one tile to the next, by one of two fixed rotations (u grows by
+// STEP - STEP/G, or one less when a group boundary is crossed), and seeded
+// exactly every few tiles.
+// Every angle is an integer position times theta_i taken from theta_i's
+// fraction of a turn in 64-bit fixed point, so it is exact modulo a turn
+// before the fp32 sincospi.
+//
+// Warps: 0-3 softmax (TMEM lanes 0-127), 4-11 key rotation, 12 and 13 TMA
+// producers of the K ring and the V ring, 14 QK issuer (one thread; TMEM
+// allocation), 15 PV issuer (one thread); all of them stage the query. After the key
+// range each CTA writes (O, m, l) of its split, and the last CTA of a (batch,
+// kv head) to arrive merges all splits in split order.
+#pragma once
+
+#include "common.cuh"
+#include "decode_sm100.cuh"
+#include "posmap.cuh"
+
+namespace ropeattn {
+
+constexpr int kTcKeys = 128;      // keys per stage (the MMA's M)
+constexpr int kTcRotThreads = 256;   // key-rotation warps 4-11
+constexpr int kTcThreads = 128 + kTcRotThreads + 128;   // 16 warps
+constexpr int kTcWarpTmaK = 12;   // K tile producer
+constexpr int kTcWarpTmaV = 13;   // V tile producer
+constexpr int kTcWarpQK = 14;     // QK^T issuer (and TMEM allocation)
+constexpr int kTcWarpPV = 15;     // PV issuer
+constexpr int kTcReseed = 8;      // tiles between exact re-seeds of the rotation phasor
+constexpr int kTcNP = 16;         // N of the PV MMA: query heads of the group, padded
+
+template <int D, int GP, int ROT>
+struct DecodeTcShape {
+  static constexpr int kRows = ROT ? 2 * GP : GP;          // staged query rows
+  static constexpr int NB = kRows <= 16 ? 16 : 32;           // N of the QK MMA
+  static constexpr int kStages = D == 128 ? 3 : 6;           // slots of each ring (K and V)
+  static constexpr int kBlk = kTcKeys * 128;                 // one 64-column swizzle block of a tile
+  static constexpr int kTileBytes = kTcKeys * D * 2;         // K or V tile
+  static constexpr int kV = 0;                               // V ring, then the K ring
+  static constexpr int kK = kStages * kTileBytes;
+  static constexpr int kQ = 2 * kStages * kTileBytes;        // [D/64][NB rows][128 B]
+  static constexpr int kQBytes = (D / 64) * NB * 128;
+  static constexpr int kP = kQ + kQBytes;                    // [2 bufs][2 key blocks][kTcNP rows][128 B]
+  static constexpr int kPBuf = 2 * kTcNP * 128;
+  static constexpr int kRed = kP + 2 * kPBuf;                // [2][4 warps][GP] tile maxima, then [4][GP] sums
+  static constexpr int kBar = kRed + 2 * 4 * GP * 4 + 64;
+  // kfull, rot, kempty, vfull, vempty [NS each]; s_full, s_free, p_full, pv_done, mx [2 each]
+  static constexpr int kNumBars = 5 * kStages + 10;
+  static constexpr int kMisc = kBar + kNumBars * 8;          // tmem base, abort flag, last flag
+  static constexpr int kTotal = kMisc + 16;
+  static constexpr int kAlloc = kTotal + 1024;               // slack to align the base to 1024
+  static constexpr uint32_t kTmemCols = (2 * NB + kTcNP) <= 64 ? 64 : 128;
+  static_assert(GP <= 16, "query heads per kv head: at most 16");
+  static_assert(kQ % 1024 == 0 && kP % 1024 == 0 && kPBuf % 1024 == 0 && (NB * 128) % 1024 == 0,
+                "swizzled operand tiles start on 1024-byte boundaries");
+  static_assert(kAlloc <= 227 * 1024, "shared memory");
+};
+
+// byte offset of element (row, col) of a K-major operand tile stored as
+// 64-column blocks of rows x 128 bytes with the 128-byte swizzle
+__device__ __forceinline__ int sw128_off(int row, int col, int block_bytes) {
+  const int c = (col & 63) >> 3;
+  return (col >> 6) * block_bytes + row * 128 + ((c ^ (row & 7)) << 4) + (col & 7) * 2;
+}
+
+template <int D, int GP, int ROT>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                     const DecodeParams p) {
+  using L = DecodeTcShape<D, GP, ROT>;
+  constexpr int NS = L::kStages;
+  constexpr int NB = L::NB;
+  constexpr int kCB = D / 64;
+  constexpr uint32_t kIdescQK = idesc_bf16_f32(kTcKeys, NB, false, false);
+  constexpr uint32_t kIdescPV = idesc_bf16_f32(128, kTcNP, false, true);   // A = V^T read MN-major
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + L::kQ;
+  uint8_t* sP = smem + L::kP;
+  float* red = reinterpret_cast<float*>(smem + L::kRed);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t* kfull = bars;            // [NS] K tile landed
+  uint64_t* rot = kfull + NS;        // [NS] remote keys of the K tile rotated
+  uint64_t* kempty = rot + NS;       // [NS] K tile read by its QK
+  uint64_t* vfull = kempty + NS;     // [NS] V tile landed
+  uint64_t* vempty = vfull + NS;     // [NS] V tile read by its PV
+  uint64_t* s_full = vempty + NS;    // [2]
+  uint64_t* s_free = s_full + 2;     // [2]
+  uint64_t* p_full = s_free + 2;     // [2]
+  uint64_t* pv_done = p_full + 2;    // [2]
+  uint64_t* mx = pv_done + 2;        // [2] tile maxima exchanged
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int split = blockIdx.x;
+  const int hkv = blockIdx.y;
+  const int b = blockIdx.z;
+
+  const int kb = min(p.n, p.k_begin + split * p.keys_per_split);
+  const int ke = min(p.n, kb + p.keys_per_split);
+  const int ntile = (ke - kb + kTcKeys - 1) / kTcKeys;
+  const int t_q = p.n - 1;   // query position index
+  const int grp = p.Hq / p.Hkv;   // query heads of the group (<= GP; the rest are zero rows)
+  // remote keys [kb, kr_end) come first: the tiles that hold any are a prefix
+  const int kr_end = ROT ? min(p.k_local, ke) : kb;
+  const int nrot = kr_end > kb ? (kr_end - kb + kTcKeys - 1) / kTcKeys : 0;
+
+  if (tid == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(kfull + i, 1);
+      mbar_init(rot + i, kTcRotThreads);
+      mbar_init(kempty + i, 1);
+      mbar_init(vfull + i, 1);
+      mbar_init(vempty + i, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(s_full + a, 1);
+      mbar_init(s_free + a, 128);
+      mbar_init(p_full + a, 128);
+      mbar_init(pv_done + a, 1);
+      mbar_init(mx + a, 4);
+    }
+    *abort_flag = 0;
+    *last_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == kTcWarpQK) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  // zero the staged query rows and both P^T buffers (rows beyond the group
+  // stay zero), then stage the rotated query rows
+  for (int i = tid; i < (L::kQBytes + 2 * L::kPBuf) / 16; i += kTcThreads)
+    reinterpret_cast<uint4*>(sQ)[i] = make_uint4(0u, 0u, 0u, 0u);
+  __syncthreads();
+  for (int i = tid; i < grp * (D / 2); i += kTcThreads) {
+    const int gi = i / (D / 2), pr = i % (D / 2);
+    const int hq = hkv * grp + gi;
+    const uint32_t xw = __ldg(reinterpret_cast<const uint32_t*>(p.q + (static_cast<size_t>(b) * p.Hq + hq) * D) + pr);
+    const float x0 = bf16lo(xw), x1 = bf16hi(xw);
+    uint32_t yl = xw;
+    if (p.m.kind != kNope) {
+      const float2 cs = turn_cs(pos_primary(p.m, t_q), p.turns[pr]);
+      float y0, y1;
+      rot_pair(x0, x1, cs.x, cs.y, y0, y1);
+      yl = pack_bf16x2(y0, y1);
+    }
+    *reinterpret_cast<uint32_t*>(sQ + sw128_off(gi, 2 * pr, NB * 128)) = yl;
+    if constexpr (ROT != 0) {
+      const float2 cs = turn_cs(pos_remote(p.m, t_q), p.turns[pr]);
+      float y0, y1;
+      rot_pair(x0, x1, cs.x, cs.y, y0, y1);
+      *reinterpret_cast<uint32_t*>(sQ + sw128_off(GP + gi, 2 * pr, NB * 128)) = pack_bf16x2(y0, y1);
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem;              // S^T buffers at [0, NB) and [NB, 2 NB)
+  const uint32_t tO = tmem + 2 * NB;     // O^T, kTcNP columns
+
+  float l_fin[GP];                      // softmax threads: per-thread sums, reduced at the end
+  float m_fin[GP];
+#pragma unroll
+  for (int gi = 0; gi < GP; ++gi) {
+    l_fin[gi] = 0.f;
+    m_fin[gi] = -INFINITY;
+  }
+  uint32_t o_fin[kTcNP];
+
+  if (warp == kTcWarpTmaK || warp == kTcWarpTmaV) {
+    // -------------------------------------------------------- TMA producers
+    // K and V tiles stream through rings of their own: a K slot is free once
+    // its QK has read it, a V slot once its PV has, so K tiles run ahead of
+    // the rotation and the values of a tile are fetched while it is scored
+    if (lane == 0) {
+      const bool is_k = warp == kTcWarpTmaK;
+      const CUtensorMap* map = is_k ? &tmK : &tmV;
+      uint64_t* fullb = is_k ? kfull : vfull;
+      uint64_t* emptyb = is_k ? kempty : vempty;
+      uint8_t* ring = smem + (is_k ? L::kK : L::kV);
+      tma_prefetch_desc(map);
+      for (int t = 0; t < ntile; ++t) {
+        const int s = t % NS;
+        if (t >= NS && !mbar_wait(emptyb + s, ((t / NS) - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(fullb + s, L::kTileBytes);
+        uint8_t* dst = ring + s * L::kTileBytes;
+        const int row = kb + t * kTcKeys;
+        for (int cb = 0; cb < kCB; ++cb) tma_load_4d(dst + cb * L::kBlk, map, fullb + s, cb * 64, hkv, row, b);
+      }
+    }
+  } else if (warp == kTcWarpQK) {
+    // -------------------------------------------------------- MMA: S^T = K Q^T
+    if (lane == 0) {
+      const uint32_t qaddr = smem_u32(sQ);
+      for (int t = 0; t < ntile; ++t) {
+        const int s = t % NS;
+        if (!mbar_wait(t < nrot ? rot + s : kfull + s, (t / NS) & 1, abort_flag)) break;
+        if (t >= 2 && !mbar_wait(s_free + (t & 1), ((t >> 1) - 1) & 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t kaddr = smem_u32(smem + L::kK + s * L::kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t kin = (kk & 3) * 32;   // K step inside a 64-column swizzle block
+          umma_ss(tS + (t & 1) * NB, sdesc_sw128(kaddr + (kk >> 2) * L::kBlk + kin, 16, 1024),
+                  sdesc_sw128(qaddr + (kk >> 2) * (NB * 128) + kin, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(s_full + (t & 1));
+        umma_commit(kempty + s);
+      }
+    }
+  } else if (warp == kTcWarpPV) {
+    // ------------------------------------------------------ MMA: O^T += V^T P^T
+    if (lane == 0) {
+      for (int t = 0; t < ntile; ++t) {
+        const int s = t % NS;
+        if (!mbar_wait(vfull + s, (t / NS) & 1, abort_flag)) break;
+        if (!mbar_wait(p_full + (t & 1), (t >> 1) & 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t vaddr = smem_u32(smem + L::kV + s * L::kTileBytes);
+        const uint32_t paddr = smem_u32(sP + (t & 1) * L::kPBuf);
+        // M = 128 output dimensions: for D = 64 the upper 64 rows read the 16 KiB
+        // that follow the V tile (the next slot, or the K ring) and land in
+        // TMEM lanes nobody reads
+#pragma unroll
+        for (int kk = 0; kk < kTcKeys / 16; ++kk) {
+          umma_ss(tO, sdesc_sw128(vaddr + kk * 2048, L::kBlk, 1024),
+                  sdesc_sw128(paddr + (kk >> 2) * (kTcNP * 128) + (kk & 3) * 32, 16, 1024), kIdescPV,
+                  (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(pv_done + (t & 1));
+        umma_commit(vempty + s);
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------- rotation of remote keys
+    if constexpr (ROT != 0) {
+      constexpr int CPR = D / 8;              // 16-byte chunks per row
+      constexpr int STEP = kTcRotThreads / CPR;   // rows between a thread's rows (16 or 32)
+      constexpr int NR = kTcKeys / STEP;      // rows per thread per tile (8 or 4)
+      const int id = tid - 128;
+      const int c = id % CPR, rg = id / CPR;
+      const int G = p.m.G;
+      const int stepq = STEP / G, stepr = STEP % G;
+      // the two row-to-row advances of u: STEP - stepq, and one less after a
+      // group boundary; (cos, sin, -sin) of -du theta for the thread's pairs
+      float2 MC[2][2], MS[2][2], MNS[2][2];   // [advance][pair pack] (pairs 4c+2j, 4c+2j+1)
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int du = STEP - stepq - e;
+          const float2 x = turn_cs(-du, p.turns[4 * c + 2 * j]);
+          const float2 y = turn_cs(-du, p.turns[4 * c + 2 * j + 1]);
+          MC[e][j] = f2(x.x, y.x);
+          MS[e][j] = f2(x.y, y.y);
+          MNS[e][j] = f2(-x.y, -y.y);
+        }
+      // The thread's rows of consecutive tiles are STEP apart across the tile
+      // boundary too, so the phasor (cos, sin)(-u(k) theta) carries from one
+      // tile to the next; it is re-seeded exactly every kTcReseed tiles.
+      int k = kb + rg;                        // key of the thread's next row
+      int rem = 0;                            // k mod G
+      float2 C[2], S[2];
+      auto seed = [&]() {
+        const int qd = k / G;
+        rem = k - qd * G;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const float2 x = turn_cs(-(k - qd), p.turns[4 * c + 2 * j]);
+          const float2 y = turn_cs(-(k - qd), p.turns[4 * c + 2 * j + 1]);
+          C[j] = f2(x.x, y.x);
+          S[j] = f2(x.y, y.y);
+        }
+      };
+      auto mult = [&](int e) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const float2 cn = fma2(C[j], MC[e][j], mul2(S[j], MNS[e][j]));
+          const float2 sn = fma2(C[j], MS[e][j], mul2(S[j], MC[e][j]));
+          C[j] = cn;
+          S[j] = sn;
+        }
+      };
+      // u(k + STEP) - u(k) = STEP - (floor((k + STEP)/G) - floor(k/G))
+      auto advance = [&]() {
+        k += STEP;
+        if (stepr == 0) {
+          mult(0);
+        } else {
+          rem += stepr;
+          if (rem >= G) {
+            rem -= G;
+            mult(1);
+          } else {
+            mult(0);
+          }
+        }
+      };
+      // (x0 c - x1 s, x0 s + x1 c) on the chunk's four pairs, (c, s) = (cos, sin)(-u theta)
+      auto turn = [&](uint4 x) -> uint4 {
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        uint32_t y[4];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const float2 X0 = f2(bf16lo(w[2 * j]), bf16lo(w[2 * j + 1]));
+          const float2 X1 = f2(bf16hi(w[2 * j]), bf16hi(w[2 * j + 1]));
+          const float2 Y0 = fma2(neg2(X1), S[j], mul2(X0, C[j]));
+          const float2 Y1 = fma2(X0, S[j], mul2(X1, C[j]));
+          y[2 * j] = pack_bf16x2(Y0.x, Y1.x);
+          y[2 * j + 1] = pack_bf16x2(Y0.y, Y1.y);
+        }
+        return make_uint4(y[0], y[1], y[2], y[3]);
+      };
+      for (int t = 0; t < nrot; ++t) {
+        const int s = t % NS;
+        if (!__all_sync(0xffffffffu, mbar_wait(kfull + s, (t / NS) & 1, abort_flag))) break;
+        if (t % kTcReseed == 0) seed();
+        uint8_t* kt = smem + L::kK + s * L::kTileBytes + (c >> 3) * L::kBlk;
+        const int k0 = kb + t * kTcKeys;
+        if (k0 + kTcKeys <= kr_end) {
+          // every row of the tile is remote: all loads first, then rotate and store
+          uint4 x[NR];
+#pragma unroll
+          for (int m = 0; m < NR; ++m) {
+            const int r = rg + STEP * m;
+            x[m] = *reinterpret_cast<const uint4*>(kt + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+          }
+#pragma unroll
+          for (int m = 0; m < NR; ++m) {
+            x[m] = turn(x[m]);
+            advance();
+          }
+#pragma unroll
+          for (int m = 0; m < NR; ++m) {
+            const int r = rg + STEP * m;
+            *reinterpret_cast<uint4*>(kt + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = x[m];
+          }
+        } else {
+          // the tile reaching the local window (or the end of the split)
+#pragma unroll
+          for (int m = 0; m < NR; ++m) {
+            const int r = rg + STEP * m;
+            if (k < kr_end) {
+              uint4* a = reinterpret_cast<uint4*>(kt + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+              *a = turn(*a);
+            }
+            advance();
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(rot + s);
+      }
+    }
+  } else {
+    // -------------------------------------------------------------- softmax
+    const int r = tid;                                   // key row of a tile; O^T row (dimension)
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const float sl2 = p.scale_log2;
+    auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+    };
+    float m_run[GP], l_thr[GP];
+#pragma unroll
+    for (int gi = 0; gi < GP; ++gi) {
+      m_run[gi] = -INFINITY;
+      l_thr[gi] = 0.f;
+    }
+    bool ok = true;
+    for (int t = 0; t < ntile; ++t) {
+      const int k = kb + t * kTcKeys + r;
+      if (!wwait(s_full + (t & 1), (t >> 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sv[NB];
+      if constexpr (NB == 16) {
+        tmem_ld16(tS + (t & 1) * NB + lane_off, *reinterpret_cast<uint32_t(*)[16]>(sv));
+      } else {
+        tmem_ld32(tS + (t & 1) * NB + lane_off, *reinterpret_cast<uint32_t(*)[32]>(sv));
+      }
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(s_free + (t & 1));
+      const bool valid = k < ke;
+      const bool remote = ROT != 0 && k < p.k_local;
+      float sc[GP], wm[GP];
+#pragma unroll
+      for (int gi = 0; gi < GP; ++gi) {
+        const uint32_t raw = remote ? sv[(ROT != 0 ? GP : 0) + gi] : sv[gi];
+        sc[gi] = valid ? __uint_as_float(raw) * sl2 : -INFINITY;
+        wm[gi] = sc[gi];
+      }
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1)
+#pragma unroll
+        for (int gi = 0; gi < GP; ++gi) wm[gi] = fmaxf(wm[gi], __shfl_xor_sync(0xffffffffu, wm[gi], off));
+      float* rb = red + (t & 1) * 4 * GP;
+      if (lane == 0) {
+#pragma unroll
+        for (int gi = 0; gi < GP; ++gi) rb[warp * GP + gi] = wm[gi];
+        mbar_arrive(mx + (t & 1));
+      }
+      if (!wwait(mx + (t & 1), (t >> 1) & 1)) { ok = false; break; }
+      bool need_any = false;
+      float corr[GP];
+      uint32_t pb[GP];
+#pragma unroll
+      for (int gi = 0; gi < GP; ++gi) {
+        const float tmax = fmaxf(fmaxf(rb[gi], rb[GP + gi]), fmaxf(rb[2 * GP + gi], rb[3 * GP + gi]));
+        // lazy rescale: move the reference max only when it grows by > 8 (x256)
+        const bool need = tmax > m_run[gi] + 8.0f;
+        const float m_new = need ? tmax : m_run[gi];
+        corr[gi] = need ? ex2(m_run[gi] - m_new) : 1.0f;
+        l_thr[gi] *= corr[gi];
+        m_run[gi] = m_new;
+        need_any |= need;
+        const float mu = m_new == -INFINITY ? 0.f : m_new;
+        const float pval = ex2(sc[gi] - mu);
+        l_thr[gi] += pval;
+        pb[gi] = pack_bf16x2(pval, 0.f) & 0xFFFFu;
+      }
+      // P^T buffer t&1 was last read by PV(t-2)
+      if (t >= 2 && !wwait(pv_done + (t & 1), ((t >> 1) - 1) & 1)) { ok = false; break; }
+      if (t >= 1 && need_any) {
+        // rescale O^T (lane r = output dimension r) once PV(t-1) has completed
+        if (!wwait(pv_done + ((t - 1) & 1), ((t - 1) >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t o[kTcNP];
+        tmem_ld16(tO + lane_off, o);
+        tmem_ld_wait();
+#pragma unroll
+        for (int gi = 0; gi < GP; ++gi) o[gi] = __float_as_uint(__uint_as_float(o[gi]) * corr[gi]);
+        tmem_st16(tO + lane_off, o);
+        tmem_st_wait();
+      }
+      uint8_t* pbuf = sP + (t & 1) * L::kPBuf;
+#pragma unroll
+      for (int gi = 0; gi < GP; ++gi)
+        *reinterpret_cast<uint16_t*>(pbuf + sw128_off(gi, r, kTcNP * 128)) = static_cast<uint16_t>(pb[gi]);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_full + (t & 1));
+    }
+    // the last PV has completed: O^T row r holds this split's unnormalised
+    // output of dimension r for every head of the group
+    if (ok && ntile > 0 && wwait(pv_done + ((ntile - 1) & 1), ((ntile - 1) >> 1) & 1)) {
+      tc_fence_after();
+      tmem_ld16(tO + lane_off, o_fin);
+      tmem_ld_wait();
+    } else {
+#pragma unroll
+      for (int i = 0; i < kTcNP; ++i) o_fin[i] = 0u;
+    }
+#pragma unroll
+    for (int gi = 0; gi < GP; ++gi) {
+      float l = l_thr[gi];
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+      l_fin[gi] = l;
+      m_fin[gi] = m_run[gi];
+    }
+  }
+
+  // ------------------------------------------------------ split partials
+  tc_fence_before();
+  __syncthreads();   // every role is done with the ring, TMEM and the reduction buffer
+  float* lsum = red;   // [4 warps][GP] sums, then [GP] maxima
+  if (warp < 4) {
+    if (lane == 0) {
+#pragma unroll
+      for (int gi = 0; gi < GP; ++gi) {
+        lsum[warp * GP + gi] = l_fin[gi];
+        if (warp == 0) lsum[4 * GP + gi] = m_fin[gi];   // the reference max, the same in every thread
+      }
+    }
+    if (tid < D) {
+#pragma unroll
+      for (int gi = 0; gi < GP; ++gi) {
+        if (gi < grp) {
+          const int hq = hkv * grp + gi;
+          const size_t pslot = (static_cast<size_t>(b) * p.Hq + hq) * p.nsplit + split;
+          p.part_o[pslot * D + tid] = __uint_as_float(o_fin[gi]);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (tid < grp) {
+    const int gi = tid;
+    const float l = (lsum[gi] + lsum[GP + gi]) + (lsum[2 * GP + gi] + lsum[3 * GP + gi]);
+    const int hq = hkv * grp + gi;
+    const size_t pslot = (static_cast<size_t>(b) * p.Hq + hq) * p.nsplit + split;
+    p.part_ml[pslot] = make_float2(lsum[4 * GP + gi], l);
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const int prev = atomicAdd(p.counters + b * p.Hkv + hkv, 1);
+    *last_flag = (prev == p.nsplit - 1) ? 1 : 0;
+  }
+  __syncthreads();
+  if (*last_flag) {
+    // last CTA of this (batch, kv head): merge every split, in split order
+    __threadfence();
+    for (int idx = tid; idx < grp * D; idx += kTcThreads) {
+      const int gi = idx / D, d = idx % D;
+      const int hq = hkv * grp + gi;
+      const size_t base = (static_cast<size_t>(b) * p.Hq + hq) * p.nsplit;
+      float M = -INFINITY;
+      for (int sp = 0; sp < p.nsplit; ++sp) {
+        const float2 ml = __ldcg(p.part_ml + base + sp);
+        if (ml.y > 0.f) M = fmaxf(M, ml.x);
+      }
+      float o = 0.f, l = 0.f;
+      for (int sp = 0; sp < p.nsplit; ++sp) {
+        const float2 ml = __ldcg(p.part_ml + base + sp);
+        if (ml.y > 0.f) {
+          const float f = ex2(ml.x - M);
+          o = fmaf(__ldcg(p.part_o + (base + sp) * D + d), f, o);
+          l = fmaf(ml.y, f, l);
+        }
+      }
+      p.out[(static_cast<size_t>(b) * p.Hq + hq) * D + d] = o / l;
+      if (d == 0) p.lse[static_cast<size_t>(b) * p.Hq + hq] = (M + __log2f(l)) * 0.69314718055994530942f;
+    }
+    if (tid == 0) p.counters[b * p.Hkv + hkv] = 0;
+  }
+  if (*abort_flag) {
+    // let in-flight TMA and MMA work drain before the CTA releases its memory
+    const unsigned long long t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 20000000ull) __nanosleep(100000);
+  }
+  if (warp == kTcWarpQK) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+}  // namespace ropeattn

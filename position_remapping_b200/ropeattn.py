@@ -124,9 +124,20 @@ def _check(rc: int):
         raise RopeAttnError(rc, lib.ropeattn_last_error().decode())
 
 
+def _current_device() -> int:
+    return torch.cuda.current_device()
+
+
+def _device_of(t: torch.Tensor):
+    return t.device.type, t.device.index
+
+
 def _stream(stream) -> Optional[int]:
     if stream is None:
         stream = torch.cuda.current_stream()
+    dev = getattr(stream, "device", None)
+    if dev is not None and dev.index != _current_device():
+        raise ValueError(f"the stream belongs to {dev}, but the current device is cuda:{_current_device()}")
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
@@ -145,9 +156,20 @@ def _need(t, name: str, dtype, shape=None) -> torch.Tensor:
         raise ValueError(f"{name} must have shape {tuple(shape)} (got {tuple(t.shape)})")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
-    if t.device.type != "cuda":
-        raise ValueError(f"{name} must be on a CUDA device (got {t.device})")
+    _need_current_device(t, name)
     return t
+
+
+def _need_current_device(t: torch.Tensor, name: str) -> None:
+    # the library builds its TMA maps and launches on the current device, so
+    # every tensor must live there (a pointer into another GPU's memory would
+    # be read by a kernel on this one)
+    kind, index = _device_of(t)
+    if kind != "cuda":
+        raise ValueError(f"{name} must be on a CUDA device (got {t.device})")
+    cur = _current_device()
+    if index != cur:
+        raise ValueError(f"{name} is on cuda:{index}, but the current device is cuda:{cur}")
 
 
 def _need_ndim(t, name: str, dtype, ndim: int) -> torch.Tensor:
@@ -159,8 +181,9 @@ def _need_ndim(t, name: str, dtype, ndim: int) -> torch.Tensor:
 def _need_workspace(ws: Optional[torch.Tensor]) -> Optional[torch.Tensor]:
     if ws is None:
         return None
-    if not isinstance(ws, torch.Tensor) or not ws.is_contiguous() or ws.device.type != "cuda":
+    if not isinstance(ws, torch.Tensor) or not ws.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA tensor")
+    _need_current_device(ws, "workspace")
     return ws
 
 

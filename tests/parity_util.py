@@ -7,6 +7,15 @@ OUT_TOL = 1e-2
 LSE_TOL = 1e-3
 
 
+def decode_staged(D):
+    """Whether the oracle decode should round its operands to bf16 for a
+    comparison with the CUDA decode: for head_dim 64 and 128 the decode
+    multiplies bf16 operands on the tensor cores (the rotated query views and
+    the corrected remote keys are rounded to bf16); at head_dim 256 it keeps
+    its rotations and dot products in fp32 registers."""
+    return D <= 128
+
+
 def max_abs(a, b):
     a = np.asarray(a, dtype=np.float64)
     b = np.asarray(b, dtype=np.float64)

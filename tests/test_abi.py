@@ -196,3 +196,30 @@ def test_binding_checks_tensors_before_the_call(ra):
     for i, fn in enumerate(cases):
         with pytest.raises((ValueError, TypeError)):
             fn()
+
+
+def test_binding_rejects_tensors_of_another_device(ra, monkeypatch):
+    # every tensor must live on the current device (the library launches there
+    # and encodes its pointers into TMA maps); the device is faked here, so no
+    # kernel and no GPU are involved
+    import torch
+    from position_remapping_b200.inputs import BIFOCAL
+    p = _p(kind=BIFOCAL, w0=4, w_pretrained=8)
+    q = torch.zeros((1, 16, 2, 64), dtype=torch.bfloat16)
+    k = torch.zeros((1, 16, 1, 64), dtype=torch.bfloat16)
+    ws = torch.zeros(1024, dtype=torch.uint8)
+    other = {id(k): 1}                                       # k claims cuda:1, the rest cuda:0
+    monkeypatch.setattr(ra, "_current_device", lambda: 0)
+    monkeypatch.setattr(ra, "_device_of", lambda t: ("cuda", other.get(id(t), 0)))
+    called = []
+    monkeypatch.setattr(ra, "_check", lambda rc: called.append(rc))
+    for fn in (lambda: ra.prefill(q, k, k, p, workspace=ws),
+               lambda: ra.decode(q[:, 0].contiguous(), k, k, p, workspace=ws),
+               lambda: ra.cache_write(k, k, q, q, p, 0)):
+        with pytest.raises(ValueError, match="cuda:1"):
+            fn()
+    other.clear()
+    other[id(ws)] = 2                                        # only the workspace elsewhere
+    with pytest.raises(ValueError, match="cuda:2"):
+        ra.prefill(q, k, k, p, workspace=ws)
+    assert not called                                        # no library call was made

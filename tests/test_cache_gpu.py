@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import oracle as O
-from parity_util import assert_close
+from parity_util import assert_close, decode_staged
 from position_remapping_b200.inputs import MapParams, make_qkv
 
 pytestmark = pytest.mark.gpu
@@ -107,7 +107,7 @@ def test_multistep_decode_across_group_changes():
     seen_G = set()
     for i, n in enumerate(range(S0 + 1, N + 1)):
         seen_G.add(O.group_size(n, params.w_pretrained))
-        ref_o, ref_l = O.decode(q[:, n - 1], cache[:, :n], v[:, :n], params)
+        ref_o, ref_l = O.decode(q[:, n - 1], cache[:, :n], v[:, :n], params, stage_bf16=decode_staged(D))
         assert_close(outs[i].cpu().numpy(), lses[i].cpu().numpy(), ref_o, ref_l, f"n={n}")
     assert seen_G == {2, 3, 4}
 
@@ -137,7 +137,7 @@ def test_batched_decode_over_caches_with_spare_rows():
     for i, n in enumerate(range(S0 + 1, N + 1)):
         if i % 7 and n not in (768, 769, 770, N):
             continue   # a sample of the steps, and every step around the G change
-        ref_o, ref_l = O.decode(q[:, n - 1], cache[:, :n], v[:, :n], params)
+        ref_o, ref_l = O.decode(q[:, n - 1], cache[:, :n], v[:, :n], params, stage_bf16=decode_staged(D))
         assert_close(outs[i][0].cpu().numpy(), outs[i][1].cpu().numpy(), ref_o, ref_l, f"n={n}")
     # the same call on a dense copy of the first n rows gives the same bits
     n = N

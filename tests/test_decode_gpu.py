@@ -6,7 +6,7 @@ import pytest
 import torch
 
 import oracle as O
-from parity_util import assert_close
+from parity_util import assert_close, decode_staged
 from position_remapping_b200.inputs import WORKLOADS, MapParams, make_qkv
 
 pytestmark = pytest.mark.gpu
@@ -28,6 +28,16 @@ SMALL = [
     ("bifocal_g2_edge_local", 1, 3000, 2, 1, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=2900, w_pretrained=1500)),
     ("bifocal_fixed_g5_phasor", 1, 3000, 4, 2, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=200, fixed_group=5)),
     ("bifocal_fixed_g4_table", 1, 5000, 8, 4, 128, MapParams(O.BIFOCAL, rope_base=1e4, w0=300, fixed_group=4)),
+    # GQA groups up to 16 (padded to a power of two on the tensor cores), group
+    # sizes G that do not divide the rotation's row step, short caches
+    ("standard_grp16_d128", 1, 3000, 32, 2, 128, MapParams(O.STANDARD, rope_base=1e4)),
+    ("bifocal_grp8_g3", 1, 6000, 16, 2, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=500, w_pretrained=2000)),
+    ("bifocal_grp16_d128", 1, 3000, 16, 1, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=300, w_pretrained=1000)),
+    ("bifocal_grp16_d64_g3", 2, 2000, 32, 2, 64, MapParams(O.BIFOCAL, rope_base=1e4, w0=100, w_pretrained=700)),
+    ("bifocal_grp3", 1, 2500, 12, 4, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=200, w_pretrained=900)),
+    ("bifocal_fixed_g7_d64", 1, 3001, 4, 2, 64, MapParams(O.BIFOCAL, rope_base=1e4, w0=129, fixed_group=7)),
+    ("bifocal_n130_w0_1", 1, 130, 2, 1, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=1, w_pretrained=64)),
+    ("endprompt_grp8_d64", 2, 1500, 16, 2, 64, MapParams(O.ENDPROMPT, rope_base=5e5, interp=8.0, seg1_len=1400, term_start=65000)),
     ("d256_standard", 1, 3000, 2, 1, 256, MapParams(O.STANDARD, rope_base=1e4)),
     ("d256_bifocal_g3_grp2", 2, 5000, 4, 2, 256, MapParams(O.BIFOCAL, rope_base=1e6, w0=400, w_pretrained=2000)),
     ("d256_periodic", 1, 2500, 2, 2, 256, MapParams(O.PERIODIC, rope_base=1e4, window=512)),
@@ -48,7 +58,7 @@ def test_decode_small(case):
     name, B, n, Hq, Hkv, D, params = case
     q, kc, vc = make_qkv(B, n, Hq, Hkv, D, seed=zlib.crc32(name.encode()) % 10000, q_len=1)
     out, lse = _run(q, kc, vc, params)
-    ref_o, ref_l = O.decode(q, kc, vc, params)
+    ref_o, ref_l = O.decode(q, kc, vc, params, stage_bf16=decode_staged(D))
     assert_close(out.cpu().numpy(), lse.cpu().numpy(), ref_o, ref_l, name)
 
 
@@ -56,7 +66,7 @@ def test_decode_full_size():
     w = WORKLOADS["bifocal_decode_n131072"]
     q, kc, vc = make_qkv(w.B, w.S, w.Hq, w.Hkv, w.D, w.seed, q_len=1)
     out, lse = _run(q, kc, vc, w.params)
-    ref_o, ref_l = O.decode(q, kc, vc, w.params)
+    ref_o, ref_l = O.decode(q, kc, vc, w.params, stage_bf16=decode_staged(w.D))
     assert_close(out.cpu().numpy(), lse.cpu().numpy(), ref_o, ref_l, w.name)
 
 

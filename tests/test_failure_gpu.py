@@ -7,7 +7,7 @@ import pytest
 import torch
 
 import oracle as O
-from parity_util import assert_close
+from parity_util import assert_close, decode_staged
 from position_remapping_b200.inputs import MapParams, make_qkv
 
 pytestmark = pytest.mark.gpu
@@ -31,7 +31,7 @@ def test_bounded_wait_gives_up_and_context_survives():
     out, lse = ra.decode(q.cuda(), kc.cuda(), vc.cuda(), params)
     torch.cuda.synchronize()
     ra.status()
-    ref_o, ref_l = O.decode(q, kc, vc, params)
+    ref_o, ref_l = O.decode(q, kc, vc, params, stage_bf16=decode_staged(128))
     assert_close(out.cpu().numpy(), lse.cpu().numpy(), ref_o, ref_l, "after timeout")
 
 

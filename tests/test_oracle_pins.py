@@ -401,6 +401,31 @@ def test_decode_equals_last_prefill_row():
 
 
 @pytest.mark.parametrize("kind", [O.STANDARD, O.ENDPROMPT, O.PERIODIC, O.NOPE, O.BIFOCAL])
+def test_staged_decode_equals_last_row_from_cache(kind):
+    # bf16 operand rounding of the decode (rotated query views, corrected
+    # remote keys) is the rounding the chunked prefill from a cache applies to
+    # the same row: prefill_from_cache rotates the raw query straight to f(t)
+    # and each key by f(s) - s, decode goes through Delta q and Delta k (Eq. 6)
+    params = {O.STANDARD: MapParams(O.STANDARD, rope_base=1e4),
+              O.ENDPROMPT: MapParams(O.ENDPROMPT, rope_base=5e5, interp=8.0, seg1_len=11, term_start=65500),
+              O.PERIODIC: MapParams(O.PERIODIC, window=5),
+              O.NOPE: MapParams(O.NOPE),
+              O.BIFOCAL: MapParams(O.BIFOCAL, rope_base=1e6, w0=3, w_pretrained=6)}[kind]
+    q, k, v = make_qkv(2, 29, 4, 2, 16, seed=36)
+    qn, kn, vn = O.to_f64(q), O.to_f64(k), O.to_f64(v)
+    cache = O.round_bf16(O.cache_keys(kn, params))          # a bf16 cache, as stored on the device
+    a = O.decode(qn[:, 28], cache, vn, params, stage_bf16=True)
+    b = O.prefill_from_cache(qn[:, 28:], cache, vn, params, 28, stage_bf16=True)
+    assert np.allclose(a[0], b[0][:, 0], atol=1e-12) and np.allclose(a[1], b[1][:, :, 0], atol=1e-12)
+    u = O.decode(qn[:, 28], cache, vn, params, stage_bf16=False)
+    d = max(np.abs(a[0] - u[0]).max(), np.abs(a[1] - u[1]).max())
+    if kind == O.NOPE:
+        assert d == 0.0        # bf16 inputs, no rotation: nothing to round
+    else:
+        assert 1e-7 < d < 0.05  # the rounding is applied, and is of bf16 size
+
+
+@pytest.mark.parametrize("kind", [O.STANDARD, O.ENDPROMPT, O.PERIODIC, O.NOPE, O.BIFOCAL])
 def test_cache_keys_match_complex_form_and_offsets(kind):
     # Eq. 4: the cache entry of token t is its key rotated at the kind's
     # position of t, whatever the chunk it is written in

@@ -15,7 +15,7 @@ import pytest
 import torch
 
 import oracle as O
-from parity_util import assert_close
+from parity_util import assert_close, decode_staged
 from position_remapping_b200.inputs import PAIR_HALF, MapParams, make_qkv
 
 pytestmark = pytest.mark.gpu
@@ -141,7 +141,7 @@ def test_half_split_decode_from_written_cache(case):
     torch.cuda.synchronize()
     ra.status()
     cache = _deinterleave(kc.cpu())          # the heads' own order, as the oracle takes it
-    ref_o, ref_l = O.decode(qd, cache, v, params)
+    ref_o, ref_l = O.decode(qd, cache, v, params, stage_bf16=decode_staged(D))
     assert_close(out.cpu().numpy(), lse.cpu().numpy(), ref_o, ref_l, name)
     if params.kind == O.BIFOCAL and Hq // Hkv <= 2 and D <= 128:
         uo, ul = ra.decode_unfused(qd.cuda(), kc, vc, params)

@@ -7,7 +7,7 @@ import pytest
 import torch
 
 import oracle as O
-from parity_util import assert_close
+from parity_util import assert_close, decode_staged
 from position_remapping_b200.inputs import MapParams, make_qkv
 
 pytestmark = pytest.mark.gpu
@@ -63,6 +63,6 @@ def test_unfused_decode_matches_oracle_and_fused(case):
     of, lf = ra.decode(qd, kd, vd, params)
     torch.cuda.synchronize()
     ra.status()
-    ref_o, ref_l = O.decode(q, kc, vc, params)
+    ref_o, ref_l = O.decode(q, kc, vc, params, stage_bf16=decode_staged(D))
     assert_close(ou.cpu().numpy(), lu.cpu().numpy(), ref_o, ref_l, name + " unfused")
     assert_close(of.cpu().numpy(), lf.cpu().numpy(), ref_o, ref_l, name + " fused")

@@ -13,7 +13,7 @@ import pytest
 import torch
 
 import oracle as O
-from parity_util import assert_close
+from parity_util import assert_close, decode_staged
 from position_remapping_b200.inputs import WORKLOADS, MapParams, make_qkv
 
 pytestmark = pytest.mark.gpu
@@ -48,6 +48,9 @@ def test_decode_noalloc_matches_decode_on_consecutive_calls():
         ra.status()
         assert_close(out.cpu().numpy(), lse.cpu().numpy(), ref_out.cpu().numpy(), ref_lse.cpu().numpy(),
                      "decode_noalloc vs decode")
+        # and both against the float64 oracle (bf16 tensor-core operands at head_dim 128)
+        o_ref, l_ref = O.decode(q.cpu(), kc.cpu(), vc.cpu(), params, stage_bf16=decode_staged(q.shape[-1]))
+        assert_close(out.cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, "decode_noalloc vs oracle")
 
 
 def test_decode_noalloc_rejects_shapes_beyond_its_scratch():
