@@ -51,6 +51,22 @@ def prefill_flops(w) -> float:
     return 4.0 * w.D * pairs * w.Hq * w.B
 
 
+def attended_pairs(w) -> int:
+    """(query, key) pairs per (batch, query head) of a whole prefill: causal,
+    or the W-key window of Periodic RoPE."""
+    S = w.S
+    if w.params.kind == 2 and 0 < w.params.window < S:   # PERIODIC
+        W = w.params.window
+        return W * (W + 1) // 2 + (S - W) * W
+    return S * (S + 1) // 2
+
+
+def prefill_io_bytes(w) -> int:
+    """Algorithmic HBM bytes of a prefill: q, k, v read once (bf16), out (fp32)
+    and lse (fp32) written once."""
+    return 2 * w.B * w.S * (w.Hq + 2 * w.Hkv) * w.D + 4 * w.B * w.S * w.Hq * (w.D + 1)
+
+
 def decode_bytes(w) -> int:
     kv = 2 * w.B * w.S * w.Hkv * w.D * 2
     return kv + w.B * w.Hq * w.D * 2 + w.B * w.Hq * (w.D + 1) * 4
@@ -235,6 +251,8 @@ def run_reference(args):
 
 
 CHUNK = 8192   # tokens of the chunked-prefill measurement (the last rows of the 131072 prefill)
+CONFIGS = ("standard_s512", "endprompt_s8192", "periodic_s32768", "nope_s32768")
+SWEEP = (4096, 8192, 16384, 32768, 65536, 98304, 131072)   # Jet-Long §4.6 Table 7 lengths
 
 
 def _event_ms(fn, reps, stream):
@@ -331,6 +349,108 @@ def measure_decode_comparators(ra, qd, kd, vd, stream):
     return {"standard_rope_decode_us": std_us, "fused_bifocal_decode_us": fused_us,
             "unfused_bifocal_decode_us": unfused_us,
             "decode_fused_vs_standard": std_us / fused_us, "decode_unfused_vs_standard": std_us / unfused_us}
+
+
+def oracle_config_sample(w, q, k, v, n_rows: int):
+    """The oracle on `n_rows` evenly spaced query rows of every query head
+    of batch entry 0 (all rows when n_rows >= S). Returns (TFLOP/s, seconds,
+    sample description)."""
+    import oracle as O
+    S = w.S
+    rows = list(range(S)) if n_rows >= S else [min(S - 1, i * (S // n_rows) + S // (2 * n_rows))
+                                               for i in range(n_rows)]
+    if w.params.kind == 2 and w.params.window > 0:
+        per_row = [min(t + 1, w.params.window) for t in rows]
+    else:
+        per_row = [t + 1 for t in rows]
+    flops = 4.0 * w.D * w.Hq * sum(per_row)
+    t0 = time.perf_counter()
+    O.prefill(q[:1], k[:1], v[:1], w.params, rows=rows, stage_bf16=True)
+    dt = time.perf_counter() - t0
+    what = "all rows" if n_rows >= S else f"{len(rows)} evenly spaced query rows"
+    return flops / dt / 1e12, dt, f"{what} x {w.Hq} query heads of batch entry 0"
+
+
+def measure_configs(ra, peaks, stream, with_oracle: bool):
+    """Every prefill workload (standard 512, EndPrompt 8192, Periodic RoPE
+    SWA and NoPE 32768; the 131072 bifocal prefill and decode are the main
+    timed region) timed alone with CUDA events after the timed region:
+    absolute time, tokens/s, TFLOP/s against the burst bf16 peak (short
+    back-to-back launches), HBM GB/s against the measured copy bandwidth,
+    and the oracle on a bounded sample on the host cores."""
+    res = {}
+    dev = torch.device("cuda", torch.cuda.current_device())
+    tpeak = float(peaks.get("bf16_tflops", 1590.0))
+    hpeak = float(peaks.get("hbm_gbs", 6650.0))
+    for name in CONFIGS:
+        w = WORKLOADS[name]
+        q, k, v = make_qkv(w.B, w.S, w.Hq, w.Hkv, w.D, w.seed, device=dev)
+        out = torch.empty((w.B, w.S, w.Hq, w.D), dtype=torch.float32, device=dev)
+        lse = torch.empty((w.B, w.Hq, w.S), dtype=torch.float32, device=dev)
+        ws = torch.empty(max(1, ra.prefill_workspace_size(w.params, w.B, w.S, w.Hq, w.Hkv, w.D)),
+                         dtype=torch.uint8, device=dev)
+        reps = 200 if w.S <= 1024 else 10
+        ms = _event_ms(lambda: ra.prefill(q, k, v, w.params, out=out, lse=lse, workspace=ws, stream=stream),
+                       reps, stream)
+        flops = 4.0 * w.D * attended_pairs(w) * w.B * w.Hq
+        byts = prefill_io_bytes(w)
+        tf = flops / (ms / 1e3) / 1e12
+        gbs = byts / (ms / 1e3) / 1e9
+        bound = {"standard_s512": "latency", "periodic_s32768": "balanced"}.get(name, "tensor")
+        r = {"ms": ms, "us": ms * 1e3, "tokens_per_s": w.B * w.S / (ms / 1e3), "tflops": tf,
+             "tensor_frac": tf / tpeak, "hbm_gbs": gbs, "hbm_frac": gbs / hpeak, "bound": bound,
+             "flop": flops, "io_bytes": byts,
+             "shape": {"B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D}}
+        if with_oracle:
+            n_rows = w.S if w.S <= 512 else (4 if w.S <= 8192 else 2)
+            otf, osec, sample = oracle_config_sample(w, q.cpu(), k.cpu(), v.cpu(), n_rows)
+            r["cpu_baseline"] = {"tflops": otf, "seconds": osec, "sample": sample, "cores": blas_threads(),
+                                 "extrapolated_full_s": flops / (otf * 1e12) if otf > 0 else None}
+        res[name] = r
+        del q, k, v, out, lse, ws
+    ra.status()
+    return {"note": "each workload alone, CUDA events, prepare + attend; tensor_frac vs the burst bf16 peak, "
+                    "hbm_frac vs the measured copy bandwidth (io_bytes = q, k, v read, out and lse written once)",
+            **res}
+
+
+def measure_sweep(ra, q, k, v, qd, kd, vd, ws, wsd, stream):
+    """Bifocal against standard RoPE over the Jet-Long Table 7 lengths (4K to
+    128K; w_pretrained 32768, so G = 1 up to 32K and the bifocal map is the
+    standard one there), prefill (32/8 heads) and decode (16/8 heads), on
+    leading slices of the 131072-token inputs, CUDA events."""
+    P, Dd = PREFILL, DECODE
+    rows = []
+    od = torch.empty((Dd.B, Dd.Hq, Dd.D), dtype=torch.float32, device=q.device)
+    ld = torch.empty((Dd.B, Dd.Hq), dtype=torch.float32, device=q.device)
+    for S in SWEEP:
+        qs, ks, vs = q[:, :S], k[:, :S], v[:, :S]
+        out = torch.empty((P.B, S, P.Hq, P.D), dtype=torch.float32, device=q.device)
+        lse = torch.empty((P.B, P.Hq, S), dtype=torch.float32, device=q.device)
+        flops = 4.0 * P.D * P.Hq * P.B * S * (S + 1) // 2
+        reps = 2 if S >= 65536 else 5
+        f_ms = _event_ms(lambda: ra.prefill(qs, ks, vs, P.params, out=out, lse=lse, workspace=ws, stream=stream),
+                         reps, stream)
+        s_ms = _event_ms(lambda: ra.prefill(qs, ks, vs, P.params.replace(kind=0), out=out, lse=lse, workspace=ws,
+                                            stream=stream), reps, stream)
+        kds, vds = kd[:, :S], vd[:, :S]
+        f_us = 1e3 * _event_ms(lambda: ra.decode(qd, kds, vds, Dd.params, out=od, lse=ld, workspace=wsd,
+                                                 stream=stream), 50, stream)
+        s_us = 1e3 * _event_ms(lambda: ra.decode(qd, kds, vds, Dd.params.replace(kind=0), out=od, lse=ld,
+                                                 workspace=wsd, stream=stream), 50, stream)
+        dbytes = 2 * Dd.B * S * Dd.Hkv * Dd.D * 2
+        rows.append({"S": S, "G": max(1, -(-S // P.params.w_pretrained)),
+                     "prefill_bifocal_ms": f_ms, "prefill_standard_ms": s_ms,
+                     "prefill_bifocal_tflops": flops / (f_ms / 1e3) / 1e12,
+                     "prefill_bifocal_tokens_per_s": S / (f_ms / 1e3),
+                     "prefill_ratio_vs_standard": s_ms / f_ms,
+                     "decode_bifocal_us": f_us, "decode_standard_us": s_us,
+                     "decode_bifocal_gbs": dbytes / (f_us / 1e6) / 1e9,
+                     "decode_ratio_vs_standard": s_us / f_us})
+        del out, lse
+    ra.status()
+    return {"note": "ratio = standard-RoPE time / bifocal time (the pages' Table 7 reports throughput relative "
+                    "to their baseline); each length alone after the timed region", "rows": rows}
 
 
 def config_dict(n_gpus):
@@ -533,6 +653,9 @@ def main():
     cache_rows = measure_cache_rows(ra, q, k, v, kd, vd, qd, stream)
     comparators = measure_comparators(ra, q, k, v, out, lse, ws, stream)
     comparators.update(measure_decode_comparators(ra, qd, kd, vd, stream))
+    sweep = measure_sweep(ra, q, k, v, qd, kd, vd, ws, wsd, stream)
+    peaks0, _ = load_peaks()
+    configs = measure_configs(ra, peaks0, stream, with_oracle=(world == 1 and not args.no_cpu_baseline))
 
     total_ms, prep_ms, attn_ms, dec_ms, e2e_ms, e2e_dec_ms = max_over_ranks(
         [total_ms, prep_ms, attn_ms, dec_ms, e2e_ms, e2e_dec_ms], world, dev)
@@ -553,7 +676,7 @@ def main():
     tpeak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     hpeak = float(peaks.get("hbm_gbs"))
     src_p = source_hash("prefill_sm100.cuh", "common.cuh")
-    src_d = source_hash("decode_sm100.cuh", "common.cuh")
+    src_d = source_hash("decode_tc_sm100.cuh", "common.cuh")
     tr_p = traffic_record("prefill_kernel", src_p)
     tr_d = traffic_record("decode_kernel", src_d)
 
@@ -576,6 +699,7 @@ def main():
         "prefill_attend_ms": attn_ms / K,
         "prefill_tokens_per_s": world * P.S * P.B * K / ((prep_ms + attn_ms) / 1e3),
         "decode_us_per_token": dec_us,
+        "decode_kcycles_per_token": (dec_us * clocks["sm_mhz"] / 1e3) if clocks else None,
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": tpeak, "unit": "TFLOP/s",
                      "frac": attn_tflops / tpeak, "traffic": tr_p,
                      "kernel": "prefill_kernel<128,4> (attention; D=128, 4 ring slots)",
@@ -583,13 +707,17 @@ def main():
                      "algorithmic": f"{flops:.6g} FLOP per launch"},
         "roofline_decode": {"bound": "hbm", "achieved": dec_gbs, "peak": hpeak, "unit": "GB/s",
                             "frac": dec_gbs / hpeak, "traffic": tr_d,
-                            "kernel": "decode_kernel<128,2,1> (D=128, GQA 2, stage-table rotation; + counter memset)",
+                            "frac_of_nominal_8tbs": dec_gbs / 8000.0,
+                            "kernel": "decode_tc_kernel<128,2,1> (tcgen05 QK/PV, D=128, GQA 2 padded to 2, "
+                                      "remote keys rotated in shared memory; + counter memset)",
                             "peak_source": f"{peak_src} hbm_gbs",
                             "algorithmic": f"{decode_bytes(Dd)} B per launch"},
         "clocks": clocks,
         "gpu_launches": 3 * K,
         "cache_rows": cache_rows,
         "comparators": comparators,
+        "length_sweep": sweep,
+        "configs": configs,
         "e2e": {"value": job_tflops(world, flops, K, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms / K,

@@ -38,6 +38,8 @@
 // kv head) to arrive merges all splits in split order.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "decode_sm100.cuh"
 #include "posmap.cuh"
@@ -100,7 +102,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   constexpr uint32_t kIdescPV = idesc_bf16_f32(128, kTcNP, false, true);   // A = V^T read MN-major
 
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base, by pointer arithmetic on the shared array so the
+  // compiler keeps shared-memory (not generic) loads and stores
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sQ = smem + L::kQ;
   uint8_t* sP = smem + L::kP;
   float* red = reinterpret_cast<float*>(smem + L::kRed);
@@ -314,21 +318,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           S[j] = sn;
         }
       };
-      // u(k + STEP) - u(k) = STEP - (floor((k + STEP)/G) - floor(k/G))
-      auto advance = [&]() {
-        k += STEP;
-        if (stepr == 0) {
-          mult(0);
-        } else {
-          rem += stepr;
-          if (rem >= G) {
-            rem -= G;
-            mult(1);
-          } else {
-            mult(0);
-          }
-        }
-      };
       // (x0 c - x1 s, x0 s + x1 c) on the chunk's four pairs, (c, s) = (cos, sin)(-u theta)
       auto turn = [&](uint4 x) -> uint4 {
         const uint32_t w[4] = {x.x, x.y, x.z, x.w};
@@ -344,6 +333,49 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         return make_uint4(y[0], y[1], y[2], y[3]);
       };
+      // u(k + STEP) - u(k) = STEP - (floor((k + STEP)/G) - floor(k/G)); the
+      // advance without a group-boundary carry when G divides STEP (FAST),
+      // else the carried one picked by selects, so a tile is straight-line code
+      auto advance = [&](auto fast_tag) {
+        constexpr bool FAST = decltype(fast_tag)::value;
+        k += STEP;
+        if constexpr (FAST) {
+          mult(0);
+        } else {
+          rem += stepr;
+          const bool e = rem >= G;
+          rem -= e ? G : 0;
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const float2 mc = e ? MC[1][j] : MC[0][j];
+            const float2 ms = e ? MS[1][j] : MS[0][j];
+            const float2 mns = e ? MNS[1][j] : MNS[0][j];
+            const float2 cn = fma2(C[j], mc, mul2(S[j], mns));
+            const float2 sn = fma2(C[j], ms, mul2(S[j], mc));
+            C[j] = cn;
+            S[j] = sn;
+          }
+        }
+      };
+      // every row of the tile is remote: all loads first, then rotate and store
+      auto tile_full = [&](uint8_t* kt, auto fast_tag) {
+        uint4 x[NR];
+#pragma unroll
+        for (int m = 0; m < NR; ++m) {
+          const int r = rg + STEP * m;
+          x[m] = *reinterpret_cast<const uint4*>(kt + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+        }
+#pragma unroll
+        for (int m = 0; m < NR; ++m) {
+          x[m] = turn(x[m]);
+          advance(fast_tag);
+        }
+#pragma unroll
+        for (int m = 0; m < NR; ++m) {
+          const int r = rg + STEP * m;
+          *reinterpret_cast<uint4*>(kt + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = x[m];
+        }
+      };
       for (int t = 0; t < nrot; ++t) {
         const int s = t % NS;
         if (!__all_sync(0xffffffffu, mbar_wait(kfull + s, (t / NS) & 1, abort_flag))) break;
@@ -351,22 +383,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         uint8_t* kt = smem + L::kK + s * L::kTileBytes + (c >> 3) * L::kBlk;
         const int k0 = kb + t * kTcKeys;
         if (k0 + kTcKeys <= kr_end) {
-          // every row of the tile is remote: all loads first, then rotate and store
-          uint4 x[NR];
-#pragma unroll
-          for (int m = 0; m < NR; ++m) {
-            const int r = rg + STEP * m;
-            x[m] = *reinterpret_cast<const uint4*>(kt + r * 128 + (((c & 7) ^ (r & 7)) << 4));
-          }
-#pragma unroll
-          for (int m = 0; m < NR; ++m) {
-            x[m] = turn(x[m]);
-            advance();
-          }
-#pragma unroll
-          for (int m = 0; m < NR; ++m) {
-            const int r = rg + STEP * m;
-            *reinterpret_cast<uint4*>(kt + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = x[m];
+          if (stepr == 0) {
+            tile_full(kt, std::true_type{});
+          } else {
+            tile_full(kt, std::false_type{});
           }
         } else {
           // the tile reaching the local window (or the end of the split)
@@ -377,7 +397,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               uint4* a = reinterpret_cast<uint4*>(kt + r * 128 + (((c & 7) ^ (r & 7)) << 4));
               *a = turn(*a);
             }
-            advance();
+            advance(std::false_type{});
           }
         }
         fence_proxy_async_smem();
