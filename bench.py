@@ -339,6 +339,16 @@ def measure_decode_comparators(ra, qd, kd, vd, stream):
     wsu = torch.empty(int(ra.lib.ropeattn_decode_unfused_workspace_size(Dd.B, Dd.S, Dd.Hq, Dd.Hkv, Dd.D)),
                       dtype=torch.uint8, device=qd.device)
     std = Dd.params.replace(kind=0)
+    # the decode alone, 200 calls back to back (no prefill output draining
+    # from L2 underneath), and the host time of one call through the binding
+    alone_us = 1e3 * _event_ms(lambda: ra.decode(qd, kd, vd, Dd.params, out=od, lse=ld, workspace=wsd,
+                                                 stream=stream), 200, stream)
+    torch.cuda.synchronize()
+    h0 = time.perf_counter()
+    for _ in range(200):
+        ra.decode(qd, kd, vd, Dd.params, out=od, lse=ld, workspace=wsd, stream=stream)
+    host_us = (time.perf_counter() - h0) / 200 * 1e6
+    torch.cuda.synchronize()
     fused_us = 1e3 * _event_ms(lambda: ra.decode(qd, kd, vd, Dd.params, out=od, lse=ld, workspace=wsd,
                                                  stream=stream), 20, stream)
     unfused_us = 1e3 * _event_ms(lambda: ra.decode_unfused(qd, kd, vd, Dd.params, out=od, lse=ld, workspace=wsu,
@@ -346,7 +356,9 @@ def measure_decode_comparators(ra, qd, kd, vd, stream):
     std_us = 1e3 * _event_ms(lambda: ra.decode(qd, kd, vd, std, out=od, lse=ld, workspace=wsd, stream=stream), 20,
                              stream)
     ra.status()
-    return {"standard_rope_decode_us": std_us, "fused_bifocal_decode_us": fused_us,
+    return {"decode_alone_us": alone_us, "decode_alone_gbs": decode_bytes(Dd) / (alone_us / 1e6) / 1e9,
+            "decode_host_us_per_call": host_us,
+            "standard_rope_decode_us": std_us, "fused_bifocal_decode_us": fused_us,
             "unfused_bifocal_decode_us": unfused_us,
             "decode_fused_vs_standard": std_us / fused_us, "decode_unfused_vs_standard": std_us / unfused_us}
 

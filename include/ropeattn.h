@@ -26,8 +26,8 @@
  *   GQA: query head h reads key/value head h / (Hq / Hkv).
  *   Supported: D in {64, 128, 256} (the prefill runs D = 256 with one
  *   128-row query tile per CTA and 64-key tiles);
- *   Hq % Hkv == 0; decode also needs Hq / Hkv <= 2 for D = 256, <= 4 for
- *   D = 128 and <= 8 for D = 64.
+ *   Hq % Hkv == 0; decode also needs Hq / Hkv <= 16 for D = 64 and 128
+ *   and Hq / Hkv <= 2 for D = 256; the backward needs D = 64 or 128.
  *   Half-split pairing (params.pairing = ROPEATTN_PAIR_HALF): q, k and v are
  *   given in their own order; the rotation pairs coordinates (i, i + D/2),
  *   and key caches hold each rotated key in adjacent order instead (element
@@ -191,6 +191,44 @@ int ropeattn_prefill_attend(const void* q, const void* k, const void* v, float* 
                             int64_t B, int64_t S, int32_t Hq, int32_t Hkv, int32_t D,
                             const ropeattn_params* params,
                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes of ropeattn_prefill_backward: per position map the rotated
+ * queries and keys (bf16) and the angle table, plus the log-sum-exp in log2
+ * units and Delta (fp32, rows padded to a multiple of 64). */
+size_t ropeattn_prefill_backward_workspace_size(const ropeattn_params* params, int64_t B, int64_t S,
+                                                int32_t Hq, int32_t Hkv, int32_t D);
+
+/* Gradients of the prefill: given the forward's inputs, its out and lse, and
+ * the upstream gradient dout of out, writes dq, dk and dv. With P the row
+ * softmax of scale * score(t,s), score(t,s) = <R_a q_t, R_b k_s> at the
+ * kind's positions (Periodic RoPE §3.1 Eq. 2, §3.2 Eq. 4; Jet-Long §3 Eq. 1
+ * and §3.1 Eq. 2-3; EndPrompt abstract), Delta_t = dout_t . out_t and
+ * dS = P (dout . v - Delta):
+ *   dv_s = sum_t P(t,s) dout_t,   dk_s = scale R_b^T sum_t dS(t,s) R_a q_t,
+ *   dq_t = scale R_a^T sum_s dS(t,s) R_b k_s,
+ * each bifocal sum split into its local (exact positions) and remote (f
+ * positions) parts. P is recomputed from lse (no softmax state is saved).
+ * Two tensor-core kernels (tcgen05, TMEM accumulators, no atomics: results
+ * are bitwise reproducible): one per 128-key tile for dk and dv (summing the
+ * query heads of each GQA group), one per 128-row query tile for dq. The
+ * rotated q and k, P and dS are bf16 operands; accumulation is fp32.
+ *   q, k, v, params: as for ropeattn_prefill (same kind, positions, scale,
+ *                    pairing); D = 64 or 128.
+ *   out [B, S, Hq, D] fp32, lse [B, Hq, S] fp32: ropeattn_prefill's results.
+ *   dout [B, S, Hq, D] bf16, device.
+ *   dq [B, S, Hq, D], dk, dv [B, S, Hkv, D]: fp32, device, caller-owned;
+ *                    every element is written (nothing is accumulated into
+ *                    them). With ROPEATTN_PAIR_HALF dq and dk are in the
+ *                    heads' own order, like q and k.
+ *   workspace: device, 256-byte aligned, >= the size above.
+ * S == 0 or B == 0 is a no-op.
+ * Errors: INVALID_ARG (also D not 64 or 128), UNSUPPORTED_DEVICE, WORKSPACE,
+ * CUDA. */
+int ropeattn_prefill_backward(const void* q, const void* k, const void* v, const float* out,
+                              const float* lse, const void* dout, float* dq, float* dk, float* dv,
+                              int64_t B, int64_t S, int32_t Hq, int32_t Hkv, int32_t D,
+                              const ropeattn_params* params, void* workspace, size_t workspace_bytes,
+                              void* stream);
 
 /* Prefill of a chunk of `count` new tokens, at positions start..L-1 with
  * L = start + count, against a decode cache that already holds all L keys

@@ -315,9 +315,12 @@ def prefill_three_call(q, k, v, params, stage_bf16: bool = True):
 # backward of the prefill: gradients of a scalar loss through the routed
 # softmax (the fine-tuning pass EndPrompt's method needs)
 # ----------------------------------------------------------------------------
-def prefill_backward(q, k, v, dout, params):
-    """(dq, dk, dv) of the prefill (unstaged, float64) for an upstream
-    gradient ``dout`` of ``out`` [B,S,Hq,D]; shapes of q, k, v.
+def prefill_backward(q, k, v, dout, params, stage_bf16: bool = False):
+    """(dq, dk, dv) of the prefill (float64) for an upstream gradient ``dout``
+    of ``out`` [B,S,Hq,D]; shapes of q, k, v. ``stage_bf16`` rounds the
+    rotated queries and keys to bf16 wherever they are used (the scores and
+    the products R_a q_t, R_b k_s of the chain rule), the operand rounding of
+    the forward's ``stage_bf16``; the rounding itself is not differentiated.
 
     With P the row softmax of scale * score(t,s) over the allowed keys and
     score(t,s) = <R_a q_t, R_b k_s> ((a, b) the positions the kind assigns
@@ -342,9 +345,13 @@ def prefill_backward(q, k, v, dout, params):
     t = np.arange(S)
     ok = np.stack([_allowed(params, int(r), t) for r in t])          # [S, S]
     local = (t[:, None] - t[None, :]) <= int(params.w0)
+    stage = round_bf16 if stage_bf16 else (lambda a: a)
 
     def rot(x, pos):
         return x if kind == NOPE else rotate(x, pos, freqs, pr)
+
+    def srot(x, pos):
+        return x if kind == NOPE else stage(rotate(x, pos, freqs, pr))
 
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
@@ -352,10 +359,10 @@ def prefill_backward(q, k, v, dout, params):
     for b in range(B):
         for h in range(Hq):
             hk = h // grp
-            ql, kl = rot(q[b, :, h], p_loc), rot(k[b, :, hk], p_loc)
+            ql, kl = srot(q[b, :, h], p_loc), srot(k[b, :, hk], p_loc)
             sc = ql @ kl.T
             if kind == BIFOCAL:
-                qr, kr = rot(q[b, :, h], p_rem), rot(k[b, :, hk], p_rem)
+                qr, kr = srot(q[b, :, h], p_rem), srot(k[b, :, hk], p_rem)
                 sc = np.where(local, sc, qr @ kr.T)
             sc = np.where(ok, sc * scale, -np.inf)
             m = sc.max(axis=1, keepdims=True)

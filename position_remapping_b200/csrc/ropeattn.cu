@@ -15,6 +15,7 @@
 #include "pairing.cuh"
 #include "decode_sm100.cuh"
 #include "decode_tc_sm100.cuh"
+#include "backward_sm100.cuh"
 #include "merge.cuh"
 #include "selftest.cuh"
 #include "posmap.cuh"
@@ -190,8 +191,25 @@ void fill_theta(const ropeattn_params* p, int D, double* theta) {
 }
 
 // theta_i / (2 pi) modulo 1 in 64-bit fixed point (units of 2^-64 turn),
-// computed in long double from the double theta_i of fill_theta.
+// computed in long double from the double theta_i of fill_theta. The last
+// few results are kept per thread (a decode step calls this every time, and
+// the long-double arithmetic costs tens of microseconds of host time).
 void fill_turns(const ropeattn_params* p, int D, unsigned long long* turns) {
+  struct Entry {
+    double base, s;
+    int D;
+    unsigned long long turns[kMaxPairs];
+  };
+  constexpr int kCache = 4;
+  thread_local Entry cache[kCache];
+  thread_local int used = 0, next = 0;
+  const double s = p->kind == ROPEATTN_ENDPROMPT ? p->interp : 1.0;
+  for (int e = 0; e < used; ++e) {
+    if (cache[e].base == p->rope_base && cache[e].s == s && cache[e].D == D) {
+      std::memcpy(turns, cache[e].turns, sizeof(unsigned long long) * (D / 2));
+      return;
+    }
+  }
   double theta[kMaxPairs];
   fill_theta(p, D, theta);
   const long double two_pi = 2.0L * std::acos(-1.0L);
@@ -201,6 +219,13 @@ void fill_turns(const ropeattn_params* p, int D, unsigned long long* turns) {
     const long double r = std::floor(std::ldexp(f, 64) + 0.5L);
     turns[i] = r >= 18446744073709551616.0L ? 0ull : static_cast<unsigned long long>(r);   // 2^64 wraps to 0
   }
+  Entry& slot = cache[next];
+  slot.base = p->rope_base;
+  slot.s = s;
+  slot.D = D;
+  std::memcpy(slot.turns, turns, sizeof(unsigned long long) * (D / 2));
+  next = (next + 1) % kCache;
+  if (used < kCache) ++used;
 }
 
 float scale_log2(const ropeattn_params* p, int D) {
@@ -1013,4 +1038,192 @@ int ropeattn_decode_noalloc(const void* q, const void* k_cache, const void* v_ca
     if (rc) return rc;
   }
   return ropeattn_decode(q, k_cache, v_cache, out, lse, B, n, Hq, Hkv, D, params, ws, kNoAllocScratchBytes, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Backward of the prefill
+// ---------------------------------------------------------------------------
+namespace {
+
+struct BwdLayout {
+  int nmaps;
+  int Sp;
+  size_t off_q[2], off_k[2], off_tab[2], off_lse2, off_delta, total;
+};
+
+// Workspace of a backward: per map the rotated queries and keys (bf16) and
+// the (cos, sin) table; the log-sum-exp in log2 units and Delta, rows padded
+// to a multiple of 64.
+BwdLayout bwd_layout(int eff_kind, long long B, long long S, int Hq, int Hkv, int D) {
+  BwdLayout L{};
+  L.nmaps = eff_kind == ROPEATTN_NOPE ? 0 : (eff_kind == ROPEATTN_BIFOCAL ? 2 : 1);
+  L.Sp = static_cast<int>((S + kBwdN - 1) / kBwdN * kBwdN);
+  size_t off = 0;
+  for (int i = 0; i < L.nmaps; ++i) {
+    L.off_q[i] = off;
+    off += align_up(static_cast<size_t>(B) * S * Hq * D * 2, 256);
+  }
+  for (int i = 0; i < L.nmaps; ++i) {
+    L.off_k[i] = off;
+    off += align_up(static_cast<size_t>(B) * S * Hkv * D * 2, 256);
+  }
+  for (int i = 0; i < L.nmaps; ++i) {
+    L.off_tab[i] = off;
+    off += align_up(static_cast<size_t>(S) * (D / 2) * sizeof(float2), 256);
+  }
+  L.off_lse2 = off;
+  off += align_up(static_cast<size_t>(B) * Hq * L.Sp * sizeof(float), 256);
+  L.off_delta = off;
+  off += align_up(static_cast<size_t>(B) * Hq * L.Sp * sizeof(float), 256);
+  L.total = off;
+  return L;
+}
+
+template <int D>
+int launch_backward(const CUtensorMap* ka, const CUtensorMap* kb, const BwdParams& bp, int grid_a, int grid_b,
+                    cudaStream_t st) {
+  using LA = BwdKVSmem<D>;
+  using LB = BwdQSmem<D>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, LA::kAlloc);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, LB::kAlloc);
+  });
+  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(backward)");
+  bwd_dkdv_kernel<D><<<grid_a, kBwdThreads, LA::kAlloc, st>>>(ka[0], ka[1], ka[2], ka[3], ka[4], ka[5], bp);
+  CUDA_TRY(cudaGetLastError(), "backward dK/dV launch");
+  bwd_dq_kernel<D><<<grid_b, kBwdThreads, LB::kAlloc, st>>>(kb[0], kb[1], kb[2], kb[3], kb[4], kb[5], bp);
+  CUDA_TRY(cudaGetLastError(), "backward dQ launch");
+  return ROPEATTN_OK;
+}
+
+}  // namespace
+
+extern "C" size_t ropeattn_prefill_backward_workspace_size(const ropeattn_params* params, int64_t B, int64_t S,
+                                                           int32_t Hq, int32_t Hkv, int32_t D) {
+  PosMap m;
+  int eff;
+  if (check_shapes(B, S, Hq, Hkv, D) || check_params(params, S, D, &m, &eff) || B == 0 || S == 0) return 0;
+  return bwd_layout(eff, B, S, Hq, Hkv, D).total;
+}
+
+extern "C" int ropeattn_prefill_backward(const void* q, const void* k, const void* v, const float* out,
+                                         const float* lse, const void* dout, float* dq, float* dk, float* dv,
+                                         int64_t B, int64_t S, int32_t Hq, int32_t Hkv, int32_t D,
+                                         const ropeattn_params* params, void* workspace, size_t workspace_bytes,
+                                         void* stream) {
+  g_last_error.clear();
+  int rc = check_shapes(B, S, Hq, Hkv, D);
+  if (rc) return rc;
+  if (D != 64 && D != 128) return fail(ROPEATTN_ERR_INVALID_ARG, "the backward supports D = 64 and 128 (got %d)", D);
+  PosMap m;
+  int eff;
+  rc = check_params(params, S, D, &m, &eff);
+  if (rc) return rc;
+  if (B == 0 || S == 0) return ROPEATTN_OK;
+  const void* ptrs[] = {q, k, v, out, lse, dout, dq, dk, dv};
+  for (const void* x : ptrs) {
+    if (!x) return fail(ROPEATTN_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned16(x)) return fail(ROPEATTN_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  }
+  const long long nkt = (S + kBM - 1) / kBM;
+  if (nkt * Hq * B > 0x7fffffffLL) return fail(ROPEATTN_ERR_INVALID_ARG, "too many tiles");
+  rc = check_device();
+  if (rc) return rc;
+  const BwdLayout lay = bwd_layout(eff, B, S, Hq, Hkv, D);
+  if (!workspace || workspace_bytes < lay.total)
+    return fail(ROPEATTN_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", lay.total,
+                workspace ? workspace_bytes : size_t(0));
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+    return fail(ROPEATTN_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  m.kind = eff;
+
+  // rotated queries and keys per map (the forward's streaming pre-rotation,
+  // run over the query rows too), and the angle tables of every position
+  const void* qm[2] = {q, q};
+  const void* km[2] = {k, k};
+  BwdParams bp{};
+  if (lay.nmaps > 0) {
+    PrepArgs a{};
+    a.tab0 = reinterpret_cast<float2*>(ws + lay.off_tab[0]);
+    a.tab1 = lay.nmaps > 1 ? reinterpret_cast<float2*>(ws + lay.off_tab[1]) : nullptr;
+    a.B = static_cast<int>(B);
+    a.S = static_cast<int>(S);
+    a.D = D;
+    a.half = half_pairing(params) ? 1 : 0;
+    a.m = m;
+    fill_theta(params, D, a.theta);
+    const int rows = 256 / (D / 2);
+    for (int side = 0; side < 2; ++side) {
+      a.k = static_cast<const uint32_t*>(side == 0 ? k : q);
+      a.Hkv = side == 0 ? Hkv : Hq;
+      const size_t* off = side == 0 ? lay.off_k : lay.off_q;
+      a.k_rot0 = reinterpret_cast<uint32_t*>(ws + off[0]);
+      a.k_rot1 = lay.nmaps > 1 ? reinterpret_cast<uint32_t*>(ws + off[1]) : nullptr;
+      rope_prep_kernel<<<static_cast<unsigned>((S + rows - 1) / rows), 256, 0, st>>>(a);
+      CUDA_TRY(cudaGetLastError(), "backward rope_prep launch");
+    }
+    for (int i = 0; i < 2; ++i) {
+      qm[i] = ws + lay.off_q[lay.nmaps > 1 ? i : 0];
+      km[i] = ws + lay.off_k[lay.nmaps > 1 ? i : 0];
+    }
+    bp.tab0 = a.tab0;
+    bp.tab1 = lay.nmaps > 1 ? a.tab1 : a.tab0;
+  }
+  {
+    BwdPrepArgs a{};
+    a.dout = static_cast<const __nv_bfloat16*>(dout);
+    a.out = out;
+    a.lse = lse;
+    a.delta = reinterpret_cast<float*>(ws + lay.off_delta);
+    a.lse2 = reinterpret_cast<float*>(ws + lay.off_lse2);
+    a.B = static_cast<int>(B);
+    a.S = static_cast<int>(S);
+    a.Hq = Hq;
+    a.D = D;
+    a.Sp = lay.Sp;
+    const long long threads = B * S * Hq * 32;
+    bwd_prep_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, st>>>(a);
+    CUDA_TRY(cudaGetLastError(), "backward prep launch");
+  }
+  // kernel A tiles: 64 query rows, 128 keys; kernel B: 128 query rows, 64 keys
+  CUtensorMap ma[6], mb[6];
+  if ((rc = make_map(&ma[0], qm[0], D, Hq, S, B, 64, kBwdN, true))) return rc;
+  if ((rc = make_map(&ma[1], qm[1], D, Hq, S, B, 64, kBwdN, true))) return rc;
+  if ((rc = make_map(&ma[2], km[0], D, Hkv, S, B, 64, kBM, true))) return rc;
+  if ((rc = make_map(&ma[3], km[1], D, Hkv, S, B, 64, kBM, true))) return rc;
+  if ((rc = make_map(&ma[4], v, D, Hkv, S, B, 64, kBM, true))) return rc;
+  if ((rc = make_map(&ma[5], dout, D, Hq, S, B, 64, kBwdN, true))) return rc;
+  if ((rc = make_map(&mb[0], qm[0], D, Hq, S, B, 64, kBM, true))) return rc;
+  if ((rc = make_map(&mb[1], qm[1], D, Hq, S, B, 64, kBM, true))) return rc;
+  if ((rc = make_map(&mb[2], km[0], D, Hkv, S, B, 64, kBwdN, true))) return rc;
+  if ((rc = make_map(&mb[3], km[1], D, Hkv, S, B, 64, kBwdN, true))) return rc;
+  if ((rc = make_map(&mb[4], v, D, Hkv, S, B, 64, kBwdN, true))) return rc;
+  if ((rc = make_map(&mb[5], dout, D, Hq, S, B, 64, kBM, true))) return rc;
+  bp.dq = dq;
+  bp.dk = dk;
+  bp.dv = dv;
+  bp.lse2 = reinterpret_cast<const float*>(ws + lay.off_lse2);
+  bp.delta = reinterpret_cast<const float*>(ws + lay.off_delta);
+  bp.B = static_cast<int>(B);
+  bp.S = static_cast<int>(S);
+  bp.Hq = Hq;
+  bp.Hkv = Hkv;
+  bp.Sp = lay.Sp;
+  bp.nkt = static_cast<int>(nkt);
+  bp.nqt = static_cast<int>(nkt);
+  bp.kind = eff;
+  bp.window = m.window;
+  bp.w0 = m.w0;
+  bp.scale_log2 = scale_log2(params, D);
+  bp.scale = params->softmax_scale > 0.0f ? params->softmax_scale : static_cast<float>(1.0 / std::sqrt(double(D)));
+  bp.half = half_pairing(params) ? 1 : 0;
+  const int grid_a = static_cast<int>(nkt * Hkv * B);
+  const int grid_b = static_cast<int>(nkt * Hq * B);
+  return D == 128 ? launch_backward<128>(ma, mb, bp, grid_a, grid_b, st)
+                  : launch_backward<64>(ma, mb, bp, grid_a, grid_b, st);
 }

@@ -28,6 +28,7 @@ EXPORTS = ("ropeattn_posmap", "ropeattn_cache_write", "ropeattn_prefill_workspac
            "ropeattn_decode_workspace_size", "ropeattn_decode", "ropeattn_decode_cache", "ropeattn_decode_noalloc",
            "ropeattn_status",
            "ropeattn_wait_selftest", "ropeattn_decode_unfused_workspace_size", "ropeattn_decode_unfused",
+           "ropeattn_prefill_backward_workspace_size", "ropeattn_prefill_backward",
            "ropeattn_last_error", "ropeattn_version")
 
 
@@ -103,6 +104,11 @@ def _load() -> ctypes.CDLL:
     lib.ropeattn_decode_unfused.restype = ctypes.c_int
     lib.ropeattn_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, P, vp]
     lib.ropeattn_decode_noalloc.restype = ctypes.c_int
+    lib.ropeattn_prefill_backward_workspace_size.argtypes = [P, i64, i64, i32, i32, i32]
+    lib.ropeattn_prefill_backward_workspace_size.restype = sz
+    lib.ropeattn_prefill_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, P, vp, sz,
+                                              vp]
+    lib.ropeattn_prefill_backward.restype = ctypes.c_int
     lib.ropeattn_status.argtypes = []
     lib.ropeattn_wait_selftest.argtypes = [i64, vp, vp]
     lib.ropeattn_wait_selftest.restype = ctypes.c_int
@@ -292,6 +298,44 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, params: MapParams
     _check(lib.ropeattn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, S, Hq, Hkv, D,
                                 ctypes.byref(cp), _ptr(workspace), ws_bytes, _stream(stream)))
     return out, lse
+
+
+def prefill_backward_workspace_size(params: MapParams, B, S, Hq, Hkv, D) -> int:
+    cp = to_cparams(params)
+    return int(lib.ropeattn_prefill_backward_workspace_size(ctypes.byref(cp), B, S, Hq, Hkv, D))
+
+
+def prefill_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, lse: torch.Tensor,
+                     dout: torch.Tensor, params: MapParams, dq: Optional[torch.Tensor] = None,
+                     dk: Optional[torch.Tensor] = None, dv: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None, stream=None):
+    """Gradients of the prefill: q, k, v as for prefill, out/lse the forward's
+    results, dout [B,S,Hq,D] bf16 the upstream gradient of out. Returns
+    (dq [B,S,Hq,D], dk [B,S,Hkv,D], dv [B,S,Hkv,D]), fp32."""
+    _check_prefill_args(q, k, v)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    _need(out, "out", torch.float32, (B, S, Hq, D))
+    _need(lse, "lse", torch.float32, (B, Hq, S))
+    _need(dout, "dout", torch.bfloat16, (B, S, Hq, D))
+    if dq is None:
+        dq = torch.empty((B, S, Hq, D), dtype=torch.float32, device=q.device)
+    if dk is None:
+        dk = torch.empty((B, S, Hkv, D), dtype=torch.float32, device=q.device)
+    if dv is None:
+        dv = torch.empty((B, S, Hkv, D), dtype=torch.float32, device=q.device)
+    _need(dq, "dq", torch.float32, (B, S, Hq, D))
+    _need(dk, "dk", torch.float32, (B, S, Hkv, D))
+    _need(dv, "dv", torch.float32, (B, S, Hkv, D))
+    _need_workspace(workspace)
+    if workspace is None:
+        workspace = _workspace(prefill_backward_workspace_size(params, B, S, Hq, Hkv, D), q.device)
+    cp = to_cparams(params)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.ropeattn_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
+                                         _ptr(dk), _ptr(dv), B, S, Hq, Hkv, D, ctypes.byref(cp), _ptr(workspace),
+                                         ws_bytes, _stream(stream)))
+    return dq, dk, dv
 
 
 def prefill_three_call(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, params: MapParams,

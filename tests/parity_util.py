@@ -7,6 +7,26 @@ OUT_TOL = 1e-2
 LSE_TOL = 1e-3
 
 
+# Bar of the backward: max-abs error of each gradient tensor at most GRAD_TOL
+# times max(1, the largest |reference| element). The kernels multiply bf16
+# operands (rotated q and k, P, dS, v, dout) with fp32 accumulation; each
+# product carries a relative rounding error of at most 2^-8 from its two
+# operands, so a gradient element that sums n such products of similar size
+# is off by about 2^-8 sqrt(n) / n of the sum's scale and at worst by 2^-8 of
+# the sum of magnitudes. 1e-2 is 2.5 x 2^-8: room for the worst case over a
+# tensor's elements, still far below a structural error (a wrong sign, map or
+# position moves elements by O(1) of the scale).
+GRAD_TOL = 1e-2
+
+
+def grad_error(got, ref):
+    """(max-abs error, bar) of one gradient tensor."""
+    err = max_abs(got, ref)
+    ref = np.asarray(ref, dtype=np.float64)
+    scale = max(1.0, float(np.abs(ref).max()) if ref.size else 0.0)
+    return err, GRAD_TOL * scale
+
+
 def decode_staged(D):
     """Whether the oracle decode should round its operands to bf16 for a
     comparison with the CUDA decode: for head_dim 64 and 128 the decode

@@ -662,3 +662,43 @@ def test_backward_closed_forms():
             for s in keys:
                 want[s] += dout[0, t, 0] / len(keys)
         assert np.allclose(dv[0, :, 0], want, atol=1e-13)
+
+
+@pytest.mark.parametrize("kind", [O.STANDARD, O.PERIODIC, O.ENDPROMPT, O.NOPE])
+def test_staged_backward_is_the_backward_at_rounded_operands(kind):
+    # for one position map, rounding R_p q to bf16 is the same as feeding the
+    # unstaged backward q' = R_p^T round(R_p q): its rotated operand is then
+    # exactly the rounded one (and likewise for k), so the two gradients of
+    # the rotated operands agree, and dq, dk differ only by R_p^T
+    params = {O.STANDARD: MapParams(O.STANDARD, rope_base=1e4),
+              O.PERIODIC: MapParams(O.PERIODIC, rope_base=1e4, window=5),
+              O.ENDPROMPT: MapParams(O.ENDPROMPT, rope_base=5e5, interp=8.0, seg1_len=7, term_start=60000),
+              O.NOPE: MapParams(O.NOPE)}[kind]
+    q, k, v = make_qkv(1, 17, 4, 2, 8, seed=37)
+    qn, kn, vn = O.to_f64(q), O.to_f64(k), O.to_f64(v)
+    dout = np.random.default_rng(5).standard_normal(qn.shape)
+    pos = O.position_maps(params, 17)[0]
+    fr = O.rope_frequencies(8, params.rope_base, params.interp if kind == O.ENDPROMPT else 1.0)
+
+    def requant(x):
+        if kind == O.NOPE:
+            return O.round_bf16(x)
+        return np.stack([O.rotate(O.round_bf16(O.rotate(x[0, :, h], pos, fr)), -pos, fr)
+                         for h in range(x.shape[2])], axis=1)[None]
+    a = O.prefill_backward(qn, kn, vn, dout, params, stage_bf16=True)
+    b = O.prefill_backward(requant(qn), requant(kn), vn, dout, params, stage_bf16=False)
+    for x, y in zip(a, b):
+        assert np.allclose(x, y, atol=1e-10)
+    u = O.prefill_backward(qn, kn, vn, dout, params, stage_bf16=False)
+    d = max(np.abs(x - y).max() for x, y in zip(a, u))
+    assert (d == 0.0) if kind == O.NOPE else (1e-8 < d < 0.1)
+
+
+def test_staged_bifocal_backward_is_close_to_unstaged():
+    params = MapParams(O.BIFOCAL, rope_base=1e6, w0=3, w_pretrained=6)
+    q, k, v = make_qkv(1, 19, 2, 1, 8, seed=38)
+    dout = np.random.default_rng(6).standard_normal((1, 19, 2, 8))
+    a = O.prefill_backward(q, k, v, dout, params, stage_bf16=True)
+    u = O.prefill_backward(q, k, v, dout, params, stage_bf16=False)
+    d = max(np.abs(x - y).max() / max(1.0, np.abs(y).max()) for x, y in zip(a, u))
+    assert 1e-8 < d < 0.05
