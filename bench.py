@@ -483,10 +483,23 @@ def run_profile_case(which: str):
     still larger than L2). prefill: the 131072-token workload's kernel on a
     32768-token sequence with w_pretrained 8192, so G = 4 as in the full run;
     prefill256: the same case at head_dim 256; decode: the full 131072-key
-    decode (512 MiB of cache)."""
+    decode (512 MiB of cache); backward: the backward of the 32768-token
+    case (G = 4)."""
     from position_remapping_b200 import ropeattn as ra
     dev = torch.device("cuda", 0)
-    if which in ("prefill", "prefill256"):
+    if which == "backward":
+        P = PREFILL
+        S = 32768
+        params = P.params.replace(w_pretrained=8192)
+        q, k, v = make_qkv(P.B, S, P.Hq, P.Hkv, P.D, P.seed, device=dev)
+        g = torch.Generator("cpu").manual_seed(P.seed + 1)
+        dout = torch.randn((P.B, S, P.Hq, P.D), generator=g).to(torch.bfloat16).to(dev)
+        out, lse = ra.prefill(q, k, v, params)
+        ws = torch.empty(ra.prefill_backward_workspace_size(params, P.B, S, P.Hq, P.Hkv, P.D), dtype=torch.uint8,
+                         device=dev)
+        for _ in range(3):
+            ra.prefill_backward(q, k, v, out, lse, dout, params, workspace=ws)
+    elif which in ("prefill", "prefill256"):
         P = PREFILL
         S = 32768
         D = 256 if which == "prefill256" else P.D
@@ -513,7 +526,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["prefill", "prefill256", "decode"], default=None,
+    ap.add_argument("--profile", choices=["prefill", "prefill256", "decode", "backward"], default=None,
                     help="run a capture-sized case of one kernel three times (for ncu); no timing, no JSON")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)

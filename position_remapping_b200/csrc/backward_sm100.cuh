@@ -32,11 +32,14 @@
 // pass first, parks its gradient (turned back) in the output rows, and adds
 // it in the local pass's epilogue, as the forward parks its remote partial.
 //
-// Warps of both kernels: 0-3 softmax and epilogue (TMEM lanes 0-127),
-// 4 TMA producer, 5 and 6 issue the two score-side MMAs (S and dP), 7 issues
-// the gradient MMAs. TMEM (512 columns): S[2] at [0,64) and [64,128), dP[2]
-// at [128,256), then the accumulators (kernel A: dV and dK, D columns each;
-// kernel B: dQ).
+// Warps of both kernels: 0-3 and 4-7 the two softmax warpgroups (each owns
+// half of the 64 columns of a score tile and half of the accumulator columns
+// in the epilogue; TMEM lane = row), 8 TMA producer, 9 and 10 issue the two
+// score-side MMAs (S and dP), 11 issues the gradient MMAs. TMEM (512
+// columns): S[2] at [0,64) and [64,128), dP[2] at [128,256), then the
+// accumulators (kernel A: dV and dK, D columns each; kernel B: dQ). The bf16
+// P and dS of a warpgroup's 32 columns are packed into the first 16 of those
+// columns, where only that warpgroup reads the fp32 scores.
 #pragma once
 
 #include "common.cuh"
@@ -46,19 +49,25 @@
 
 namespace ropeattn {
 
-constexpr int kBwdThreads = 256;
+constexpr int kBwdThreads = 384;
 constexpr int kBwdN = 64;       // the 64-wide side of every score tile
+constexpr int kBwdWarpTMA = 8, kBwdWarpS = 9, kBwdWarpDP = 10, kBwdWarpG = 11;
+
+// TMEM column of the bf16 operand (P or dS) for K step kk (16 columns of the
+// score tile): warpgroup 0 packs columns 0-31 into [0,16), warpgroup 1
+// columns 32-63 into [32,48)
+__device__ __forceinline__ uint32_t bwd_pcol(int kk) { return (kk >> 1) * 32 + (kk & 1) * 8; }
 
 struct BwdParams {
   float* dq;             // [B, S, Hq, D]
   float* dk;             // [B, S, Hkv, D]
   float* dv;             // [B, S, Hkv, D]
-  const float* lse2;     // [B, Hq, Sp] forward log-sum-exp times log2(e)
-  const float* delta;    // [B, Hq, Sp] rowsum(dO * O)
+  const float* nlse2;    // [B, Hq, Sp] minus the forward log-sum-exp times log2(e)
+  const float* ndelta;   // [B, Hq, Sp] minus rowsum(dO * O)
   const float2* tab0;    // [S][D/2] (cos, sin) at map-0 positions (null for NoPE)
   const float2* tab1;    // [S][D/2] at remote positions (bifocal)
   int B, S, Hq, Hkv;
-  int Sp;                // row stride of lse2 and delta: S rounded up to 64 (aligned bulk copies)
+  int Sp;                // row stride of nlse2 and ndelta: S rounded up to 64 (aligned bulk copies)
   int nkt, nqt;          // 128-row key tiles / query tiles per sequence
   int kind, window, w0;
   float scale_log2;      // softmax scale * log2(e)
@@ -88,35 +97,87 @@ __device__ __forceinline__ void unrot_pair(float y0, float y1, float c, float s,
   x1 = __fmaf_rn(y1, c, -__fmul_rn(y0, s));
 }
 
-// Writes one gradient row (D fp32 values in adjacent pair order, already
-// turned back and scaled) to `dst`, adding the parked value when `add`;
-// for half-split pairing element pairs (2i, 2i+1) go to (i, i + D/2).
+// Writes half a gradient row: the D/2 fp32 values g of adjacent-order
+// columns [c0, c0 + D/2) (already turned back and scaled) into the row `dst`,
+// adding the parked value when `add`; for half-split pairing element pairs
+// (2i, 2i+1) go to coordinates (i, i + D/2).
 template <int D>
-__device__ __forceinline__ void store_grad_row(float* dst, const float* g, bool add, bool half) {
+__device__ __forceinline__ void store_grad_half(float* dst, const float* g, int c0, bool add, bool half) {
   if (!half) {
 #pragma unroll
-    for (int e = 0; e < D; e += 4) {
+    for (int e = 0; e < D / 2; e += 4) {
       float4 o = make_float4(g[e], g[e + 1], g[e + 2], g[e + 3]);
       if (add) {
-        const float4 pr = *reinterpret_cast<const float4*>(dst + e);
+        const float4 pr = *reinterpret_cast<const float4*>(dst + c0 + e);
         o.x += pr.x; o.y += pr.y; o.z += pr.z; o.w += pr.w;
       }
-      *reinterpret_cast<float4*>(dst + e) = o;
+      *reinterpret_cast<float4*>(dst + c0 + e) = o;
     }
   } else {
+    const int i0 = c0 / 2;
 #pragma unroll
-    for (int i = 0; i < D / 2; i += 4) {
+    for (int i = 0; i < D / 4; i += 4) {
       float4 lo = make_float4(g[2 * i], g[2 * i + 2], g[2 * i + 4], g[2 * i + 6]);
       float4 hi = make_float4(g[2 * i + 1], g[2 * i + 3], g[2 * i + 5], g[2 * i + 7]);
       if (add) {
-        const float4 a = *reinterpret_cast<const float4*>(dst + i);
-        const float4 c = *reinterpret_cast<const float4*>(dst + D / 2 + i);
+        const float4 a = *reinterpret_cast<const float4*>(dst + i0 + i);
+        const float4 c = *reinterpret_cast<const float4*>(dst + D / 2 + i0 + i);
         lo.x += a.x; lo.y += a.y; lo.z += a.z; lo.w += a.w;
         hi.x += c.x; hi.y += c.y; hi.z += c.z; hi.w += c.w;
       }
-      *reinterpret_cast<float4*>(dst + i) = lo;
-      *reinterpret_cast<float4*>(dst + D / 2 + i) = hi;
+      *reinterpret_cast<float4*>(dst + i0 + i) = lo;
+      *reinterpret_cast<float4*>(dst + D / 2 + i0 + i) = hi;
     }
+  }
+}
+
+// Reads D/2 accumulator columns [c0, c0 + D/2) of this thread's TMEM lane,
+// scales them, and for a rotating kind turns each pair back by the table
+// entry of position row `pos` (R^T of the forward's rotation).
+template <int D>
+__device__ __forceinline__ void grad_half_from_tmem(uint32_t taddr, float scale, const float2* tab, int c0,
+                                                    float (&g)[D / 2]) {
+  uint32_t rr[32];
+#pragma unroll
+  for (int c = 0; c < D / 64; ++c) {
+    tmem_ld32(taddr + c0 + c * 32, rr);
+    tmem_ld_wait();
+#pragma unroll
+    for (int e = 0; e < 32; ++e) g[c * 32 + e] = __uint_as_float(rr[e]) * scale;
+  }
+  if (tab != nullptr) {
+#pragma unroll
+    for (int i = 0; i < D / 4; ++i) {
+      const float2 cs = __ldg(tab + c0 / 2 + i);
+      unrot_pair(g[2 * i], g[2 * i + 1], cs.x, cs.y, g[2 * i], g[2 * i + 1]);
+    }
+  }
+}
+
+// P = exp2(score * scale_log2 - lse2) and dS = P (dP - Delta) of 32 columns,
+// packed to bf16 pairs (P only when WITH_P): nl and nd hold -lse2 and -Delta
+// per column (kernel A, nstride 1) or one value for the whole row (kernel B,
+// nstride 0); allowed(c) masks a column.
+template <bool MASK, bool WITH_P, typename Allowed>
+__device__ __forceinline__ void bwd_p_ds(const uint32_t (&sv)[32], const uint32_t (&dv)[32], const float* nl,
+                                         const float* nd, int nstride, float sl2, Allowed allowed,
+                                         uint32_t (&pk)[16], uint32_t (&dk)[16]) {
+  const float2 sl22 = make_float2(sl2, sl2);
+#pragma unroll
+  for (int c = 0; c < 32; c += 2) {
+    const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl22,
+                                make_float2(nl[c * nstride], nl[(c + 1) * nstride]));
+    float2 pv = make_float2(ex2(x.x), ex2(x.y));
+    const float2 dd = __fadd2_rn(make_float2(__uint_as_float(dv[c]), __uint_as_float(dv[c + 1])),
+                                 make_float2(nd[c * nstride], nd[(c + 1) * nstride]));
+    float2 ds = __fmul2_rn(pv, dd);
+    if constexpr (MASK) {
+      // masked columns may hold stale values: select, never multiply
+      if (!allowed(c)) pv.x = ds.x = 0.f;
+      if (!allowed(c + 1)) pv.y = ds.y = 0.f;
+    }
+    if constexpr (WITH_P) pk[c >> 1] = pack_bf16x2(pv.x, pv.y);
+    dk[c >> 1] = pack_bf16x2(ds.x, ds.y);
   }
 }
 
@@ -130,14 +191,14 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint3
 }
 
 // ---------------------------------------------------------------------------
-// Delta_t = dO_t . O_t and the log-sum-exp in log2 units, one warp per row
+// -Delta_t = -dO_t . O_t and minus the log-sum-exp in log2 units, one warp per row
 // ---------------------------------------------------------------------------
 struct BwdPrepArgs {
   const __nv_bfloat16* dout;   // [B, S, Hq, D]
   const float* out;            // [B, S, Hq, D]
   const float* lse;            // [B, Hq, S] natural log
-  float* delta;                // [B, Hq, Sp]
-  float* lse2;                 // [B, Hq, Sp]
+  float* ndelta;               // [B, Hq, Sp] -Delta
+  float* nlse2;                // [B, Hq, Sp] -lse * log2(e)
   int B, S, Hq, D, Sp;
 };
 
@@ -163,8 +224,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdPrepArgs a) {
   for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (lane == 0) {
     const size_t i = (static_cast<size_t>(b) * a.Hq + h) * a.Sp + t;
-    a.delta[i] = acc;
-    a.lse2[i] = __ldg(a.lse + (static_cast<size_t>(b) * a.Hq + h) * a.S + t) * 1.4426950408889634074f;
+    a.ndelta[i] = -acc;
+    a.nlse2[i] = -__ldg(a.lse + (static_cast<size_t>(b) * a.Hq + h) * a.S + t) * 1.4426950408889634074f;
   }
 }
 
@@ -259,10 +320,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(s_full + a, 1);
       mbar_init(dp_full + a, 1);
-      mbar_init(p_full + a, kBM);
+      mbar_init(p_full + a, 2 * kBM);
       mbar_init(sd_free + a, 1);
     }
-    mbar_init(dk_free, kBM);
+    mbar_init(dk_free, 2 * kBM);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -276,7 +337,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t tS = tmem, tDP = tmem + 128, tDV = tmem + 256, tDK = tmem + 256 + D;
 
-  if (warp == 4) {
+  if (warp == kBwdWarpTMA) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0) {
       mbar_arrive_expect_tx(kv_full, (two_maps ? 3 : 2) * L::kKTile);
@@ -305,16 +366,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             float* ld = reinterpret_cast<float*>(smem + L::kLD) + slot * 2 * kBwdN;
             const size_t row = (static_cast<size_t>(b) * p.Hq + h) * p.Sp + t0;
-            bulk_load(ld, p.lse2 + row, ldb, ring_full + slot);
-            bulk_load(ld + kBwdN, p.delta + row, ldb, ring_full + slot);
+            bulk_load(ld, p.nlse2 + row, ldb, ring_full + slot);
+            bulk_load(ld + kBwdN, p.ndelta + row, ldb, ring_full + slot);
           }
         }
       }
     }
-  } else if (warp == 5 || warp == 6) {
+  } else if (warp == kBwdWarpS || warp == kBwdWarpDP) {
     // ------------------------------------- MMA: S^T = K_r Q_r^T, dP^T = V dO^T
     if (lane == 0) {
-      const bool is_s = warp == 5;
+      const bool is_s = warp == kBwdWarpS;
       uint64_t* done = is_s ? s_full : dp_full;
       const uint32_t dcol = is_s ? tS : tDP;
       bool ok = mbar_wait(kv_full, 0, abort_flag);
@@ -339,7 +400,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
     }
-  } else if (warp == 7) {
+  } else if (warp == kBwdWarpG) {
     // ------------------------------ MMA: dV += P^T dO, dK += dS^T Q_r (A from TMEM)
     if (lane == 0) {
       int g = 0;
@@ -356,25 +417,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const uint32_t oaddr = qaddr + L::kQTile;
 #pragma unroll
           for (int kk = 0; kk < kBwdN / 16; ++kk) {
-            umma_ts(tDV, tS + buf * kBwdN + kk * 8, sdesc_sw128(oaddr + kk * 2048, kBwdN * 128, 1024), kIdescG,
-                    (g > 0 || kk > 0) ? 1u : 0u);
+            umma_ts(tDV, tS + buf * kBwdN + bwd_pcol(kk), sdesc_sw128(oaddr + kk * 2048, kBwdN * 128, 1024),
+                    kIdescG, (g > 0 || kk > 0) ? 1u : 0u);
           }
 #pragma unroll
           for (int kk = 0; kk < kBwdN / 16; ++kk) {
-            umma_ts(tDK, tDP + buf * kBwdN + kk * 8, sdesc_sw128(qaddr + kk * 2048, kBwdN * 128, 1024), kIdescG,
-                    (step > 0 || kk > 0) ? 1u : 0u);
+            umma_ts(tDK, tDP + buf * kBwdN + bwd_pcol(kk), sdesc_sw128(qaddr + kk * 2048, kBwdN * 128, 1024),
+                    kIdescG, (step > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(sd_free + buf);
           umma_commit(ring_empty + slot);
         }
       }
     }
-  } else {
+  } else if (warp < 8) {
     // ----------------------------------------------- softmax side, epilogue
-    const int r = tid;                       // key row in the tile = TMEM lane
+    const int r = tid & (kBM - 1);           // key row in the tile = TMEM lane
+    const int hw = warp >> 2;                // warpgroup: columns [32 hw, 32 hw + 32)
     const int s = s0 + r;
     const bool row_ok = s < p.S;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
     };
@@ -393,103 +455,63 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           break;
         }
         tc_fence_after();
-        uint32_t sv[kBwdN], dv[kBwdN];
-        tmem_ld32(tS + buf * kBwdN + lane_off, *reinterpret_cast<uint32_t(*)[32]>(sv));
-        tmem_ld32(tS + buf * kBwdN + 32 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
-        tmem_ld32(tDP + buf * kBwdN + lane_off, *reinterpret_cast<uint32_t(*)[32]>(dv));
-        tmem_ld32(tDP + buf * kBwdN + 32 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(dv + 32));
+        uint32_t sv[32], dv[32];
+        tmem_ld32(tS + buf * kBwdN + hw * 32 + lane_off, sv);
+        tmem_ld32(tDP + buf * kBwdN + hw * 32 + lane_off, dv);
         tmem_ld_wait();
-        const float4* ld4 = reinterpret_cast<const float4*>(smem + L::kLD + slot * 2 * kBwdN * 4);
-        const int t0 = j * kBwdN;
-        // the tile is inside the band for every (t, s) pair: no per-element test
-        const bool full = (static_cast<long long>(t0) - s_last >= ps.hi) &&
-                          (static_cast<long long>(t0 + kBwdN - 1) - s0 <= ps.lo) && (t0 + kBwdN <= p.S) &&
-                          (s0 + kBM <= p.S);
-        uint32_t pk[kBwdN / 2], dk2[kBwdN / 2];
-#pragma unroll
-        for (int c4 = 0; c4 < kBwdN / 4; ++c4) {
-          const float4 l4 = ld4[c4];
-          const float4 d4 = ld4[kBwdN / 4 + c4];
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-          const float dl[4] = {d4.x, d4.y, d4.z, d4.w};
-          float pv[4], dsv[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = c4 * 4 + e;
-            bool allowed = true;
-            if (!full) {
-              const int t = t0 + c;
-              const int dd = t - s;
-              allowed = row_ok && t < p.S && dd >= ps.hi && dd <= ps.lo;
-            }
-            const float x = __fmaf_rn(__uint_as_float(sv[c]), sl2, -lv[e]);
-            pv[e] = allowed ? ex2(x) : 0.f;
-            // (masked columns past S hold stale shared memory: never multiply them)
-            dsv[e] = allowed ? pv[e] * (__uint_as_float(dv[c]) - dl[e]) : 0.f;
-          }
-          pk[2 * c4] = pack_bf16x2(pv[0], pv[1]);
-          pk[2 * c4 + 1] = pack_bf16x2(pv[2], pv[3]);
-          dk2[2 * c4] = pack_bf16x2(dsv[0], dsv[1]);
-          dk2[2 * c4 + 1] = pack_bf16x2(dsv[2], dsv[3]);
+        const float* nl = reinterpret_cast<const float*>(smem + L::kLD) + slot * 2 * kBwdN + hw * 32;
+        const int t0 = j * kBwdN + hw * 32;   // query row of this warpgroup's first column
+        // every (t, s) pair of the tile is inside the band: no per-column test
+        const bool full = (static_cast<long long>(j * kBwdN) - s_last >= ps.hi) &&
+                          (static_cast<long long>(j * kBwdN + kBwdN - 1) - s0 <= ps.lo) &&
+                          (j * kBwdN + kBwdN <= p.S) && (s0 + kBM <= p.S);
+        uint32_t pk[16], dk2[16];
+        if (full) {
+          bwd_p_ds<false, true>(sv, dv, nl, nl + kBwdN, 1, sl2, [](int) { return true; }, pk, dk2);
+        } else {
+          auto allowed = [&](int c) {
+            const int dd = t0 + c - s;
+            return row_ok && t0 + c < p.S && dd >= ps.hi && dd <= ps.lo;
+          };
+          bwd_p_ds<true, true>(sv, dv, nl, nl + kBwdN, 1, sl2, allowed, pk, dk2);
         }
-        // P^T and dS^T (bf16) over the first 32 columns of their fp32 buffers
-        tmem_st32(tS + buf * kBwdN + lane_off, pk);
-        tmem_st32(tDP + buf * kBwdN + lane_off, dk2);
+        // P^T and dS^T (bf16) over the first 16 of this warpgroup's columns
+        tmem_st16(tS + buf * kBwdN + hw * 32 + lane_off, pk);
+        tmem_st16(tDP + buf * kBwdN + hw * 32 + lane_off, dk2);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(p_full + buf);
       }
       if (!ok) break;
-      // ---- pass epilogue: dK of this map, turned back and scaled
+      // ---- pass epilogue: dK of this map, turned back and scaled; this
+      // warpgroup's half of the columns
       if (!wwait(sd_free + ((g - 1) & 1), ((g - 1) >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
-      float gk[D];
-      {
-        uint32_t rr[32];
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          tmem_ld32(tDK + c * 32 + lane_off, rr);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) gk[c * 32 + e] = __uint_as_float(rr[e]) * p.scale;
-        }
-      }
+      float gk[D / 2];
+      const float2* tab = p.tab0 == nullptr ? nullptr
+                          : (ps.sel ? p.tab1 : p.tab0) + static_cast<size_t>(row_ok ? s : 0) * (D / 2);
+      grad_half_from_tmem<D>(tDK + lane_off, p.scale, tab, hw * (D / 2), gk);
       tc_fence_before();
       if (pi + 1 < npass) mbar_arrive(dk_free);   // the next pass may reset dK
       if (row_ok) {
-        if (p.tab0 != nullptr) {
-          const float2* tab = (ps.sel ? p.tab1 : p.tab0) + static_cast<size_t>(s) * (D / 2);
-#pragma unroll
-          for (int i = 0; i < D / 2; ++i) {
-            const float2 cs = __ldg(tab + i);
-            unrot_pair(gk[2 * i], gk[2 * i + 1], cs.x, cs.y, gk[2 * i], gk[2 * i + 1]);
-          }
-        }
         float* dst = p.dk + ((static_cast<size_t>(b) * p.S + s) * p.Hkv + hk) * D;
-        store_grad_row<D>(dst, gk, two_maps && pi > 0, p.half != 0);
+        store_grad_half<D>(dst, gk, hw * (D / 2), two_maps && pi > 0, p.half != 0);
       }
     }
     // ---- dV (every pass and head), after the last gradient MMA
     if (ok && g > 0 && wwait(sd_free + ((g - 1) & 1), ((g - 1) >> 1) & 1)) {
       tc_fence_after();
-      float* dst = p.dv + ((static_cast<size_t>(b) * p.S + (row_ok ? s : 0)) * p.Hkv + hk) * D;
-      uint32_t rr[32];
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        tmem_ld32(tDV + c * 32 + lane_off, rr);
-        tmem_ld_wait();
-        if (row_ok) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(dst + c * 32 + e) = make_float4(
-                __uint_as_float(rr[e]), __uint_as_float(rr[e + 1]), __uint_as_float(rr[e + 2]), __uint_as_float(rr[e + 3]));
-        }
+      float gv[D / 2];
+      grad_half_from_tmem<D>(tDV + lane_off, 1.0f, nullptr, hw * (D / 2), gv);
+      if (row_ok) {
+        float* dst = p.dv + ((static_cast<size_t>(b) * p.S + s) * p.Hkv + hk) * D;
+        store_grad_half<D>(dst, gv, hw * (D / 2), false, false);
       }
     } else if (ok && g == 0 && row_ok) {
-      // a key no query attends (cannot happen for a causal band, kept for safety)
+      // a key no query attends (not reached for causal bands, kept for safety)
       float* dst = p.dv + ((static_cast<size_t>(b) * p.S + s) * p.Hkv + hk) * D;
       float* dstk = p.dk + ((static_cast<size_t>(b) * p.S + s) * p.Hkv + hk) * D;
-      for (int e = 0; e < D; ++e) dst[e] = dstk[e] = 0.f;
+      for (int e = hw * (D / 2); e < (hw + 1) * (D / 2); ++e) dst[e] = dstk[e] = 0.f;
     }
   }
 
@@ -587,7 +609,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (tid == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_free, 1);
-    mbar_init(dq_free, kBM);
+    mbar_init(dq_free, 2 * kBM);
     for (int i = 0; i < NS; ++i) {
       mbar_init(ring_full + i, 1);
       mbar_init(ring_empty + i, 1);
@@ -595,7 +617,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(s_full + a, 1);
       mbar_init(dp_full + a, 1);
-      mbar_init(p_full + a, kBM);
+      mbar_init(p_full + a, 2 * kBM);
       mbar_init(sd_free + a, 1);
     }
     *abort_flag = 0;
@@ -611,7 +633,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t tS = tmem, tDP = tmem + 128, tDQ = tmem + 256;
 
-  if (warp == 4) {
+  if (warp == kBwdWarpTMA) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0) {
       int g = 0;
@@ -638,10 +660,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
     }
-  } else if (warp == 5 || warp == 6) {
+  } else if (warp == kBwdWarpS || warp == kBwdWarpDP) {
     // ----------------------------------------- MMA: S = Q_r K_r^T, dP = dO V^T
     if (lane == 0) {
-      const bool is_s = warp == 5;
+      const bool is_s = warp == kBwdWarpS;
       uint64_t* done = is_s ? s_full : dp_full;
       const uint32_t dcol = is_s ? tS : tDP;
       const uint32_t aaddr = smem_u32(smem + (is_s ? L::kQ : L::kDO));
@@ -666,7 +688,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
     }
-  } else if (warp == 7) {
+  } else if (warp == kBwdWarpG) {
     // ------------------------------------------ MMA: dQ += dS K_r (A from TMEM)
     if (lane == 0) {
       int g = 0;
@@ -681,8 +703,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const uint32_t kaddr = smem_u32(smem + L::kRing + slot * L::kSlotBytes);
 #pragma unroll
           for (int kk = 0; kk < kBwdN / 16; ++kk) {
-            umma_ts(tDQ, tS + buf * kBwdN + kk * 8, sdesc_sw128(kaddr + kk * 2048, kBwdN * 128, 1024), kIdescG,
-                    (step > 0 || kk > 0) ? 1u : 0u);
+            umma_ts(tDQ, tS + buf * kBwdN + bwd_pcol(kk), sdesc_sw128(kaddr + kk * 2048, kBwdN * 128, 1024),
+                    kIdescG, (step > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(sd_free + buf);
           umma_commit(ring_empty + slot);
@@ -690,19 +712,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
     }
-  } else {
+  } else if (warp < 8) {
     // ----------------------------------------------- softmax side, epilogue
-    const int r = tid;                       // query row in the tile = TMEM lane
+    const int r = tid & (kBM - 1);           // query row in the tile = TMEM lane
+    const int hw = warp >> 2;                // warpgroup: key columns [32 hw, 32 hw + 32)
     const int t = t0 + r;
     const bool row_ok = t < p.S;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
     };
     const float sl2 = p.scale_log2;
     const size_t lrow = (static_cast<size_t>(b) * p.Hq + h) * p.Sp + (row_ok ? t : 0);
-    const float lse2 = __ldg(p.lse2 + lrow);
-    const float dlt = __ldg(p.delta + lrow);
+    const float nl = __ldg(p.nlse2 + lrow);
+    const float nd = __ldg(p.ndelta + lrow);
     float* dst = p.dq + ((static_cast<size_t>(b) * p.S + (row_ok ? t : 0)) * p.Hq + h) * D;
     bool ok = true;
     int g = 0;
@@ -714,69 +737,44 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int kv0 = (ps.j_lo + step) * kBwdN;
         if (!wwait(s_full + buf, (g >> 1) & 1) || !wwait(dp_full + buf, (g >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
-        uint32_t sv[kBwdN], dv[kBwdN];
-        tmem_ld32(tS + buf * kBwdN + lane_off, *reinterpret_cast<uint32_t(*)[32]>(sv));
-        tmem_ld32(tS + buf * kBwdN + 32 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
-        tmem_ld32(tDP + buf * kBwdN + lane_off, *reinterpret_cast<uint32_t(*)[32]>(dv));
-        tmem_ld32(tDP + buf * kBwdN + 32 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(dv + 32));
+        uint32_t sv[32], dv[32];
+        tmem_ld32(tS + buf * kBwdN + hw * 32 + lane_off, sv);
+        tmem_ld32(tDP + buf * kBwdN + hw * 32 + lane_off, dv);
         tmem_ld_wait();
         const bool full = (static_cast<long long>(t0) - (kv0 + kBwdN - 1) >= ps.hi) &&
                           (static_cast<long long>(t_last) - kv0 <= ps.lo) && (t0 + kBM <= p.S) &&
                           (kv0 + kBwdN <= p.S);
-        uint32_t dk2[kBwdN / 2];
-#pragma unroll
-        for (int c = 0; c < kBwdN; c += 2) {
-          float ds[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            bool allowed = true;
-            if (!full) {
-              const int sk = kv0 + c + e;
-              const int dd = t - sk;
-              allowed = row_ok && sk < p.S && dd >= ps.hi && dd <= ps.lo;
-            }
-            const float x = __fmaf_rn(__uint_as_float(sv[c + e]), sl2, -lse2);
-            const float pv = allowed ? ex2(x) : 0.f;
-            ds[e] = allowed ? pv * (__uint_as_float(dv[c + e]) - dlt) : 0.f;
-          }
-          dk2[c >> 1] = pack_bf16x2(ds[0], ds[1]);
+        const int k0 = kv0 + hw * 32;        // key of this warpgroup's first column
+        uint32_t pk[16], dk2[16];
+        if (full) {
+          bwd_p_ds<false, false>(sv, dv, &nl, &nd, 0, sl2, [](int) { return true; }, pk, dk2);
+        } else {
+          auto allowed = [&](int c) {
+            const int dd = t - (k0 + c);
+            return row_ok && k0 + c < p.S && dd >= ps.hi && dd <= ps.lo;
+          };
+          bwd_p_ds<true, false>(sv, dv, &nl, &nd, 0, sl2, allowed, pk, dk2);
         }
-        tmem_st32(tS + buf * kBwdN + lane_off, dk2);
+        tmem_st16(tS + buf * kBwdN + hw * 32 + lane_off, dk2);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(p_full + buf);
       }
       if (!ok) break;
-      // ---- pass epilogue: dQ of this map, turned back and scaled
+      // ---- pass epilogue: dQ of this map, turned back and scaled; this
+      // warpgroup's half of the columns
       if (!wwait(sd_free + ((g - 1) & 1), ((g - 1) >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
-      float gq[D];
-      {
-        uint32_t rr[32];
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          tmem_ld32(tDQ + c * 32 + lane_off, rr);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) gq[c * 32 + e] = __uint_as_float(rr[e]) * p.scale;
-        }
-      }
+      float gq[D / 2];
+      const float2* tab = p.tab0 == nullptr ? nullptr
+                          : (ps.sel ? p.tab1 : p.tab0) + static_cast<size_t>(row_ok ? t : 0) * (D / 2);
+      grad_half_from_tmem<D>(tDQ + lane_off, p.scale, tab, hw * (D / 2), gq);
       tc_fence_before();
       if (pi + 1 < npass) mbar_arrive(dq_free);
-      if (row_ok) {
-        if (p.tab0 != nullptr) {
-          const float2* tab = (ps.sel ? p.tab1 : p.tab0) + static_cast<size_t>(t) * (D / 2);
-#pragma unroll
-          for (int i = 0; i < D / 2; ++i) {
-            const float2 cs = __ldg(tab + i);
-            unrot_pair(gq[2 * i], gq[2 * i + 1], cs.x, cs.y, gq[2 * i], gq[2 * i + 1]);
-          }
-        }
-        store_grad_row<D>(dst, gq, two_maps && pi > 0, p.half != 0);
-      }
+      if (row_ok) store_grad_half<D>(dst, gq, hw * (D / 2), two_maps && pi > 0, p.half != 0);
     }
     if (ok && npass == 0 && row_ok) {
-      for (int e = 0; e < D; ++e) dst[e] = 0.f;
+      for (int e = hw * (D / 2); e < (hw + 1) * (D / 2); ++e) dst[e] = 0.f;
     }
   }
 

@@ -1179,8 +1179,8 @@ extern "C" int ropeattn_prefill_backward(const void* q, const void* k, const voi
     a.dout = static_cast<const __nv_bfloat16*>(dout);
     a.out = out;
     a.lse = lse;
-    a.delta = reinterpret_cast<float*>(ws + lay.off_delta);
-    a.lse2 = reinterpret_cast<float*>(ws + lay.off_lse2);
+    a.ndelta = reinterpret_cast<float*>(ws + lay.off_delta);
+    a.nlse2 = reinterpret_cast<float*>(ws + lay.off_lse2);
     a.B = static_cast<int>(B);
     a.S = static_cast<int>(S);
     a.Hq = Hq;
@@ -1207,8 +1207,8 @@ extern "C" int ropeattn_prefill_backward(const void* q, const void* k, const voi
   bp.dq = dq;
   bp.dk = dk;
   bp.dv = dv;
-  bp.lse2 = reinterpret_cast<const float*>(ws + lay.off_lse2);
-  bp.delta = reinterpret_cast<const float*>(ws + lay.off_delta);
+  bp.nlse2 = reinterpret_cast<const float*>(ws + lay.off_lse2);
+  bp.ndelta = reinterpret_cast<const float*>(ws + lay.off_delta);
   bp.B = static_cast<int>(B);
   bp.S = static_cast<int>(S);
   bp.Hq = Hq;
