@@ -465,6 +465,35 @@ def measure_sweep(ra, q, k, v, qd, kd, vd, ws, wsd, stream):
                     "to their baseline); each length alone after the timed region", "rows": rows}
 
 
+def measure_backward(ra, q, k, v, out, lse, peaks, stream):
+    """The backward of the 131072-token bifocal prefill (dq, dk, dv from the
+    forward's out and lse and a seeded upstream gradient), CUDA events after
+    the timed region. The algorithmic work is 2.5x the forward's FLOPs (five
+    contractions per attended pair against the forward's two); the kernels
+    execute 3.5x (S and dP are recomputed by the dq kernel)."""
+    P = PREFILL
+    g = torch.Generator("cpu").manual_seed(P.seed + 1)
+    dout = torch.randn((P.B, P.S, P.Hq, P.D), generator=g).to(torch.bfloat16).to(q.device)
+    dq = torch.empty((P.B, P.S, P.Hq, P.D), dtype=torch.float32, device=q.device)
+    dk = torch.empty((P.B, P.S, P.Hkv, P.D), dtype=torch.float32, device=q.device)
+    dv = torch.empty_like(dk)
+    ws = torch.empty(ra.prefill_backward_workspace_size(P.params, P.B, P.S, P.Hq, P.Hkv, P.D), dtype=torch.uint8,
+                     device=q.device)
+    ra.prefill(q, k, v, P.params, out=out, lse=lse, stream=stream)
+    ms = _event_ms(lambda: ra.prefill_backward(q, k, v, out, lse, dout, P.params, dq=dq, dk=dk, dv=dv, workspace=ws,
+                                               stream=stream), 3, stream)
+    ra.status()
+    flops = 2.5 * prefill_flops(P)
+    tf = flops / (ms / 1e3) / 1e12
+    tpeak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    del dout, dq, dk, dv, ws
+    return {"ms": ms, "tflops": tf, "tokens_per_s": P.B * P.S / (ms / 1e3), "peak": tpeak, "frac": tf / tpeak,
+            "algorithmic": f"{flops:.6g} FLOP per call (2.5x the forward)",
+            "kernels": "rope_prep_kernel x2, bwd_prep_kernel, bwd_dkdv_kernel<128>, bwd_dq_kernel<128>",
+            "note": "prefill backward, 131072 tokens, 32/8 heads, D 128, G = 4; frac vs the measured sustained "
+                    "bf16 peak"}
+
+
 def config_dict(n_gpus):
     return {"workload": f"{PREFILL.name} + {DECODE.name}",
             "prefill": {"B": PREFILL.B, "S": PREFILL.S, "Hq": PREFILL.Hq, "Hkv": PREFILL.Hkv, "D": PREFILL.D,
@@ -680,6 +709,7 @@ def main():
     comparators.update(measure_decode_comparators(ra, qd, kd, vd, stream))
     sweep = measure_sweep(ra, q, k, v, qd, kd, vd, ws, wsd, stream)
     peaks0, _ = load_peaks()
+    backward = measure_backward(ra, q, k, v, out, lse, peaks0, stream)
     configs = measure_configs(ra, peaks0, stream, with_oracle=(world == 1 and not args.no_cpu_baseline))
 
     total_ms, prep_ms, attn_ms, dec_ms, e2e_ms, e2e_dec_ms = max_over_ranks(
@@ -741,6 +771,7 @@ def main():
         "gpu_launches": 3 * K,
         "cache_rows": cache_rows,
         "comparators": comparators,
+        "backward": backward,
         "length_sweep": sweep,
         "configs": configs,
         "e2e": {"value": job_tflops(world, flops, K, e2e_ms), "unit": "TFLOP/s",
