@@ -327,10 +327,12 @@ int ropeattn_decode(const void* q, const void* k_cache, const void* v_cache,
  * (a file-scope __device__ array that every GPU loading the library holds
  * until process exit). Shapes whose ropeattn_decode_workspace_size exceeds
  * 4 MiB are rejected with ROPEATTN_ERR_WORKSPACE before any launch.
- * The first call on a device looks up the array's device address (once per
- * device, with that device current); make that first call before any stream
- * capture. The call itself allocates nothing: it clears the scratch counters
- * with cudaMemsetAsync on `stream` and launches the decode kernel.
+ * Every call looks up the array's device address on the current device (a
+ * table lookup that allocates nothing, so an address never outlives a device
+ * reset); the first call on a device may load the library's device code, so
+ * make that first call before any stream capture. The call allocates
+ * nothing: it clears the scratch counters with cudaMemsetAsync on `stream`
+ * and launches the decode kernel.
  * All calls share the one array: calls that may overlap on the GPU (different
  * streams without ordering, or different host threads) race and must not be
  * issued; calls on one stream are safe. */

@@ -257,16 +257,20 @@ def prefill(q, k, v, params, rows=None, stage_bf16: bool = True):
                 for c0 in range(0, len(rows), 64):
                     rr = rows[c0:c0 + 64]
                     nk = int(rr.max()) + 1            # keys beyond the last row are masked
-                    ok = np.stack([_allowed(params, int(t), keys[:nk]) for t in rr])
+                    # Periodic RoPE: keys before the window of the chunk's first
+                    # row are outside every row's window {t-W+1..t}: skipped
+                    k0 = max(0, int(rr.min()) - int(params.window) + 1) if kind == PERIODIC else 0
+                    ks = keys[k0:nk]
+                    ok = np.stack([_allowed(params, int(t), ks) for t in rr])
                     qq = q[b, rr, h, :]
                     ql = qq if kind == NOPE else stage(rotate(qq, p_loc[rr], freqs, pr))
-                    sc = (ql @ kl[:nk].T) * scale                         # [r, nk]
+                    sc = (ql @ kl[k0:nk].T) * scale                       # [r, nk - k0]
                     if kind == BIFOCAL:
                         qr = stage(rotate(qq, p_rem[rr], freqs, pr))
-                        sr = (qr @ kr[:nk].T) * scale
-                        local = (rr[:, None] - keys[None, :nk]) <= int(params.w0)
+                        sr = (qr @ kr[k0:nk].T) * scale
+                        local = (rr[:, None] - ks[None, :]) <= int(params.w0)
                         sc = np.where(local, sc, sr)
-                    o, l = _softmax_rows(sc, ok, v[b, :nk, hk, :])
+                    o, l = _softmax_rows(sc, ok, v[b, k0:nk, hk, :])
                     out[b, c0:c0 + 64, h, :] = o
                     lse[b, h, c0:c0 + 64] = l
     return out, lse

@@ -349,12 +349,15 @@ __global__ void __launch_bounds__(DecodeShape<D, GRP>::kThreads, 1)
     }
     __syncwarp();
     if (lane == 0) {
-      // the last warp to release the slot refills it with stage st + NS; the
-      // fences order every warp's reads of the slot before the copy's writes
+      // the last warp to release the slot refills it with stage st + NS: the
+      // block fences and the counter order every warp's (generic) reads of the
+      // slot before the last release, and the proxy fence orders them before
+      // the copy engine's (async proxy) writes into the slot
       __threadfence_block();
       if (atomicAdd(released + slot, 1) == NW - 1) {
         __threadfence_block();
         released[slot] = 0;
+        fence_proxy_async_smem();
         if (st + NS < nstage) issue(st + NS);
       }
     }

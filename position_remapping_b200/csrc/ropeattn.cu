@@ -950,21 +950,14 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 namespace {
 
-// Device address of g_noalloc_scratch on the current device, looked up once
-// per device (the host-side name is only a stand-in, never a device address).
+// Device address of g_noalloc_scratch on the current device (the host-side
+// name is only a stand-in, never a device address). Looked up on every call:
+// it is a table lookup that allocates nothing, and a cached address would
+// outlive a device reset that reloads the library's device code.
 int noalloc_scratch_ptr(void** out) {
-  static std::mutex mu;
-  static void* ptrs[64];
-  int dev = 0;
-  CUDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
-  if (dev < 0 || dev >= 64) return fail(ROPEATTN_ERR_UNSUPPORTED_DEVICE, "device index %d", dev);
-  std::lock_guard<std::mutex> lk(mu);
-  if (!ptrs[dev]) {
-    void* p = nullptr;
-    CUDA_TRY(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress(scratch)");
-    ptrs[dev] = p;
-  }
-  *out = ptrs[dev];
+  void* p = nullptr;
+  CUDA_TRY(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress(scratch)");
+  *out = p;
   return ROPEATTN_OK;
 }
 

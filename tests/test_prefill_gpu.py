@@ -104,8 +104,10 @@ def test_prefill_full_size_sampled_rows(name):
     w = WORKLOADS[name]
     q, k, v = make_qkv(w.B, w.S, w.Hq, w.Hkv, w.D, w.seed)
     out, lse = _run(q, k, v, w.params)
-    n_random = 48 if name == "bifocal_prefill_s131072" else 256
-    rows = sample_rows(w.S, w.params, n_random=n_random, edge=32 if w.S > 100000 else 64)
+    if name == "periodic_s32768":
+        rows = list(range(w.S))          # every row: the windowed oracle is cheap here
+    else:
+        rows = sample_rows(w.S, w.params, n_random=512, edge=32 if w.S > 100000 else 64)
     ref_o, ref_l = O.prefill(q, k, v, w.params, rows=rows, stage_bf16=True)
     got_o = out.cpu().numpy()[:, rows]
     got_l = lse.cpu().numpy()[:, :, rows]
