@@ -513,10 +513,21 @@ def run_profile_case(which: str):
     32768-token sequence with w_pretrained 8192, so G = 4 as in the full run;
     prefill256: the same case at head_dim 256; decode: the full 131072-key
     decode (512 MiB of cache); backward: the backward of the 32768-token
-    case (G = 4)."""
+    case (G = 4); prefill131072: the full-size attention, for one-pass
+    counters only."""
     from position_remapping_b200 import ropeattn as ra
     dev = torch.device("cuda", 0)
-    if which == "backward":
+    if which == "prefill131072":
+        # the full-size attention, for one-pass counters (DRAM bytes) only
+        P = PREFILL
+        q, k, v = make_qkv(P.B, P.S, P.Hq, P.Hkv, P.D, P.seed, device=dev)
+        out = torch.empty((P.B, P.S, P.Hq, P.D), dtype=torch.float32, device=dev)
+        lse = torch.empty((P.B, P.Hq, P.S), dtype=torch.float32, device=dev)
+        ws = torch.empty(ra.prefill_workspace_size(P.params, P.B, P.S, P.Hq, P.Hkv, P.D), dtype=torch.uint8,
+                         device=dev)
+        for _ in range(2):
+            ra.prefill(q, k, v, P.params, out=out, lse=lse, workspace=ws)
+    elif which == "backward":
         P = PREFILL
         S = 32768
         params = P.params.replace(w_pretrained=8192)
@@ -555,7 +566,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["prefill", "prefill256", "decode", "backward"], default=None,
+    ap.add_argument("--profile", choices=["prefill", "prefill131072", "prefill256", "decode", "backward"], default=None,
                     help="run a capture-sized case of one kernel three times (for ncu); no timing, no JSON")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
