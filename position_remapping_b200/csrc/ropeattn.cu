@@ -74,10 +74,16 @@ int check_device() {
   return ROPEATTN_OK;
 }
 
+// SM count of the current device, looked up once per device
 int sm_count() {
+  static int cached[64];
   int dev = 0, n = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return n;
+  if (cached[dev] > 0) return cached[dev];
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  n = n > 0 ? n : 148;
+  cached[dev] = n;
+  return n;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {

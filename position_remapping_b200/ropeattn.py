@@ -56,7 +56,23 @@ class CParams(ctypes.Structure):
     ]
 
 
+_CPARAMS_CACHE: dict = {}
+
+
+def _cparams(p: MapParams) -> CParams:
+    """The C parameter struct of `p` for the binding's own calls, which never
+    modify it (cached: MapParams is frozen, and a decode step runs every
+    token)."""
+    c = _CPARAMS_CACHE.get(p)
+    if c is None:
+        c = to_cparams(p)
+        if len(_CPARAMS_CACHE) < 256:
+            _CPARAMS_CACHE[p] = c
+    return c
+
+
 def to_cparams(p: MapParams) -> CParams:
+    """A fresh C parameter struct of `p`."""
     c = CParams()
     c.kind = int(p.kind)
     c.fixed_group = int(p.fixed_group)
@@ -227,7 +243,7 @@ def status() -> None:
 
 
 def posmap(params: MapParams, L: int, device="cuda", stream=None) -> Tuple[torch.Tensor, torch.Tensor, int]:
-    cp = to_cparams(params)
+    cp = _cparams(params)
     loc = torch.empty(max(L, 1), dtype=torch.int32, device=device)
     rem = torch.empty(max(L, 1), dtype=torch.int32, device=device)
     G = ctypes.c_int32(0)
@@ -250,18 +266,18 @@ def cache_write(k: torch.Tensor, v: Optional[torch.Tensor], k_cache: torch.Tenso
         _need(v, "v", torch.bfloat16, k.shape)
         _need(v_cache, "v_cache", torch.bfloat16, k_cache.shape)
     cache_len = k_cache.shape[1]
-    cp = to_cparams(params)
+    cp = _cparams(params)
     _check(lib.ropeattn_cache_write(_ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), B, int(start), count, cache_len,
                                     Hkv, D, ctypes.byref(cp), _stream(stream)))
 
 
 def prefill_workspace_size(params: MapParams, B, S, Hq, Hkv, D) -> int:
-    cp = to_cparams(params)
+    cp = _cparams(params)
     return int(lib.ropeattn_prefill_workspace_size(ctypes.byref(cp), B, S, Hq, Hkv, D))
 
 
 def prefill_chunk_workspace_size(params: MapParams, B, start, count, Hq, Hkv, D) -> int:
-    cp = to_cparams(params)
+    cp = _cparams(params)
     return int(lib.ropeattn_prefill_chunk_workspace_size(ctypes.byref(cp), B, start, count, Hq, Hkv, D))
 
 
@@ -293,7 +309,7 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, params: MapParams
     need = prefill_workspace_size(params, B, S, Hq, Hkv, D)
     if workspace is None:
         workspace = _workspace(need, q.device)
-    cp = to_cparams(params)
+    cp = _cparams(params)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.ropeattn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, S, Hq, Hkv, D,
                                 ctypes.byref(cp), _ptr(workspace), ws_bytes, _stream(stream)))
@@ -301,7 +317,7 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, params: MapParams
 
 
 def prefill_backward_workspace_size(params: MapParams, B, S, Hq, Hkv, D) -> int:
-    cp = to_cparams(params)
+    cp = _cparams(params)
     return int(lib.ropeattn_prefill_backward_workspace_size(ctypes.byref(cp), B, S, Hq, Hkv, D))
 
 
@@ -330,7 +346,7 @@ def prefill_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: tor
     _need_workspace(workspace)
     if workspace is None:
         workspace = _workspace(prefill_backward_workspace_size(params, B, S, Hq, Hkv, D), q.device)
-    cp = to_cparams(params)
+    cp = _cparams(params)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.ropeattn_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
                                          _ptr(dk), _ptr(dv), B, S, Hq, Hkv, D, ctypes.byref(cp), _ptr(workspace),
@@ -353,7 +369,7 @@ def prefill_three_call(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, params
     _need(out, "out", torch.float32, (B, S, Hq, D))
     _need(lse, "lse", torch.float32, (B, Hq, S))
     _need_workspace(workspace)
-    cp = to_cparams(params)
+    cp = _cparams(params)
     if workspace is None:
         workspace = _workspace(int(lib.ropeattn_prefill_three_call_workspace_size(ctypes.byref(cp), B, S, Hq, Hkv, D)),
                                q.device)
@@ -368,7 +384,7 @@ def prefill_prepare(k: torch.Tensor, Hq: int, params: MapParams, workspace: torc
     _need_ndim(k, "k", torch.bfloat16, 4)
     _need_workspace(workspace)
     B, S, Hkv, D = k.shape
-    cp = to_cparams(params)
+    cp = _cparams(params)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.ropeattn_prefill_prepare(_ptr(k), B, S, Hq, Hkv, D, ctypes.byref(cp), _ptr(workspace), ws_bytes,
                                         _stream(stream)))
@@ -383,7 +399,7 @@ def prefill_attend(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, params: Ma
     _need(out, "out", torch.float32, (B, S, Hq, D))
     _need(lse, "lse", torch.float32, (B, Hq, S))
     _need_workspace(workspace)
-    cp = to_cparams(params)
+    cp = _cparams(params)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.ropeattn_prefill_attend(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, S, Hq, Hkv, D,
                                        ctypes.byref(cp), _ptr(workspace), ws_bytes, _stream(stream)))
@@ -410,7 +426,7 @@ def prefill_chunk(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
     _need(out, "out", torch.float32, (B, count, Hq, D))
     _need(lse, "lse", torch.float32, (B, Hq, count))
     _need_workspace(workspace)
-    cp = to_cparams(params)
+    cp = _cparams(params)
     if workspace is None:
         workspace = _workspace(prefill_chunk_workspace_size(params, B, int(start), count, Hq, Hkv, D), q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
@@ -438,7 +454,7 @@ def decode_cache(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, 
     _need_workspace(workspace)
     if workspace is None:
         workspace = _workspace(decode_workspace_size(B, n, Hq, Hkv, D), q.device)
-    cp = to_cparams(params)
+    cp = _cparams(params)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.ropeattn_decode_cache(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse), B, int(n), cache_len,
                                      Hq, Hkv, D, ctypes.byref(cp), _ptr(workspace), ws_bytes, _stream(stream)))
@@ -463,7 +479,7 @@ def decode_unfused(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
     _need_workspace(workspace)
     if workspace is None:
         workspace = _workspace(int(lib.ropeattn_decode_unfused_workspace_size(B, n, Hq, Hkv, D)), q.device)
-    cp = to_cparams(params)
+    cp = _cparams(params)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.ropeattn_decode_unfused(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse), B, n, Hq, Hkv,
                                        D, ctypes.byref(cp), _ptr(workspace), ws_bytes, _stream(stream)))
@@ -488,7 +504,7 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, params
     _need_workspace(workspace)
     if workspace is None:
         workspace = _workspace(decode_workspace_size(B, n, Hq, Hkv, D), q.device)
-    cp = to_cparams(params)
+    cp = _cparams(params)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.ropeattn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse), B, n, Hq, Hkv, D,
                                ctypes.byref(cp), _ptr(workspace), ws_bytes, _stream(stream)))
