@@ -4,7 +4,8 @@
 // Split-KV: CTA (split, kv head, batch) owns a contiguous key range of one kv
 // head; the grid is one wave. The range streams through shared memory by TMA
 // in 128-key tiles (128-byte swizzle, no multicast), K tiles and V tiles in
-// rings of their own. Per tile, with the GQA group's query heads as the MMA's N
+// rings of their own: K in whole tiles, V in 64-key halves, so a V slot is
+// free as soon as the four PV MMAs of its half have read it. Per tile, with the GQA group's query heads as the MMA's N
 // dimension (the tensor cores see the keys as M = 128 rows):
 //   S^T = K' Q^T   tcgen05.mma, A = the K tile (K-major), B = the staged
 //                  query rows (K-major), fp32 into TMEM (lane = key);
@@ -55,33 +56,57 @@ constexpr int kTcWarpQK = 14;     // QK^T issuer (and TMEM allocation)
 constexpr int kTcWarpPV = 15;     // PV issuer
 constexpr int kTcReseed = 8;      // tiles between exact re-seeds of the rotation phasor
 constexpr int kTcNP = 16;         // N of the PV MMA: query heads of the group, padded
+constexpr int kTcMaxSplits = 256;   // key-range splits per (batch, kv head), at most
 
 template <int D, int GP, int ROT>
 struct DecodeTcShape {
   static constexpr int kRows = ROT ? 2 * GP : GP;          // staged query rows
   static constexpr int NB = kRows <= 16 ? 16 : 32;           // N of the QK MMA
-  static constexpr int kStages = D == 128 ? 3 : 6;           // slots of each ring (K and V)
-  static constexpr int kBlk = kTcKeys * 128;                 // one 64-column swizzle block of a tile
-  static constexpr int kTileBytes = kTcKeys * D * 2;         // K or V tile
+  // A K slot is busy from its load through the rotation and the QK MMA; a V
+  // half from its load through its PV MMAs. Each ring must cover the DRAM
+  // latency under load (~4000 cycles) plus that work at the HBM rate, with
+  // the SM clock as low as the power cap takes it: four K tiles and five V
+  // halves at head_dim 128 (208 KiB), seven and twelve at 64.
+  static constexpr int kKSlots = D == 128 ? 4 : 7;           // K ring: whole tiles
+  static constexpr int kVHalves = D == 128 ? 5 : 12;         // V ring: 64-key halves
+  static constexpr int kHalfKeys = kTcKeys / 2;
+  static constexpr int kBlk = kTcKeys * 128;                 // one 64-column swizzle block of a K tile
+  static constexpr int kBlkH = kHalfKeys * 128;              // the same block of a V half
+  static constexpr int kTileBytes = kTcKeys * D * 2;         // K tile
+  static constexpr int kHalfBytes = kHalfKeys * D * 2;       // V half
   static constexpr int kV = 0;                               // V ring, then the K ring
-  static constexpr int kK = kStages * kTileBytes;
-  static constexpr int kQ = 2 * kStages * kTileBytes;        // [D/64][NB rows][128 B]
+  static constexpr int kK = kVHalves * kHalfBytes;
+  static constexpr int kQ = kK + kKSlots * kTileBytes;       // [D/64][NB rows][128 B]
   static constexpr int kQBytes = (D / 64) * NB * 128;
   static constexpr int kP = kQ + kQBytes;                    // [2 bufs][2 key blocks][kTcNP rows][128 B]
   static constexpr int kPBuf = 2 * kTcNP * 128;
   static constexpr int kRed = kP + 2 * kPBuf;                // [2][4 warps][GP] tile maxima, then [4][GP] sums
   static constexpr int kBar = kRed + 2 * 4 * GP * 4 + 64;
-  // kfull, rot, kempty, vfull, vempty [NS each]; s_full, s_free, p_full, pv_done, mx [2 each]
-  static constexpr int kNumBars = 5 * kStages + 10;
+  // kfull, rot, kempty [kKSlots each]; vfull, vempty [kVHalves each];
+  // s_full, s_free, p_full, pv_done, mx [2 each]
+  static constexpr int kNumBars = 3 * kKSlots + 2 * kVHalves + 10;
   static constexpr int kMisc = kBar + kNumBars * 8;          // tmem base, abort flag, last flag
   static constexpr int kTotal = kMisc + 16;
   static constexpr int kAlloc = kTotal + 1024;               // slack to align the base to 1024
   static constexpr uint32_t kTmemCols = (2 * NB + kTcNP) <= 64 ? 64 : 128;
   static_assert(GP <= 16, "query heads per kv head: at most 16");
-  static_assert(kQ % 1024 == 0 && kP % 1024 == 0 && kPBuf % 1024 == 0 && (NB * 128) % 1024 == 0,
+  static_assert(kK % 1024 == 0 && kQ % 1024 == 0 && kP % 1024 == 0 && kPBuf % 1024 == 0 &&
+                    (NB * 128) % 1024 == 0 && kHalfBytes % 1024 == 0,
                 "swizzled operand tiles start on 1024-byte boundaries");
+  // the merge of the splits stages (m, l) of every split of the group in the
+  // (then idle) V ring
+  static_assert(kK >= kTcMaxSplits * 16 * 8, "the V ring holds (m, l) of every split of a 16-head group");
   static_assert(kAlloc <= 227 * 1024, "shared memory");
 };
+
+// one ring slot: kCB boxes of 64 columns x the slot's keys, from key row `row`
+template <int kCB>
+__device__ __forceinline__ void dec_tile_load(uint8_t* dst, int blk_bytes, int bytes, const CUtensorMap* map,
+                                              uint64_t* full, int hkv, int row, int b) {
+  mbar_arrive_expect_tx(full, bytes);
+#pragma unroll
+  for (int cb = 0; cb < kCB; ++cb) tma_load_4d(dst + cb * blk_bytes, map, full, cb * 64, hkv, row, b);
+}
 
 // byte offset of element (row, col) of a K-major operand tile stored as
 // 64-column blocks of rows x 128 bytes with the 128-byte swizzle
@@ -95,7 +120,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const DecodeParams p) {
   using L = DecodeTcShape<D, GP, ROT>;
-  constexpr int NS = L::kStages;
+  constexpr int NK = L::kKSlots;
+  constexpr int NVH = L::kVHalves;
   constexpr int NB = L::NB;
   constexpr int kCB = D / 64;
   constexpr uint32_t kIdescQK = idesc_bf16_f32(kTcKeys, NB, false, false);
@@ -109,12 +135,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint8_t* sP = smem + L::kP;
   float* red = reinterpret_cast<float*>(smem + L::kRed);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  uint64_t* kfull = bars;            // [NS] K tile landed
-  uint64_t* rot = kfull + NS;        // [NS] remote keys of the K tile rotated
-  uint64_t* kempty = rot + NS;       // [NS] K tile read by its QK
-  uint64_t* vfull = kempty + NS;     // [NS] V tile landed
-  uint64_t* vempty = vfull + NS;     // [NS] V tile read by its PV
-  uint64_t* s_full = vempty + NS;    // [2]
+  uint64_t* kfull = bars;            // [NK] K tile landed
+  uint64_t* rot = kfull + NK;        // [NK] remote keys of the K tile rotated
+  uint64_t* kempty = rot + NK;       // [NK] K tile read by its QK
+  uint64_t* vfull = kempty + NK;     // [NVH] V half landed
+  uint64_t* vempty = vfull + NVH;    // [NVH] V half read by its PV MMAs
+  uint64_t* s_full = vempty + NVH;   // [2]
   uint64_t* s_free = s_full + 2;     // [2]
   uint64_t* p_full = s_free + 2;     // [2]
   uint64_t* pv_done = p_full + 2;    // [2]
@@ -140,10 +166,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int nrot = kr_end > kb ? (kr_end - kb + kTcKeys - 1) / kTcKeys : 0;
 
   if (tid == 0) {
-    for (int i = 0; i < NS; ++i) {
+    for (int i = 0; i < NK; ++i) {
       mbar_init(kfull + i, 1);
       mbar_init(rot + i, kTcRotThreads);
       mbar_init(kempty + i, 1);
+    }
+    for (int i = 0; i < NVH; ++i) {
       mbar_init(vfull + i, 1);
       mbar_init(vempty + i, 1);
     }
@@ -167,10 +195,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   for (int i = tid; i < (L::kQBytes + 2 * L::kPBuf) / 16; i += kTcThreads)
     reinterpret_cast<uint4*>(sQ)[i] = make_uint4(0u, 0u, 0u, 0u);
   __syncthreads();
-  for (int i = tid; i < grp * (D / 2); i += kTcThreads) {
+  // the query words of this thread's staging items (at most two: GP <= 16)
+  constexpr int kQItems = (GP * (D / 2) + kTcThreads - 1) / kTcThreads;
+  uint32_t qw[kQItems];
+#pragma unroll
+  for (int u = 0; u < kQItems; ++u) {
+    const int i = tid + u * kTcThreads;
+    if (i < grp * (D / 2)) {
+      const int hq = hkv * grp + i / (D / 2);
+      qw[u] = __ldg(reinterpret_cast<const uint32_t*>(p.q + (static_cast<size_t>(b) * p.Hq + hq) * D) + i % (D / 2));
+    }
+  }
+  // the first loads of both rings need no free slot: issue them now (after
+  // the query loads, which would otherwise queue behind them), so their DRAM
+  // latency overlaps the query staging
+  const int nhalf = 2 * ntile;
+  if (lane == 0 && warp == kTcWarpTmaK) {
+    tma_prefetch_desc(&tmK);
+    for (int t = 0; t < min(NK, ntile); ++t)
+      dec_tile_load<kCB>(smem + L::kK + (t % NK) * L::kTileBytes, L::kBlk, L::kTileBytes, &tmK, kfull + t % NK,
+                         hkv, kb + t * kTcKeys, b);
+  } else if (lane == 0 && warp == kTcWarpTmaV) {
+    tma_prefetch_desc(&tmV);
+    for (int j = 0; j < min(NVH, nhalf); ++j)
+      dec_tile_load<kCB>(smem + L::kV + (j % NVH) * L::kHalfBytes, L::kBlkH, L::kHalfBytes, &tmV, vfull + j % NVH,
+                         hkv, kb + j * L::kHalfKeys, b);
+  }
+#pragma unroll
+  for (int u = 0; u < kQItems; ++u) {
+    const int i = tid + u * kTcThreads;
+    if (i >= grp * (D / 2)) continue;
     const int gi = i / (D / 2), pr = i % (D / 2);
-    const int hq = hkv * grp + gi;
-    const uint32_t xw = __ldg(reinterpret_cast<const uint32_t*>(p.q + (static_cast<size_t>(b) * p.Hq + hq) * D) + pr);
+    const uint32_t xw = qw[u];
     const float x0 = bf16lo(xw), x1 = bf16hi(xw);
     uint32_t yl = xw;
     if (p.m.kind != kNope) {
@@ -206,23 +262,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (warp == kTcWarpTmaK || warp == kTcWarpTmaV) {
     // -------------------------------------------------------- TMA producers
-    // K and V tiles stream through rings of their own: a K slot is free once
-    // its QK has read it, a V slot once its PV has, so K tiles run ahead of
-    // the rotation and the values of a tile are fetched while it is scored
+    // K tiles and V halves stream through rings of their own: a K slot is
+    // free once its QK has read it, a V half once its PV MMAs have, so K
+    // tiles run ahead of the rotation and the values of a tile are fetched
+    // while it is scored
     if (lane == 0) {
-      const bool is_k = warp == kTcWarpTmaK;
-      const CUtensorMap* map = is_k ? &tmK : &tmV;
-      uint64_t* fullb = is_k ? kfull : vfull;
-      uint64_t* emptyb = is_k ? kempty : vempty;
-      uint8_t* ring = smem + (is_k ? L::kK : L::kV);
-      tma_prefetch_desc(map);
-      for (int t = 0; t < ntile; ++t) {
-        const int s = t % NS;
-        if (t >= NS && !mbar_wait(emptyb + s, ((t / NS) - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(fullb + s, L::kTileBytes);
-        uint8_t* dst = ring + s * L::kTileBytes;
-        const int row = kb + t * kTcKeys;
-        for (int cb = 0; cb < kCB; ++cb) tma_load_4d(dst + cb * L::kBlk, map, fullb + s, cb * 64, hkv, row, b);
+      if (warp == kTcWarpTmaK) {
+        for (int t = NK; t < ntile; ++t) {
+          if (!mbar_wait(kempty + t % NK, ((t / NK) - 1) & 1, abort_flag)) break;
+          dec_tile_load<kCB>(smem + L::kK + (t % NK) * L::kTileBytes, L::kBlk, L::kTileBytes, &tmK, kfull + t % NK,
+                             hkv, kb + t * kTcKeys, b);
+        }
+      } else {
+        for (int j = NVH; j < nhalf; ++j) {
+          if (!mbar_wait(vempty + j % NVH, ((j / NVH) - 1) & 1, abort_flag)) break;
+          dec_tile_load<kCB>(smem + L::kV + (j % NVH) * L::kHalfBytes, L::kBlkH, L::kHalfBytes, &tmV, vfull + j % NVH,
+                             hkv, kb + j * L::kHalfKeys, b);
+        }
       }
     }
   } else if (warp == kTcWarpQK) {
@@ -230,8 +286,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0) {
       const uint32_t qaddr = smem_u32(sQ);
       for (int t = 0; t < ntile; ++t) {
-        const int s = t % NS;
-        if (!mbar_wait(t < nrot ? rot + s : kfull + s, (t / NS) & 1, abort_flag)) break;
+        const int s = t % NK;
+        if (!mbar_wait(t < nrot ? rot + s : kfull + s, (t / NK) & 1, abort_flag)) break;
         if (t >= 2 && !mbar_wait(s_free + (t & 1), ((t >> 1) - 1) & 1, abort_flag)) break;
         tc_fence_after();
         const uint32_t kaddr = smem_u32(smem + L::kK + s * L::kTileBytes);
@@ -249,23 +305,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ------------------------------------------------------ MMA: O^T += V^T P^T
     if (lane == 0) {
       for (int t = 0; t < ntile; ++t) {
-        const int s = t % NS;
-        if (!mbar_wait(vfull + s, (t / NS) & 1, abort_flag)) break;
         if (!mbar_wait(p_full + (t & 1), (t >> 1) & 1, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t vaddr = smem_u32(smem + L::kV + s * L::kTileBytes);
         const uint32_t paddr = smem_u32(sP + (t & 1) * L::kPBuf);
-        // M = 128 output dimensions: for D = 64 the upper 64 rows read the 16 KiB
-        // that follow the V tile (the next slot, or the K ring) and land in
-        // TMEM lanes nobody reads
+        bool okv = true;
 #pragma unroll
-        for (int kk = 0; kk < kTcKeys / 16; ++kk) {
-          umma_ss(tO, sdesc_sw128(vaddr + kk * 2048, L::kBlk, 1024),
-                  sdesc_sw128(paddr + (kk >> 2) * (kTcNP * 128) + (kk & 3) * 32, 16, 1024), kIdescPV,
-                  (t > 0 || kk > 0) ? 1u : 0u);
+        for (int h = 0; h < 2; ++h) {
+          const int j = 2 * t + h;
+          const int s = j % NVH;
+          if (!mbar_wait(vfull + s, (j / NVH) & 1, abort_flag)) { okv = false; break; }
+          tc_fence_after();
+          const uint32_t vaddr = smem_u32(smem + L::kV + s * L::kHalfBytes);
+          // M = 128 output dimensions: for D = 64 the upper 64 rows read the
+          // 8 KiB that follow the V half (the next half, or the K ring) and
+          // land in TMEM lanes nobody reads
+#pragma unroll
+          for (int kq = 0; kq < L::kHalfKeys / 16; ++kq) {
+            const int kk = h * (L::kHalfKeys / 16) + kq;
+            umma_ss(tO, sdesc_sw128(vaddr + kq * 2048, L::kBlkH, 1024),
+                    sdesc_sw128(paddr + (kk >> 2) * (kTcNP * 128) + (kk & 3) * 32, 16, 1024), kIdescPV,
+                    (t > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(vempty + s);
         }
+        if (!okv) break;
         umma_commit(pv_done + (t & 1));
-        umma_commit(vempty + s);
       }
     }
   } else if (warp >= 4) {
@@ -377,8 +440,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       };
       for (int t = 0; t < nrot; ++t) {
-        const int s = t % NS;
-        if (!__all_sync(0xffffffffu, mbar_wait(kfull + s, (t / NS) & 1, abort_flag))) break;
+        const int s = t % NK;
+        if (!__all_sync(0xffffffffu, mbar_wait(kfull + s, (t / NK) & 1, abort_flag))) break;
         if (t % kTcReseed == 0) seed();
         uint8_t* kt = smem + L::kK + s * L::kTileBytes + (c >> 3) * L::kBlk;
         const int k0 = kb + t * kTcKeys;
@@ -551,26 +614,41 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
   __syncthreads();
   if (*last_flag) {
-    // last CTA of this (batch, kv head): merge every split, in split order
+    // last CTA of this (batch, kv head): merge every split, in split order.
+    // The (m, l) of all splits of the group are staged in the idle V ring
+    // and turned into the weights exp2(m_s - M) once, so each output element
+    // is one pass of independent loads over the splits
     __threadfence();
+    const int ns = p.nsplit;
+    float2* wml = reinterpret_cast<float2*>(smem + L::kV);   // [grp][ns] (m, l), then (weight, 0)
+    float* wtot = reinterpret_cast<float*>(smem + L::kK);   // [grp] (M, L), in the idle K ring
+    const size_t gbase = (static_cast<size_t>(b) * p.Hq + hkv * grp) * ns;
+    for (int i = tid; i < grp * ns; i += kTcThreads) wml[i] = __ldcg(p.part_ml + gbase + i);
+    __syncthreads();
+    if (tid < grp) {
+      float2* w = wml + tid * ns;
+      float M = -INFINITY;
+      for (int sp = 0; sp < ns; ++sp)
+        if (w[sp].y > 0.f) M = fmaxf(M, w[sp].x);
+      float l = 0.f;
+      for (int sp = 0; sp < ns; ++sp) {
+        const float f = w[sp].y > 0.f ? ex2(w[sp].x - M) : 0.f;
+        l = fmaf(w[sp].y, f, l);
+        w[sp].x = f;
+      }
+      wtot[2 * tid] = M;
+      wtot[2 * tid + 1] = l;
+    }
+    __syncthreads();
     for (int idx = tid; idx < grp * D; idx += kTcThreads) {
       const int gi = idx / D, d = idx % D;
+      const float2* w = wml + gi * ns;
+      const float* po = p.part_o + (gbase + static_cast<size_t>(gi) * ns) * D + d;
+      float o = 0.f;
+#pragma unroll 8
+      for (int sp = 0; sp < ns; ++sp) o = fmaf(__ldcg(po + static_cast<size_t>(sp) * D), w[sp].x, o);
       const int hq = hkv * grp + gi;
-      const size_t base = (static_cast<size_t>(b) * p.Hq + hq) * p.nsplit;
-      float M = -INFINITY;
-      for (int sp = 0; sp < p.nsplit; ++sp) {
-        const float2 ml = __ldcg(p.part_ml + base + sp);
-        if (ml.y > 0.f) M = fmaxf(M, ml.x);
-      }
-      float o = 0.f, l = 0.f;
-      for (int sp = 0; sp < p.nsplit; ++sp) {
-        const float2 ml = __ldcg(p.part_ml + base + sp);
-        if (ml.y > 0.f) {
-          const float f = ex2(ml.x - M);
-          o = fmaf(__ldcg(p.part_o + (base + sp) * D + d), f, o);
-          l = fmaf(ml.y, f, l);
-        }
-      }
+      const float M = wtot[2 * gi], l = wtot[2 * gi + 1];
       p.out[(static_cast<size_t>(b) * p.Hq + hq) * D + d] = o / l;
       if (d == 0) p.lse[static_cast<size_t>(b) * p.Hq + hq] = (M + __log2f(l)) * 0.69314718055994530942f;
     }

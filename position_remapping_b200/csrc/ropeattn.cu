@@ -312,6 +312,7 @@ struct DecodeLayout {
 int decode_nsplit(long long B, long long keys, int Hkv) {
   long long want = static_cast<long long>(sm_count()) / (Hkv * B);
   long long cap = (keys + 255) / 256;
+  if (cap > kTcMaxSplits) cap = kTcMaxSplits;   // the merge stages every split's (m, l) on chip
   long long ns = want < cap ? want : cap;
   return static_cast<int>(ns < 1 ? 1 : ns);
 }
@@ -929,9 +930,10 @@ int ropeattn_decode_cache(const void* q, const void* k_cache, const void* v_cach
 
   CUtensorMap tk, tv;
   if (tc) {
-    // 128-key tiles in 64-column blocks with the 128-byte swizzle (tcgen05 operands)
+    // 64-column blocks with the 128-byte swizzle (tcgen05 operands): K in
+    // 128-key tiles, V in 64-key halves
     if ((rc = make_map(&tk, k_cache, D, Hkv, n, B, 64, kTcKeys, true, cache_len))) return rc;
-    if ((rc = make_map(&tv, v_cache, D, Hkv, n, B, 64, kTcKeys, true, cache_len))) return rc;
+    if ((rc = make_map(&tv, v_cache, D, Hkv, n, B, 64, kTcKeys / 2, true, cache_len))) return rc;
   } else {
     if ((rc = make_map(&tk, k_cache, D, Hkv, n, B, D, kDecKeys, false, cache_len))) return rc;
     if ((rc = make_map(&tv, v_cache, D, Hkv, n, B, D, kDecKeys, false, cache_len))) return rc;
