@@ -31,7 +31,7 @@ What it computes, and where each step is defined:
 * The literal three-call inclusion-exclusion merge: Jet-Long, §3.3 Eq. 7
   (kept as a self-check; the routed softmax is the definition it reaches).
 
-Readings where the pages leave a step open (each listed in the design notes):
+Readings where the pages leave a step open:
 adjacent pairing (2i, 2i+1); natural-log LSE of the scaled scores; the local
 set of the bifocal score is 0 <= q-k <= w0 inclusive; for prefill L = S; for
 decode L = n, the cache length including the current token at n-1.
