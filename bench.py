@@ -507,6 +507,9 @@ def config_dict(n_gpus):
 # ----------------------------------------------------------------------------
 # GPU arm
 # ----------------------------------------------------------------------------
+CONFIG_PROFILES = ("standard_s512", "endprompt_s8192", "periodic_s32768", "nope_s32768")
+
+
 def run_profile_case(which: str):
     """Capture-sized cases for ncu (a few GB on the device at most, inputs
     still larger than L2). prefill: the 131072-token workload's kernel on a
@@ -514,7 +517,8 @@ def run_profile_case(which: str):
     prefill256: the same case at head_dim 256; decode: the full 131072-key
     decode (512 MiB of cache); backward: the backward of the 32768-token
     case (G = 4); prefill131072: the full-size attention, for one-pass
-    counters only."""
+    counters only; standard_s512, endprompt_s8192, periodic_s32768,
+    nope_s32768: those workloads at full size (under 2 GB each)."""
     from position_remapping_b200 import ropeattn as ra
     dev = torch.device("cuda", 0)
     if which == "prefill131072":
@@ -539,6 +543,15 @@ def run_profile_case(which: str):
                          device=dev)
         for _ in range(3):
             ra.prefill_backward(q, k, v, out, lse, dout, params, workspace=ws)
+    elif which in CONFIG_PROFILES:
+        w = WORKLOADS[which]
+        q, k, v = make_qkv(w.B, w.S, w.Hq, w.Hkv, w.D, w.seed, device=dev)
+        out = torch.empty((w.B, w.S, w.Hq, w.D), dtype=torch.float32, device=dev)
+        lse = torch.empty((w.B, w.Hq, w.S), dtype=torch.float32, device=dev)
+        ws = torch.empty(max(1, ra.prefill_workspace_size(w.params, w.B, w.S, w.Hq, w.Hkv, w.D)), dtype=torch.uint8,
+                         device=dev)
+        for _ in range(3):
+            ra.prefill(q, k, v, w.params, out=out, lse=lse, workspace=ws)
     elif which in ("prefill", "prefill256"):
         P = PREFILL
         S = 32768
@@ -566,7 +579,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["prefill", "prefill131072", "prefill256", "decode", "backward"], default=None,
+    ap.add_argument("--profile", choices=["prefill", "prefill131072", "prefill256", "decode", "backward",
+                                          *CONFIG_PROFILES], default=None,
                     help="run a capture-sized case of one kernel three times (for ncu); no timing, no JSON")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
