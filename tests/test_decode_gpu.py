@@ -42,6 +42,14 @@ SMALL = [
     ("d256_bifocal_g3_grp2", 2, 5000, 4, 2, 256, MapParams(O.BIFOCAL, rope_base=1e6, w0=400, w_pretrained=2000)),
     ("d256_periodic", 1, 2500, 2, 2, 256, MapParams(O.PERIODIC, rope_base=1e4, window=512)),
     ("d256_bifocal_grp1", 1, 4097, 2, 2, 256, MapParams(O.BIFOCAL, rope_base=1e4, w0=100, w_pretrained=1024)),
+    # long key ranges per split (8 kv heads: 18 splits on 148 SMs, 12-19
+    # tiles each), so the K-tile ring and the V-half ring wrap many times
+    # at both head dims and the phasor is re-seeded mid-split
+    ("long_bifocal_d128_grp2", 1, 40000, 16, 8, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=2048, w_pretrained=12000)),
+    ("long_bifocal_d64_grp8_g3", 1, 40000, 64, 8, 64, MapParams(O.BIFOCAL, rope_base=1e4, w0=500, w_pretrained=15000)),
+    ("long_standard_d64_grp16", 1, 30001, 128, 8, 64, MapParams(O.STANDARD, rope_base=1e4)),
+    ("long_periodic_d128_grp4", 1, 33000, 32, 8, 128, MapParams(O.PERIODIC, rope_base=1e4, window=30000)),
+    ("long_bifocal_b2_d128_grp4", 2, 20000, 32, 8, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=700, w_pretrained=6000)),
 ]
 
 
