@@ -426,6 +426,79 @@ def measure_configs(ra, peaks, stream, with_oracle: bool):
             **res}
 
 
+def measure_variants(ra, peaks, q, k, v, kd, vd, stream):
+    """The variants of the method beside the main path, each alone with CUDA
+    events: prefill at 32768 tokens (bifocal, 32/8 heads, G = 4 via
+    w_pretrained 8192) with adjacent and half-split pairing, a fixed group
+    size and head_dim 256; decode of the 131072-key bifocal cache at
+    head_dim 64 and 256, GQA groups 8 and 16, and half-split pairing.
+    Inputs are leading slices of the resident tensors, or seeded N(0, 1)
+    draws on the device where a shape differs (the kernels do no
+    data-dependent work)."""
+    dev = q.device
+    tpeak = float(peaks.get("bf16_tflops", 1590.0))
+    hpeak = float(peaks.get("hbm_gbs", 6650.0))
+    P, Dd = PREFILL, DECODE
+    gen = torch.Generator(device=dev).manual_seed(20261)
+
+    def draw(*shape):
+        return torch.randn(*shape, generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
+
+    S = 32768
+    base = P.params.replace(w_pretrained=8192)
+    pre = {}
+    pairs = S * (S + 1) // 2
+    cases = [("bifocal_s32768_d128", 128, base), ("bifocal_s32768_half_split", 128, base.replace(pairing=1)),
+             ("bifocal_s32768_fixed_g4", 128, base.replace(fixed_group=4)), ("bifocal_s32768_d256", 256, base)]
+    for name, D, prm in cases:
+        if D == P.D:
+            qs, ks, vs = q[:, :S], k[:, :S], v[:, :S]
+        else:
+            qs, ks, vs = draw(P.B, S, P.Hq, D), draw(P.B, S, P.Hkv, D), draw(P.B, S, P.Hkv, D)
+        out = torch.empty((P.B, S, P.Hq, D), dtype=torch.float32, device=dev)
+        lse = torch.empty((P.B, P.Hq, S), dtype=torch.float32, device=dev)
+        ws = torch.empty(ra.prefill_workspace_size(prm, P.B, S, P.Hq, P.Hkv, D), dtype=torch.uint8, device=dev)
+        # two rounds, the faster kept: the first launches after other work
+        # run at whatever clock that work left
+        ms = min(_event_ms(lambda: ra.prefill(qs, ks, vs, prm, out=out, lse=lse, workspace=ws, stream=stream), 5,
+                           stream) for _ in range(2))
+        tf = 4.0 * D * pairs * P.B * P.Hq / (ms / 1e3) / 1e12
+        pre[name] = {"ms": ms, "tflops": tf, "tensor_frac": tf / tpeak, "D": D, "pairing": prm.pairing,
+                     "fixed_group": prm.fixed_group}
+        del qs, ks, vs, out, lse, ws
+    for name in pre:
+        pre[name]["time_vs_d128_adjacent"] = pre[name]["ms"] / pre["bifocal_s32768_d128"]["ms"]
+    dec = {}
+    n = Dd.S
+    dcases = [("bifocal_n131072_d128_grp2", 128, 16, Dd.params), ("bifocal_n131072_half_split", 128, 16,
+                                                                     Dd.params.replace(pairing=1)),
+              ("bifocal_n131072_d128_grp8", 128, 64, Dd.params), ("bifocal_n131072_d128_grp16", 128, 128, Dd.params),
+              ("bifocal_n131072_d64_grp2", 64, 16, Dd.params), ("bifocal_n131072_d256_grp2", 256, 16, Dd.params)]
+    for name, D, Hq, prm in dcases:
+        if D == Dd.D:
+            kc, vc = kd, vd
+        else:
+            kc, vc = draw(Dd.B, n, Dd.Hkv, D), draw(Dd.B, n, Dd.Hkv, D)
+        qq = draw(Dd.B, Hq, D)
+        od = torch.empty((Dd.B, Hq, D), dtype=torch.float32, device=dev)
+        ld = torch.empty((Dd.B, Hq), dtype=torch.float32, device=dev)
+        wsd = torch.empty(ra.decode_workspace_size(Dd.B, n, Hq, Dd.Hkv, D), dtype=torch.uint8, device=dev)
+        us = 1e3 * _event_ms(lambda: ra.decode(qq, kc, vc, prm, out=od, lse=ld, workspace=wsd, stream=stream),
+                             100, stream)
+        byts = 2 * Dd.B * n * Dd.Hkv * D * 2
+        dec[name] = {"us": us, "gbs": byts / (us / 1e6) / 1e9, "hbm_frac": byts / (us / 1e6) / 1e9 / hpeak,
+                     "kv_bytes": byts, "D": D, "Hq": Hq, "Hkv": Dd.Hkv, "pairing": prm.pairing,
+                     "kernel": "decode_tc_kernel" if D <= 128 else "decode_kernel (CUDA cores)"}
+        del qq, od, ld, wsd
+        if D != Dd.D:
+            del kc, vc
+    ra.status()
+    return {"note": "each alone, CUDA events (prefill: pre-pass + attention, the faster of two rounds of 5 calls; "
+                    "decode: 100 calls back to "
+                    "back, host cost included where it exceeds the kernel); tensor_frac vs the burst bf16 peak, "
+                    "hbm_frac vs the measured copy bandwidth", "prefill": pre, "decode": dec}
+
+
 def measure_sweep(ra, q, k, v, qd, kd, vd, ws, wsd, stream):
     """Bifocal against standard RoPE over the Jet-Long Table 7 lengths (4K to
     128K; w_pretrained 32768, so G = 1 up to 32K and the bifocal map is the
@@ -734,6 +807,7 @@ def main():
     comparators.update(measure_decode_comparators(ra, qd, kd, vd, stream))
     sweep = measure_sweep(ra, q, k, v, qd, kd, vd, ws, wsd, stream)
     peaks0, _ = load_peaks()
+    variants = measure_variants(ra, peaks0, q, k, v, kd, vd, stream)
     backward = measure_backward(ra, q, k, v, out, lse, peaks0, stream)
     configs = measure_configs(ra, peaks0, stream, with_oracle=(world == 1 and not args.no_cpu_baseline))
 
@@ -798,6 +872,7 @@ def main():
         "comparators": comparators,
         "backward": backward,
         "length_sweep": sweep,
+        "variants": variants,
         "configs": configs,
         "e2e": {"value": job_tflops(world, flops, K, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
