@@ -488,7 +488,7 @@ def measure_variants(ra, peaks, q, k, v, kd, vd, stream):
         byts = 2 * Dd.B * n * Dd.Hkv * D * 2
         dec[name] = {"us": us, "gbs": byts / (us / 1e6) / 1e9, "hbm_frac": byts / (us / 1e6) / 1e9 / hpeak,
                      "kv_bytes": byts, "D": D, "Hq": Hq, "Hkv": Dd.Hkv, "pairing": prm.pairing,
-                     "kernel": "decode_tc_kernel" if D <= 128 else "decode_kernel (CUDA cores)"}
+                     "kernel": "decode_tc_kernel"}
         del qq, od, ld, wsd
         if D != Dd.D:
             del kc, vc

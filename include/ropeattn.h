@@ -26,8 +26,8 @@
  *   GQA: query head h reads key/value head h / (Hq / Hkv).
  *   Supported: D in {64, 128, 256} (the prefill runs D = 256 with one
  *   128-row query tile per CTA and 64-key tiles);
- *   Hq % Hkv == 0; decode also needs Hq / Hkv <= 16 for D = 64 and 128
- *   and Hq / Hkv <= 2 for D = 256; the backward needs D = 64 or 128.
+ *   Hq % Hkv == 0; decode also needs Hq / Hkv <= 16; the backward needs
+ *   D = 64 or 128.
  *   Half-split pairing (params.pairing = ROPEATTN_PAIR_HALF): q, k and v are
  *   given in their own order; the rotation pairs coordinates (i, i + D/2),
  *   and key caches hold each rotated key in adjacent order instead (element

@@ -1,5 +1,5 @@
 // One decode step over an untouched RoPE key cache (Jet-Long §3.2) on the
-// fifth-generation tensor cores, sm_100a, for head_dim 64 and 128.
+// fifth-generation tensor cores, sm_100a, for head_dim 64, 128 and 256.
 //
 // Split-KV: CTA (split, kv head, batch) owns a contiguous key range of one kv
 // head; the grid is one wave. The range streams through shared memory by TMA
@@ -66,9 +66,12 @@ struct DecodeTcShape {
   // half from its load through its PV MMAs. Each ring must cover the DRAM
   // latency under load (~4000 cycles) plus that work at the HBM rate, with
   // the SM clock as low as the power cap takes it: four K tiles and five V
-  // halves at head_dim 128 (208 KiB), seven and twelve at 64.
-  static constexpr int kKSlots = D == 128 ? 4 : 7;           // K ring: whole tiles
-  static constexpr int kVHalves = D == 128 ? 5 : 12;         // V ring: 64-key halves
+  // halves at head_dim 128 (208 KiB), seven and twelve at 64; at 256 a tile
+  // carries twice the bytes (so twice the time at the HBM rate) and two K
+  // tiles and two V halves fill the same space (192 KiB).
+  static constexpr int kKSlots = D == 256 ? 2 : (D == 128 ? 4 : 7);      // K ring: whole tiles
+  static constexpr int kVHalves = D == 256 ? 2 : (D == 128 ? 5 : 12);    // V ring: 64-key halves
+  static constexpr int kMB = D > 128 ? D / 128 : 1;          // O^T blocks of 128 output dimensions
   static constexpr int kHalfKeys = kTcKeys / 2;
   static constexpr int kBlk = kTcKeys * 128;                 // one 64-column swizzle block of a K tile
   static constexpr int kBlkH = kHalfKeys * 128;              // the same block of a V half
@@ -88,7 +91,7 @@ struct DecodeTcShape {
   static constexpr int kMisc = kBar + kNumBars * 8;          // tmem base, abort flag, last flag
   static constexpr int kTotal = kMisc + 16;
   static constexpr int kAlloc = kTotal + 1024;               // slack to align the base to 1024
-  static constexpr uint32_t kTmemCols = (2 * NB + kTcNP) <= 64 ? 64 : 128;
+  static constexpr uint32_t kTmemCols = (2 * NB + kMB * kTcNP) <= 64 ? 64 : 128;
   static_assert(GP <= 16, "query heads per kv head: at most 16");
   static_assert(kK % 1024 == 0 && kQ % 1024 == 0 && kP % 1024 == 0 && kPBuf % 1024 == 0 &&
                     (NB * 128) % 1024 == 0 && kHalfBytes % 1024 == 0,
@@ -123,6 +126,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   constexpr int NK = L::kKSlots;
   constexpr int NVH = L::kVHalves;
   constexpr int NB = L::NB;
+  constexpr int kMB = L::kMB;
   constexpr int kCB = D / 64;
   constexpr uint32_t kIdescQK = idesc_bf16_f32(kTcKeys, NB, false, false);
   constexpr uint32_t kIdescPV = idesc_bf16_f32(128, kTcNP, false, true);   // A = V^T read MN-major
@@ -249,7 +253,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tS = tmem;              // S^T buffers at [0, NB) and [NB, 2 NB)
-  const uint32_t tO = tmem + 2 * NB;     // O^T, kTcNP columns
+  const uint32_t tO = tmem + 2 * NB;     // O^T, kTcNP columns per block of 128 dimensions
 
   float l_fin[GP];                      // softmax threads: per-thread sums, reduced at the end
   float m_fin[GP];
@@ -258,7 +262,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     l_fin[gi] = 0.f;
     m_fin[gi] = -INFINITY;
   }
-  uint32_t o_fin[kTcNP];
+  uint32_t o_fin[kMB][kTcNP];
 
   if (warp == kTcWarpTmaK || warp == kTcWarpTmaV) {
     // -------------------------------------------------------- TMA producers
@@ -315,16 +319,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (!mbar_wait(vfull + s, (j / NVH) & 1, abort_flag)) { okv = false; break; }
           tc_fence_after();
           const uint32_t vaddr = smem_u32(smem + L::kV + s * L::kHalfBytes);
-          // M = 128 output dimensions: for D = 64 the upper 64 rows read the
-          // 8 KiB that follow the V half (the next half, or the K ring) and
-          // land in TMEM lanes nobody reads
+          // M = 128 output dimensions per MMA (two 64-column blocks of the
+          // half, one O^T block); for D = 64 the upper 64 rows read the 8 KiB
+          // that follow the V half (the next half, or the K ring) and land in
+          // TMEM lanes nobody reads
 #pragma unroll
-          for (int kq = 0; kq < L::kHalfKeys / 16; ++kq) {
-            const int kk = h * (L::kHalfKeys / 16) + kq;
-            umma_ss(tO, sdesc_sw128(vaddr + kq * 2048, L::kBlkH, 1024),
-                    sdesc_sw128(paddr + (kk >> 2) * (kTcNP * 128) + (kk & 3) * 32, 16, 1024), kIdescPV,
-                    (t > 0 || kk > 0) ? 1u : 0u);
-          }
+          for (int mb = 0; mb < kMB; ++mb)
+#pragma unroll
+            for (int kq = 0; kq < L::kHalfKeys / 16; ++kq) {
+              const int kk = h * (L::kHalfKeys / 16) + kq;
+              umma_ss(tO + mb * kTcNP, sdesc_sw128(vaddr + 2 * mb * L::kBlkH + kq * 2048, L::kBlkH, 1024),
+                      sdesc_sw128(paddr + (kk >> 2) * (kTcNP * 128) + (kk & 3) * 32, 16, 1024), kIdescPV,
+                      (t > 0 || kk > 0) ? 1u : 0u);
+            }
           umma_commit(vempty + s);
         }
         if (!okv) break;
@@ -539,12 +546,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // rescale O^T (lane r = output dimension r) once PV(t-1) has completed
         if (!wwait(pv_done + ((t - 1) & 1), ((t - 1) >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
-        uint32_t o[kTcNP];
-        tmem_ld16(tO + lane_off, o);
-        tmem_ld_wait();
 #pragma unroll
-        for (int gi = 0; gi < GP; ++gi) o[gi] = __float_as_uint(__uint_as_float(o[gi]) * corr[gi]);
-        tmem_st16(tO + lane_off, o);
+        for (int mb = 0; mb < kMB; ++mb) {
+          uint32_t o[kTcNP];
+          tmem_ld16(tO + mb * kTcNP + lane_off, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int gi = 0; gi < GP; ++gi) o[gi] = __float_as_uint(__uint_as_float(o[gi]) * corr[gi]);
+          tmem_st16(tO + mb * kTcNP + lane_off, o);
+        }
         tmem_st_wait();
       }
       uint8_t* pbuf = sP + (t & 1) * L::kPBuf;
@@ -555,15 +565,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_before();
       mbar_arrive(p_full + (t & 1));
     }
-    // the last PV has completed: O^T row r holds this split's unnormalised
-    // output of dimension r for every head of the group
+    // the last PV has completed: row r of O^T block mb holds this split's
+    // unnormalised output of dimension 128 mb + r for every head of the group
     if (ok && ntile > 0 && wwait(pv_done + ((ntile - 1) & 1), ((ntile - 1) >> 1) & 1)) {
       tc_fence_after();
-      tmem_ld16(tO + lane_off, o_fin);
+#pragma unroll
+      for (int mb = 0; mb < kMB; ++mb) tmem_ld16(tO + mb * kTcNP + lane_off, o_fin[mb]);
       tmem_ld_wait();
     } else {
 #pragma unroll
-      for (int i = 0; i < kTcNP; ++i) o_fin[i] = 0u;
+      for (int mb = 0; mb < kMB; ++mb)
+#pragma unroll
+        for (int i = 0; i < kTcNP; ++i) o_fin[mb][i] = 0u;
     }
 #pragma unroll
     for (int gi = 0; gi < GP; ++gi) {
@@ -587,13 +600,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (warp == 0) lsum[4 * GP + gi] = m_fin[gi];   // the reference max, the same in every thread
       }
     }
-    if (tid < D) {
 #pragma unroll
-      for (int gi = 0; gi < GP; ++gi) {
-        if (gi < grp) {
-          const int hq = hkv * grp + gi;
-          const size_t pslot = (static_cast<size_t>(b) * p.Hq + hq) * p.nsplit + split;
-          p.part_o[pslot * D + tid] = __uint_as_float(o_fin[gi]);
+    for (int mb = 0; mb < kMB; ++mb) {
+      const int d = mb * 128 + tid;
+      if (d < D) {
+#pragma unroll
+        for (int gi = 0; gi < GP; ++gi) {
+          if (gi < grp) {
+            const int hq = hkv * grp + gi;
+            const size_t pslot = (static_cast<size_t>(b) * p.Hq + hq) * p.nsplit + split;
+            p.part_o[pslot * D + d] = __uint_as_float(o_fin[mb][gi]);
+          }
         }
       }
     }

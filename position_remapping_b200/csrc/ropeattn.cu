@@ -329,21 +329,6 @@ DecodeLayout decode_layout(long long B, long long keys, int Hq, int Hkv, int D) 
   return L;
 }
 
-template <int D, int GRP, int ROT>
-int launch_decode_rot(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& dp, dim3 grid,
-                      cudaStream_t st) {
-  using L = DecodeSmem<D>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(decode_kernel<D, GRP, ROT>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal);
-  });
-  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(decode)");
-  decode_kernel<D, GRP, ROT><<<grid, DecodeShape<D, GRP>::kThreads, L::kTotal, st>>>(tk, tv, dp);
-  CUDA_TRY(cudaGetLastError(), "decode launch");
-  return ROPEATTN_OK;
-}
-
 template <int D, int GP, int ROT>
 int launch_decode_tc_rot(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& dp, dim3 grid,
                          cudaStream_t st) {
@@ -371,18 +356,6 @@ int launch_decode_tc(int grp, const CUtensorMap& tk, const CUtensorMap& tv, cons
   if (grp <= 4) return r ? launch_decode_tc_rot<D, 4, 1>(tk, tv, dp, grid, st) : launch_decode_tc_rot<D, 4, 0>(tk, tv, dp, grid, st);
   if (grp <= 8) return r ? launch_decode_tc_rot<D, 8, 1>(tk, tv, dp, grid, st) : launch_decode_tc_rot<D, 8, 0>(tk, tv, dp, grid, st);
   return r ? launch_decode_tc_rot<D, 16, 1>(tk, tv, dp, grid, st) : launch_decode_tc_rot<D, 16, 0>(tk, tv, dp, grid, st);
-}
-
-// Rotation of remote keys: none (no bifocal map), shared per-stage tables
-// when one key per lane group, else (two keys per group) the per-lane
-// phasor recurrence.
-template <int D, int GRP>
-int launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& dp, dim3 grid, cudaStream_t st) {
-  if (!dp.bifocal) return launch_decode_rot<D, GRP, kRotNone>(tk, tv, dp, grid, st);
-  if constexpr (DecodeShape<D, GRP>::kKeysPerGroup == 1) {
-    return launch_decode_rot<D, GRP, kRotTable>(tk, tv, dp, grid, st);
-  }
-  return launch_decode_rot<D, GRP, kRotPhasor>(tk, tv, dp, grid, st);
 }
 
 }  // namespace
@@ -881,8 +854,7 @@ int ropeattn_decode_cache(const void* q, const void* k_cache, const void* v_cach
   if (rc) return rc;
   if (B == 0 || n == 0) return ROPEATTN_OK;
   const int grp = Hq / Hkv;
-  if (!((D == 256 && (grp == 1 || grp == 2)) || (D <= 128 && grp <= 16)))
-    return fail(ROPEATTN_ERR_INVALID_ARG, "decode supports Hq/Hkv <= 16 for D = 64 and 128, and in {1, 2} for D = 256");
+  if (grp > 16) return fail(ROPEATTN_ERR_INVALID_ARG, "decode supports Hq/Hkv <= 16");
   if (!q || !k_cache || !v_cache || !out || !lse) return fail(ROPEATTN_ERR_INVALID_ARG, "null tensor pointer");
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || !aligned16(lse))
     return fail(ROPEATTN_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
@@ -917,9 +889,7 @@ int ropeattn_decode_cache(const void* q, const void* k_cache, const void* v_cach
   dp.Hq = Hq;
   dp.Hkv = Hkv;
   dp.nsplit = lay.nsplit;
-  const bool tc = D <= 128;   // tensor-core decode; D = 256 runs on the CUDA cores
-  const int stage_keys = tc ? kTcKeys : kDecKeys;
-  dp.keys_per_split = static_cast<int>(align_up(static_cast<size_t>((keys + lay.nsplit - 1) / lay.nsplit), stage_keys));
+  dp.keys_per_split = static_cast<int>(align_up(static_cast<size_t>((keys + lay.nsplit - 1) / lay.nsplit), kTcKeys));
   dp.k_begin = static_cast<int>(k_begin);
   dp.bifocal = eff == ROPEATTN_BIFOCAL ? 1 : 0;
   dp.k_local = dp.bifocal ? static_cast<int>(t - m.w0 > 0 ? t - m.w0 : 0) : 0;
@@ -928,19 +898,14 @@ int ropeattn_decode_cache(const void* q, const void* k_cache, const void* v_cach
   dp.scale_log2 = scale_log2(params, D);
   fill_turns(params, D, dp.turns);
 
+  // 64-column blocks with the 128-byte swizzle (tcgen05 operands): K in
+  // 128-key tiles, V in 64-key halves
   CUtensorMap tk, tv;
-  if (tc) {
-    // 64-column blocks with the 128-byte swizzle (tcgen05 operands): K in
-    // 128-key tiles, V in 64-key halves
-    if ((rc = make_map(&tk, k_cache, D, Hkv, n, B, 64, kTcKeys, true, cache_len))) return rc;
-    if ((rc = make_map(&tv, v_cache, D, Hkv, n, B, 64, kTcKeys / 2, true, cache_len))) return rc;
-  } else {
-    if ((rc = make_map(&tk, k_cache, D, Hkv, n, B, D, kDecKeys, false, cache_len))) return rc;
-    if ((rc = make_map(&tv, v_cache, D, Hkv, n, B, D, kDecKeys, false, cache_len))) return rc;
-  }
+  if ((rc = make_map(&tk, k_cache, D, Hkv, n, B, 64, kTcKeys, true, cache_len))) return rc;
+  if ((rc = make_map(&tv, v_cache, D, Hkv, n, B, 64, kTcKeys / 2, true, cache_len))) return rc;
   CUDA_TRY(cudaMemsetAsync(dp.counters, 0, static_cast<size_t>(B) * Hkv * sizeof(int), st), "memset counters");
   dim3 grid(lay.nsplit, Hkv, static_cast<unsigned>(B));
-  if (D == 256) return grp == 1 ? launch_decode<256, 1>(tk, tv, dp, grid, st) : launch_decode<256, 2>(tk, tv, dp, grid, st);
+  if (D == 256) return launch_decode_tc<256>(grp, tk, tv, dp, grid, st);
   if (D == 128) return launch_decode_tc<128>(grp, tk, tv, dp, grid, st);
   return launch_decode_tc<64>(grp, tk, tv, dp, grid, st);
 }

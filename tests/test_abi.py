@@ -98,8 +98,9 @@ def test_host_argument_checks(ra):
     assert lib.ropeattn_prefill_three_call_workspace_size(bif, 1, 4096, 2, 1, 256) > \
         lib.ropeattn_prefill_workspace_size(bif, 1, 4096, 2, 1, 256) > 0
     assert lib.ropeattn_decode_workspace_size(1, 1000, 2, 1, 256) > 0
-    assert lib.ropeattn_decode(nullp, nullp, nullp, nullp, nullp, 1, 1000, 8, 1, 256,
-                               ctypes.byref(cp(_p(kind=STANDARD))), nullp, 0, nullp) == ra.ERR_INVALID_ARG  # GQA 8
+    assert lib.ropeattn_decode(nullp, nullp, nullp, nullp, nullp, 1, 1000, 32, 1, 256,
+                               ctypes.byref(cp(_p(kind=STANDARD))), nullp, 0, nullp) == ra.ERR_INVALID_ARG  # GQA 32
+    assert "16" in lib.ropeattn_last_error().decode()
     bad = [_p(kind=9), _p(kind=PERIODIC, window=0), _p(kind=BIFOCAL, w0=-1, w_pretrained=8),
            _p(kind=BIFOCAL, w0=4, w_pretrained=0), _p(kind=ENDPROMPT, interp=0.5),
            _p(kind=STANDARD, rope_base=1.0), _p(kind=STANDARD, softmax_scale=-1.0),

@@ -50,6 +50,11 @@ SMALL = [
     ("long_standard_d64_grp16", 1, 30001, 128, 8, 64, MapParams(O.STANDARD, rope_base=1e4)),
     ("long_periodic_d128_grp4", 1, 33000, 32, 8, 128, MapParams(O.PERIODIC, rope_base=1e4, window=30000)),
     ("long_bifocal_b2_d128_grp4", 2, 20000, 32, 8, 128, MapParams(O.BIFOCAL, rope_base=1e6, w0=700, w_pretrained=6000)),
+    # head_dim 256 on the tensor cores: two O^T blocks, two-slot rings, GQA up to 16
+    ("d256_bifocal_grp4_g3", 1, 5000, 8, 2, 256, MapParams(O.BIFOCAL, rope_base=1e6, w0=400, w_pretrained=2000)),
+    ("d256_bifocal_grp8", 2, 3000, 16, 2, 256, MapParams(O.BIFOCAL, rope_base=1e4, w0=128, w_pretrained=1024)),
+    ("d256_standard_grp16", 1, 2000, 32, 2, 256, MapParams(O.STANDARD, rope_base=1e4)),
+    ("long_bifocal_d256_grp2", 1, 40000, 16, 8, 256, MapParams(O.BIFOCAL, rope_base=1e6, w0=2048, w_pretrained=12000)),
 ]
 
 
