@@ -29,11 +29,10 @@ def grad_error(got, ref):
 
 def decode_staged(D):
     """Whether the oracle decode should round its operands to bf16 for a
-    comparison with the CUDA decode: for head_dim 64 and 128 the decode
-    multiplies bf16 operands on the tensor cores (the rotated query views and
-    the corrected remote keys are rounded to bf16); at head_dim 256 it keeps
-    its rotations and dot products in fp32 registers."""
-    return D <= 128
+    comparison with the CUDA decode: at every head_dim (64, 128, 256) the
+    decode multiplies bf16 operands on the tensor cores (the rotated query
+    views and the corrected remote keys are rounded to bf16)."""
+    return D in (64, 128, 256)
 
 
 def max_abs(a, b):
