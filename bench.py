@@ -581,6 +581,7 @@ def config_dict(n_gpus):
 # GPU arm
 # ----------------------------------------------------------------------------
 CONFIG_PROFILES = ("standard_s512", "endprompt_s8192", "periodic_s32768", "nope_s32768")
+DECODE_PROFILES = {"decode256": 256, "decode64": 64}
 
 
 def run_profile_case(which: str):
@@ -591,7 +592,9 @@ def run_profile_case(which: str):
     decode (512 MiB of cache); backward: the backward of the 32768-token
     case (G = 4); prefill131072: the full-size attention, for one-pass
     counters only; standard_s512, endprompt_s8192, periodic_s32768,
-    nope_s32768: those workloads at full size (under 2 GB each)."""
+    nope_s32768: those workloads at full size (under 2 GB each); decode256,
+    decode64: the 131072-key bifocal decode at head_dim 256 (1 GiB of cache)
+    and 64."""
     from position_remapping_b200 import ropeattn as ra
     dev = torch.device("cuda", 0)
     if which == "prefill131072":
@@ -638,7 +641,8 @@ def run_profile_case(which: str):
             ra.prefill(q, k, v, params, out=out, lse=lse, workspace=ws)
     else:
         Dd = DECODE
-        qd, kd, vd = make_qkv(Dd.B, Dd.S, Dd.Hq, Dd.Hkv, Dd.D, Dd.seed, device=dev, q_len=1)
+        D = DECODE_PROFILES.get(which, Dd.D)
+        qd, kd, vd = make_qkv(Dd.B, Dd.S, Dd.Hq, Dd.Hkv, D, Dd.seed, device=dev, q_len=1)
         for _ in range(3):
             ra.decode(qd, kd, vd, Dd.params)
     torch.cuda.synchronize()
@@ -653,7 +657,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", choices=["prefill", "prefill131072", "prefill256", "decode", "backward",
-                                          *CONFIG_PROFILES], default=None,
+                                          *CONFIG_PROFILES, *DECODE_PROFILES], default=None,
                     help="run a capture-sized case of one kernel three times (for ncu); no timing, no JSON")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)

@@ -1,5 +1,6 @@
 """Shared helpers of the GPU parity tests: tolerances and comparisons."""
 import numpy as np
+import torch
 
 # Bars for floating-point parity with the float64 oracle on bf16 inputs:
 # max-abs error of the attention output and of the natural-log LSE.
@@ -33,6 +34,13 @@ def decode_staged(D):
     decode multiplies bf16 operands on the tensor cores (the rotated query
     views and the corrected remote keys are rounded to bf16)."""
     return D in (64, 128, 256)
+
+
+def deinterleave(x):
+    """Adjacent storage order (element 2i = coordinate i, 2i+1 = coordinate
+    i + D/2, as half-split key caches hold each rotated key) -> the heads'
+    own order along the last axis."""
+    return torch.cat([x[..., 0::2], x[..., 1::2]], dim=-1)
 
 
 def max_abs(a, b):
