@@ -57,17 +57,21 @@ class CParams(ctypes.Structure):
 
 
 _CPARAMS_CACHE: dict = {}
+_CPARAMS_LAST: list = [None, None]   # the last (MapParams object, struct): a decode loop passes the same object
 
 
 def _cparams(p: MapParams) -> CParams:
     """The C parameter struct of `p` for the binding's own calls, which never
     modify it (cached: MapParams is frozen, and a decode step runs every
     token)."""
+    if _CPARAMS_LAST[0] is p:
+        return _CPARAMS_LAST[1]
     c = _CPARAMS_CACHE.get(p)
     if c is None:
         c = to_cparams(p)
         if len(_CPARAMS_CACHE) < 256:
             _CPARAMS_CACHE[p] = c
+    _CPARAMS_LAST[0], _CPARAMS_LAST[1] = p, c
     return c
 
 
@@ -151,20 +155,27 @@ def _current_device() -> int:
 
 
 def _device_of(t: torch.Tensor):
-    return t.device.type, t.device.index
+    idx = t.get_device()   # -1 for a CPU tensor
+    if idx >= 0 and t.is_cuda:
+        return "cuda", idx
+    d = t.device
+    return d.type, d.index
 
 
 def _stream(stream) -> Optional[int]:
     if stream is None:
         stream = torch.cuda.current_stream()
-    dev = getattr(stream, "device", None)
-    if dev is not None and dev.index != _current_device():
-        raise ValueError(f"the stream belongs to {dev}, but the current device is cuda:{_current_device()}")
+    idx = getattr(stream, "device_index", None)
+    if idx is None:
+        dev = getattr(stream, "device", None)
+        idx = None if dev is None else dev.index
+    if idx is not None and idx != _current_device():
+        raise ValueError(f"the stream belongs to cuda:{idx}, but the current device is cuda:{_current_device()}")
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
 def _ptr(t: Optional[torch.Tensor]):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    return None if t is None else t.data_ptr()   # the argtypes declare void*
 
 
 # The C ABI sees only pointers and sizes: the dtype, layout and device of
@@ -174,7 +185,7 @@ def _need(t, name: str, dtype, shape=None) -> torch.Tensor:
         raise TypeError(f"{name} must be a torch.Tensor")
     if t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype} (got {t.dtype})")
-    if shape is not None and tuple(t.shape) != tuple(shape):
+    if shape is not None and t.shape != shape:
         raise ValueError(f"{name} must have shape {tuple(shape)} (got {tuple(t.shape)})")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
