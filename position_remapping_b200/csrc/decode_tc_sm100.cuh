@@ -5,14 +5,16 @@
 // head; the grid is one wave. The range streams through shared memory by TMA
 // in 128-key tiles (128-byte swizzle, no multicast), K tiles and V tiles in
 // rings of their own: K in whole tiles, V in 64-key halves, so a V slot is
-// free as soon as the four PV MMAs of its half have read it. Per tile, with the GQA group's query heads as the MMA's N
-// dimension (the tensor cores see the keys as M = 128 rows):
+// free as soon as the four PV MMAs of its half have read it. Per tile, with
+// the GQA group's query heads as the MMA's N dimension (the tensor cores see
+// the keys as M = 128 rows):
 //   S^T = K' Q^T   tcgen05.mma, A = the K tile (K-major), B = the staged
 //                  query rows (K-major), fp32 into TMEM (lane = key);
-//   softmax        lane = key: the score of each head, the tile maximum per
-//                  head (warp shuffles, then an mbarrier exchange between the
-//                  four softmax warps), exp2 with a lazily moved reference
-//                  maximum, P^T (bf16) into shared memory;
+//   softmax        lane = key: the score of each head, exp2 against a lazily
+//                  moved reference maximum per head (one barrier reduction
+//                  over the four softmax warps asks whether any score exceeds
+//                  it by more than 2^8; only then are the tile maxima
+//                  exchanged), P^T (bf16) into shared memory;
 //   O^T += V^T P^T tcgen05.mma, A = the V tile read MN-major (the head_dim
 //                  axis as M), B = P^T, fp32 accumulator in TMEM (lane = one
 //                  output dimension).
@@ -83,11 +85,11 @@ struct DecodeTcShape {
   static constexpr int kQBytes = (D / 64) * NB * 128;
   static constexpr int kP = kQ + kQBytes;                    // [2 bufs][2 key blocks][kTcNP rows][128 B]
   static constexpr int kPBuf = 2 * kTcNP * 128;
-  static constexpr int kRed = kP + 2 * kPBuf;                // [2][4 warps][GP] tile maxima, then [4][GP] sums
+  static constexpr int kRed = kP + 2 * kPBuf;                // [4 warps][GP] tile maxima, then [4][GP] sums
   static constexpr int kBar = kRed + 2 * 4 * GP * 4 + 64;
   // kfull, rot, kempty [kKSlots each]; vfull, vempty [kVHalves each];
-  // s_full, s_free, p_full, pv_done, mx [2 each]
-  static constexpr int kNumBars = 3 * kKSlots + 2 * kVHalves + 10;
+  // s_full, s_free, p_full, pv_done [2 each]
+  static constexpr int kNumBars = 3 * kKSlots + 2 * kVHalves + 8;
   static constexpr int kMisc = kBar + kNumBars * 8;          // tmem base, abort flag, last flag
   static constexpr int kTotal = kMisc + 16;
   static constexpr int kAlloc = kTotal + 1024;               // slack to align the base to 1024
@@ -148,7 +150,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* s_free = s_full + 2;     // [2]
   uint64_t* p_full = s_free + 2;     // [2]
   uint64_t* pv_done = p_full + 2;    // [2]
-  uint64_t* mx = pv_done + 2;        // [2] tile maxima exchanged
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   volatile int* last_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
@@ -184,7 +185,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(s_free + a, 128);
       mbar_init(p_full + a, 128);
       mbar_init(pv_done + a, 1);
-      mbar_init(mx + a, 4);
     }
     *abort_flag = 0;
     *last_flag = 0;
@@ -491,60 +491,84 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     bool ok = true;
     for (int t = 0; t < ntile; ++t) {
       const int k = kb + t * kTcKeys + r;
-      if (!wwait(s_full + (t & 1), (t >> 1) & 1)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t sv[NB];
-      if constexpr (NB == 16) {
-        tmem_ld16(tS + (t & 1) * NB + lane_off, *reinterpret_cast<uint32_t(*)[16]>(sv));
+      // a failed wait does not leave the loop on its own: it is reduced with
+      // the other softmax warps at the tile's barrier below, so all four
+      // leave together and none waits at a barrier the others have left
+      const bool okw = ok && wwait(s_full + (t & 1), (t >> 1) & 1);
+      float sc[GP];
+      bool raise = false;   // a score above the reference maximum by more than 8 (x256)
+      if (okw) {
+        tc_fence_after();
+        uint32_t sv[NB];
+        if constexpr (NB == 16) {
+          tmem_ld16(tS + (t & 1) * NB + lane_off, *reinterpret_cast<uint32_t(*)[16]>(sv));
+        } else {
+          tmem_ld32(tS + (t & 1) * NB + lane_off, *reinterpret_cast<uint32_t(*)[32]>(sv));
+        }
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(s_free + (t & 1));
+        const bool valid = k < ke;
+        const bool remote = ROT != 0 && k < p.k_local;
+#pragma unroll
+        for (int gi = 0; gi < GP; ++gi) {
+          const uint32_t raw = remote ? sv[(ROT != 0 ? GP : 0) + gi] : sv[gi];
+          sc[gi] = valid ? __uint_as_float(raw) * sl2 : -INFINITY;
+          raise |= sc[gi] > m_run[gi] + 8.0f;
+        }
       } else {
-        tmem_ld32(tS + (t & 1) * NB + lane_off, *reinterpret_cast<uint32_t(*)[32]>(sv));
+#pragma unroll
+        for (int gi = 0; gi < GP; ++gi) sc[gi] = -INFINITY;
       }
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(s_free + (t & 1));
-      const bool valid = k < ke;
-      const bool remote = ROT != 0 && k < p.k_local;
-      float sc[GP], wm[GP];
-#pragma unroll
-      for (int gi = 0; gi < GP; ++gi) {
-        const uint32_t raw = remote ? sv[(ROT != 0 ? GP : 0) + gi] : sv[gi];
-        sc[gi] = valid ? __uint_as_float(raw) * sl2 : -INFINITY;
-        wm[gi] = sc[gi];
-      }
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1)
-#pragma unroll
-        for (int gi = 0; gi < GP; ++gi) wm[gi] = fmaxf(wm[gi], __shfl_xor_sync(0xffffffffu, wm[gi], off));
-      float* rb = red + (t & 1) * 4 * GP;
-      if (lane == 0) {
-#pragma unroll
-        for (int gi = 0; gi < GP; ++gi) rb[warp * GP + gi] = wm[gi];
-        mbar_arrive(mx + (t & 1));
-      }
-      if (!wwait(mx + (t & 1), (t >> 1) & 1)) { ok = false; break; }
+      // lazy rescale: the reference maximum of a head moves only when the
+      // tile's maximum exceeds it by more than 8. Whether any head must move
+      // (or any wait failed) is one barrier reduction over the 128 softmax
+      // threads; only then are the tile maxima exchanged
       bool need_any = false;
       float corr[GP];
+#pragma unroll
+      for (int gi = 0; gi < GP; ++gi) corr[gi] = 1.0f;
+      if (bar_red_or(1, 128, raise || !okw)) {
+        if (bar_red_or(1, 128, !okw)) { ok = false; break; }
+        float wm[GP];
+#pragma unroll
+        for (int gi = 0; gi < GP; ++gi) wm[gi] = sc[gi];
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1)
+#pragma unroll
+          for (int gi = 0; gi < GP; ++gi) wm[gi] = fmaxf(wm[gi], __shfl_xor_sync(0xffffffffu, wm[gi], off));
+        // one buffer: every thread has read it before any passes the next
+        // tile's barrier reduction, and only then is it written again
+        if (lane == 0) {
+#pragma unroll
+          for (int gi = 0; gi < GP; ++gi) red[warp * GP + gi] = wm[gi];
+        }
+        bar_sync_named(1, 128);
+#pragma unroll
+        for (int gi = 0; gi < GP; ++gi) {
+          const float tmax = fmaxf(fmaxf(red[gi], red[GP + gi]), fmaxf(red[2 * GP + gi], red[3 * GP + gi]));
+          const bool need = tmax > m_run[gi] + 8.0f;
+          const float m_new = need ? tmax : m_run[gi];
+          corr[gi] = need ? ex2(m_run[gi] - m_new) : 1.0f;
+          l_thr[gi] *= corr[gi];
+          m_run[gi] = m_new;
+          need_any |= need;
+        }
+      }
       uint32_t pb[GP];
 #pragma unroll
       for (int gi = 0; gi < GP; ++gi) {
-        const float tmax = fmaxf(fmaxf(rb[gi], rb[GP + gi]), fmaxf(rb[2 * GP + gi], rb[3 * GP + gi]));
-        // lazy rescale: move the reference max only when it grows by > 8 (x256)
-        const bool need = tmax > m_run[gi] + 8.0f;
-        const float m_new = need ? tmax : m_run[gi];
-        corr[gi] = need ? ex2(m_run[gi] - m_new) : 1.0f;
-        l_thr[gi] *= corr[gi];
-        m_run[gi] = m_new;
-        need_any |= need;
-        const float mu = m_new == -INFINITY ? 0.f : m_new;
+        const float mu = m_run[gi] == -INFINITY ? 0.f : m_run[gi];
         const float pval = ex2(sc[gi] - mu);
         l_thr[gi] += pval;
         pb[gi] = pack_bf16x2(pval, 0.f) & 0xFFFFu;
       }
-      // P^T buffer t&1 was last read by PV(t-2)
-      if (t >= 2 && !wwait(pv_done + (t & 1), ((t >> 1) - 1) & 1)) { ok = false; break; }
+      // P^T buffer t&1 was last read by PV(t-2); a failed wait skips the
+      // rest of the tile and is reduced at the next tile's barrier
+      if (t >= 2 && !wwait(pv_done + (t & 1), ((t >> 1) - 1) & 1)) { ok = false; continue; }
       if (t >= 1 && need_any) {
         // rescale O^T (lane r = output dimension r) once PV(t-1) has completed
-        if (!wwait(pv_done + ((t - 1) & 1), ((t - 1) >> 1) & 1)) { ok = false; break; }
+        if (!wwait(pv_done + ((t - 1) & 1), ((t - 1) >> 1) & 1)) { ok = false; continue; }
         tc_fence_after();
 #pragma unroll
         for (int mb = 0; mb < kMB; ++mb) {
