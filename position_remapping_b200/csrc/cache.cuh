@@ -2,13 +2,14 @@
 // at its own position, and the cache is never rewritten afterwards, however
 // the bifocal group size G changes as the sequence grows.
 //
-// One thread per (token, rotation pair), as in the prefill key pre-pass: the
-// angle p * theta_i is taken in double precision (p the kind's primary
-// position of the token's absolute index), sincos in double, rounded to fp32;
-// the pair is rotated in fp32 and rounded to bf16 (nearest even) for every
-// (batch, kv head) row of the token. The value pair is copied alongside.
-// Consecutive threads touch consecutive 4-byte words of a row. Half-split
-// keys are read pair (i, i + D/2) and stored in adjacent order (pairing.cuh).
+// One thread per (token, four rotation pairs), as in the prefill key
+// pre-pass: the angle p * theta_i is taken in double precision (p the kind's
+// primary position of the token's absolute index), sincos in double, rounded
+// to fp32; each pair is rotated in fp32 and rounded to bf16 (nearest even)
+// for every (batch, kv head) row of the token. The value quad is copied
+// alongside. Consecutive threads touch consecutive 16-byte groups of a row.
+// Half-split keys are read pair (i, i + D/2) and stored in adjacent order
+// (pairing.cuh).
 #pragma once
 
 #include "common.cuh"
@@ -29,35 +30,47 @@ struct CacheArgs {
   double theta[kMaxPairs];
 };
 
+// One thread per (token, four rotation pairs); the host launches
+// ceil(count / (256 / (D/8))) blocks of 256 threads.
 __global__ void __launch_bounds__(256) cache_write_kernel(const CacheArgs a) {
   const int P = a.D >> 1;
-  const int rows = blockDim.x / P;
-  const long long i_tok = static_cast<long long>(blockIdx.x) * rows + threadIdx.x / P;
-  const int i = threadIdx.x % P;
+  const int Q = P >> 2;                       // four-pair chunks per row
+  const int rows = blockDim.x / Q;
+  const long long i_tok = static_cast<long long>(blockIdx.x) * rows + threadIdx.x / Q;
+  const int c = threadIdx.x % Q;
   if (i_tok >= a.count) return;
   const long long t = a.start + i_tok;
-  float c = 1.f, s = 0.f;
+  float cs[4] = {1.f, 1.f, 1.f, 1.f}, sn[4] = {0.f, 0.f, 0.f, 0.f};
   if (a.m.kind != kNope) {
-    double sd, cd;
-    sincos(static_cast<double>(pos_primary(a.m, static_cast<int>(t))) * a.theta[i], &sd, &cd);
-    c = static_cast<float>(cd);
-    s = static_cast<float>(sd);
-  }
-  for (int b = 0; b < a.B; ++b) {
-    for (int h = 0; h < a.Hkv; ++h) {
-      const size_t src_row = ((static_cast<size_t>(b) * a.count + i_tok) * a.Hkv + h) * P;
-      const size_t src = src_row + i;
-      const size_t dst = ((static_cast<size_t>(b) * a.cache_len + t) * a.Hkv + h) * P + i;
-      if (a.m.kind == kNope) {
-        a.k_cache[dst] = __ldg(a.k + src);
-      } else {
-        float x0, x1, y0, y1;
-        load_rot_pair(a.k, src_row, i, P, a.half != 0, x0, x1);
-        rot_pair(x0, x1, c, s, y0, y1);
-        a.k_cache[dst] = pack_bf16x2(y0, y1);
-      }
-      if (a.v != nullptr) a.v_cache[dst] = __ldg(a.v + src);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      double sd, cd;
+      sincos(static_cast<double>(pos_primary(a.m, static_cast<int>(t))) * a.theta[4 * c + j], &sd, &cd);
+      cs[j] = static_cast<float>(cd);
+      sn[j] = static_cast<float>(sd);
     }
+  }
+#pragma unroll 4
+  for (int bh = 0; bh < a.B * a.Hkv; ++bh) {
+    const int b = bh / a.Hkv, h = bh % a.Hkv;
+    const size_t src_row = ((static_cast<size_t>(b) * a.count + i_tok) * a.Hkv + h) * P;
+    const size_t dst_row = ((static_cast<size_t>(b) * a.cache_len + t) * a.Hkv + h) * P;
+    if (a.m.kind == kNope) {
+      reinterpret_cast<uint4*>(a.k_cache + dst_row)[c] = __ldg(reinterpret_cast<const uint4*>(a.k + src_row) + c);
+    } else {
+      float x0[4], x1[4];
+      load_rot_quad(a.k, src_row, c, P, a.half != 0, x0, x1);
+      uint32_t y[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float y0, y1;
+        rot_pair(x0[j], x1[j], cs[j], sn[j], y0, y1);
+        y[j] = pack_bf16x2(y0, y1);
+      }
+      reinterpret_cast<uint4*>(a.k_cache + dst_row)[c] = make_uint4(y[0], y[1], y[2], y[3]);
+    }
+    if (a.v != nullptr)
+      reinterpret_cast<uint4*>(a.v_cache + dst_row)[c] = __ldg(reinterpret_cast<const uint4*>(a.v + src_row) + c);
   }
 }
 

@@ -34,6 +34,29 @@ __device__ __forceinline__ void load_rot_pair(const uint32_t* words, size_t row_
   }
 }
 
+// Rotation pairs 4c .. 4c+3 of a row, as rotate-ready values: x0[j], x1[j]
+// are the pair 4c+j ((x_{2i}, x_{2i+1}) adjacent, (x_i, x_{i+D/2})
+// half-split). One 16-byte load (adjacent) or two 8-byte loads (half-split);
+// row_word indexes the row's first 4-byte word (16-byte aligned rows), P = D/2.
+__device__ __forceinline__ void load_rot_quad(const uint32_t* words, size_t row_word, int c, int P, bool half,
+                                              float (&x0)[4], float (&x1)[4]) {
+  if (!half) {
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(words + row_word) + c);
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      x0[j] = bf16lo(ww[j]);
+      x1[j] = bf16hi(ww[j]);
+    }
+  } else {
+    const uint2* g = reinterpret_cast<const uint2*>(words + row_word);
+    const uint2 lo = __ldg(g + c);            // x_{4c} .. x_{4c+3}
+    const uint2 hi = __ldg(g + P / 4 + c);    // x_{P+4c} .. x_{P+4c+3}
+    x0[0] = bf16lo(lo.x); x0[1] = bf16hi(lo.x); x0[2] = bf16lo(lo.y); x0[3] = bf16hi(lo.y);
+    x1[0] = bf16lo(hi.x); x1[1] = bf16hi(hi.x); x1[2] = bf16lo(hi.y); x1[3] = bf16hi(hi.y);
+  }
+}
+
 // out[r] = pi(in[r]) for rows of D bf16 values: out[2i] = in[i],
 // out[2i+1] = in[i + D/2]. Four pairs per thread: two 8-byte loads, one
 // 16-byte store. Both buffers 16-byte aligned; D a multiple of 8.

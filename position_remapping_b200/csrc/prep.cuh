@@ -32,29 +32,48 @@ struct PrepArgs {
   double theta[kMaxPairs];
 };
 
+// One thread per (token, four rotation pairs): the angles of its pairs
+// under each map once, then for every (batch, head) row one 16-byte load of
+// the key quad, rotated under every map, one 16-byte store per map. The
+// host launches ceil(S / (256 / (D/8))) blocks of 256 threads.
 __global__ void __launch_bounds__(256) rope_prep_kernel(const PrepArgs a) {
   const int P = a.D >> 1;
-  const int rows = blockDim.x / P;
-  const int t = blockIdx.x * rows + threadIdx.x / P;
-  const int i = threadIdx.x % P;
+  const int Q = P >> 2;                       // four-pair chunks per row
+  const int rows = blockDim.x / Q;
+  const int t = blockIdx.x * rows + threadIdx.x / Q;
+  const int c = threadIdx.x % Q;
   if (t >= a.S) return;
   const int nmaps = a.k_rot1 ? 2 : 1;
+  float cs[2][4], sn[2][4];
   for (int mi = 0; mi < nmaps; ++mi) {
     const int p = mi == 0 ? pos_primary(a.m, t) : pos_remote(a.m, t);
-    double sd, cd;
-    sincos(static_cast<double>(p) * a.theta[i], &sd, &cd);
-    const float c = static_cast<float>(cd), s = static_cast<float>(sd);
-    float2* tab = mi == 0 ? a.tab0 : a.tab1;
-    tab[static_cast<size_t>(t) * P + i] = make_float2(c, s);
-    uint32_t* dst = mi == 0 ? a.k_rot0 : a.k_rot1;
-    for (int b = 0; b < a.B; ++b) {
-      for (int h = 0; h < a.Hkv; ++h) {
-        const size_t row = ((static_cast<size_t>(b) * a.S + t) * a.Hkv + h) * P;
-        float x0, x1, y0, y1;
-        load_rot_pair(a.k, row, i, P, a.half != 0, x0, x1);
-        rot_pair(x0, x1, c, s, y0, y1);
-        dst[row + i] = pack_bf16x2(y0, y1);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      double sd, cd;
+      sincos(static_cast<double>(p) * a.theta[4 * c + j], &sd, &cd);
+      cs[mi][j] = static_cast<float>(cd);
+      sn[mi][j] = static_cast<float>(sd);
+    }
+    float4* tab = reinterpret_cast<float4*>((mi == 0 ? a.tab0 : a.tab1) + static_cast<size_t>(t) * P + 4 * c);
+    tab[0] = make_float4(cs[mi][0], sn[mi][0], cs[mi][1], sn[mi][1]);
+    tab[1] = make_float4(cs[mi][2], sn[mi][2], cs[mi][3], sn[mi][3]);
+  }
+#pragma unroll 4
+  for (int bh = 0; bh < a.B * a.Hkv; ++bh) {
+    const int b = bh / a.Hkv, h = bh % a.Hkv;
+    const size_t row = ((static_cast<size_t>(b) * a.S + t) * a.Hkv + h) * P;
+    float x0[4], x1[4];
+    load_rot_quad(a.k, row, c, P, a.half != 0, x0, x1);
+    for (int mi = 0; mi < nmaps; ++mi) {
+      uint32_t y[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float y0, y1;
+        rot_pair(x0[j], x1[j], cs[mi][j], sn[mi][j], y0, y1);
+        y[j] = pack_bf16x2(y0, y1);
       }
+      uint32_t* dst = mi == 0 ? a.k_rot0 : a.k_rot1;
+      reinterpret_cast<uint4*>(dst + row)[c] = make_uint4(y[0], y[1], y[2], y[3]);
     }
   }
 }

@@ -448,7 +448,7 @@ int ropeattn_cache_write(const void* k, const void* v, void* k_cache, void* v_ca
   m.kind = params->kind == ROPEATTN_BIFOCAL ? ROPEATTN_STANDARD : params->kind;  // primary position: t
   a.m = m;
   fill_theta(params, D, a.theta);
-  const int rows = 256 / (D / 2);
+  const int rows = 256 / (D / 8);   // four rotation pairs per thread
   cache_write_kernel<<<static_cast<unsigned>((count + rows - 1) / rows), 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
   CUDA_TRY(cudaGetLastError(), "cache_write launch");
   return ROPEATTN_OK;
@@ -521,7 +521,7 @@ int prefill_impl(int stages, const void* q, const void* k, const void* v, float*
     a.m = m;
     if (stages & kStagePrepare) {
       fill_theta(params, D, a.theta);
-      const int rows = 256 / (D / 2);
+      const int rows = 256 / (D / 8);   // four rotation pairs per thread
       rope_prep_kernel<<<static_cast<unsigned>((S + rows - 1) / rows), 256, 0, st>>>(a);
       CUDA_TRY(cudaGetLastError(), "rope_prep launch");
     }
@@ -749,7 +749,7 @@ int ropeattn_prefill_three_call(const void* q, const void* k, const void* v, flo
   a.half = lay.half ? 1 : 0;
   a.m = m;
   fill_theta(params, D, a.theta);
-  const int prow = 256 / (D / 2);
+  const int prow = 256 / (D / 8);   // four rotation pairs per thread
   rope_prep_kernel<<<static_cast<unsigned>((S + prow - 1) / prow), 256, 0, st>>>(a);
   CUDA_TRY(cudaGetLastError(), "rope_prep launch");
   if (lay.half) {
@@ -1123,7 +1123,7 @@ extern "C" int ropeattn_prefill_backward(const void* q, const void* k, const voi
     a.half = half_pairing(params) ? 1 : 0;
     a.m = m;
     fill_theta(params, D, a.theta);
-    const int rows = 256 / (D / 2);
+    const int rows = 256 / (D / 8);   // four rotation pairs per thread
     for (int side = 0; side < 2; ++side) {
       a.k = static_cast<const uint32_t*>(side == 0 ? k : q);
       a.Hkv = side == 0 ? Hkv : Hq;
