@@ -134,8 +134,9 @@ int ropeattn_posmap(const ropeattn_params* params, int64_t L,
  * adjacent order (element 2i = rotated coordinate i, 2i+1 = rotated
  * coordinate i + D/2), the order every cache reader of this library expects
  * for half-split params; values are copied as given.
- *   k, v:             [B, count, Hkv, D] bf16, device, 4-byte aligned
- *   k_cache, v_cache: [B, cache_len, Hkv, D] bf16, device; caller-owned
+ *   k, v:             [B, count, Hkv, D] bf16, device, 16-byte aligned
+ *   k_cache, v_cache: [B, cache_len, Hkv, D] bf16, device, 16-byte aligned;
+ *                     caller-owned
  *   v, v_cache:       both NULL to write keys only
  *   start + count <= cache_len. A prefill of S tokens emits its cache with
  *   start = 0, count = S; a decode step appends its token with start = n-1

@@ -91,32 +91,44 @@ struct UnfusedRotArgs {
   double theta[kMaxPairs];
 };
 
+// One thread per (key, four rotation pairs); the host launches
+// ceil(n / (256 / (D/8))) blocks of 256 threads.
 __global__ void __launch_bounds__(256) unfused_rotate_kernel(const UnfusedRotArgs a) {
   const int P = a.D >> 1;
-  const int rows = blockDim.x / P;
-  const int s = blockIdx.x * rows + threadIdx.x / P;
-  const int i = threadIdx.x % P;
+  const int Q = P >> 2;                       // four-pair chunks per row
+  const int rows = blockDim.x / Q;
+  const int s = blockIdx.x * rows + threadIdx.x / Q;
+  const int c = threadIdx.x % Q;
   if (s >= a.n) return;
   const bool remote = s < a.k_local;
-  float c = 1.f, sn = 0.f;
+  float cs[4] = {1.f, 1.f, 1.f, 1.f}, sn[4] = {0.f, 0.f, 0.f, 0.f};
   if (remote) {
-    double sd, cd;
-    sincos(static_cast<double>(pos_remote(a.m, s) - s - a.dq) * a.theta[i], &sd, &cd);
-    c = static_cast<float>(cd);
-    sn = static_cast<float>(sd);
-  }
-  for (int b = 0; b < a.B; ++b) {
-    for (int h = 0; h < a.Hkv; ++h) {
-      const size_t w = ((static_cast<size_t>(b) * a.n + s) * a.Hkv + h) * P + i;
-      const uint32_t x = __ldg(a.k_cache + w);
-      if (remote) {
-        float y0, y1;
-        rot_pair(bf16lo(x), bf16hi(x), c, sn, y0, y1);
-        a.k_out[w] = pack_bf16x2(y0, y1);
-      } else {
-        a.k_out[w] = x;
-      }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      double sd, cd;
+      sincos(static_cast<double>(pos_remote(a.m, s) - s - a.dq) * a.theta[4 * c + j], &sd, &cd);
+      cs[j] = static_cast<float>(cd);
+      sn[j] = static_cast<float>(sd);
     }
+  }
+#pragma unroll 4
+  for (int bh = 0; bh < a.B * a.Hkv; ++bh) {
+    const int b = bh / a.Hkv, h = bh % a.Hkv;
+    const size_t row = ((static_cast<size_t>(b) * a.n + s) * a.Hkv + h) * P;
+    const uint4 x = __ldg(reinterpret_cast<const uint4*>(a.k_cache + row) + c);
+    uint4 y = x;
+    if (remote) {
+      const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+      uint32_t yw[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float y0, y1;
+        rot_pair(bf16lo(xw[j]), bf16hi(xw[j]), cs[j], sn[j], y0, y1);
+        yw[j] = pack_bf16x2(y0, y1);
+      }
+      y = make_uint4(yw[0], yw[1], yw[2], yw[3]);
+    }
+    reinterpret_cast<uint4*>(a.k_out + row)[c] = y;
   }
 }
 

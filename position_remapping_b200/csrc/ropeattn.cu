@@ -429,8 +429,8 @@ int ropeattn_cache_write(const void* k, const void* v, void* k_cache, void* v_ca
   if ((v == nullptr) != (v_cache == nullptr))
     return fail(ROPEATTN_ERR_INVALID_ARG, "v and v_cache must be both given or both NULL");
   if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v) |
-       reinterpret_cast<uintptr_t>(v_cache)) & 3u)
-    return fail(ROPEATTN_ERR_INVALID_ARG, "tensor pointers must be 4-byte aligned");
+       reinterpret_cast<uintptr_t>(v_cache)) & 15u)
+    return fail(ROPEATTN_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
   rc = check_device();
   if (rc) return rc;
   CacheArgs a{};
@@ -979,7 +979,7 @@ int ropeattn_decode_unfused(const void* q, const void* k_cache, const void* v_ca
   a.m = m;
   a.dq = pos_remote(m, static_cast<int>(t)) - static_cast<int>(t);
   fill_theta(params, D, a.theta);
-  const int rows = 256 / (D / 2);
+  const int rows = 256 / (D / 8);   // four rotation pairs per thread
   unfused_rotate_kernel<<<static_cast<unsigned>((n + rows - 1) / rows), 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
   CUDA_TRY(cudaGetLastError(), "unfused rotate launch");
   // standard RoPE decode over the rotated copy: query at p(t) = t, keys as stored

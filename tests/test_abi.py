@@ -146,9 +146,12 @@ def test_cache_write_argument_checks(ra):
     # v and v_cache must come together; k must be given
     assert lib.ropeattn_cache_write(fake, fake, fake, nullp, 1, 0, 2, 100, 2, 64, p, nullp) == ra.ERR_INVALID_ARG
     assert lib.ropeattn_cache_write(nullp, nullp, fake, nullp, 1, 0, 2, 100, 2, 64, p, nullp) == ra.ERR_INVALID_ARG
-    # misaligned pointer
-    odd = ctypes.c_void_p((1 << 20) + 2)
-    assert lib.ropeattn_cache_write(odd, nullp, fake, nullp, 1, 0, 2, 100, 2, 64, p, nullp) == ra.ERR_INVALID_ARG
+    # misaligned pointers (the kernel moves 16-byte groups)
+    for off in (2, 4, 8):
+        odd = ctypes.c_void_p((1 << 20) + off)
+        assert lib.ropeattn_cache_write(odd, nullp, fake, nullp, 1, 0, 2, 100, 2, 64, p, nullp) == ra.ERR_INVALID_ARG
+        assert lib.ropeattn_cache_write(fake, nullp, odd, nullp, 1, 0, 2, 100, 2, 64, p, nullp) == ra.ERR_INVALID_ARG
+        assert "16-byte" in lib.ropeattn_last_error().decode()
     # nothing to write
     q = ctypes.byref(ra.to_cparams(_p(kind=STANDARD)))
     assert lib.ropeattn_cache_write(nullp, nullp, nullp, nullp, 1, 5, 0, 100, 2, 64, q, nullp) == ra.OK
