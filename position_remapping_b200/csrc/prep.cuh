@@ -95,35 +95,52 @@ struct ChunkPrepArgs {
   double theta[kMaxPairs];
 };
 
+// One thread per (token, four rotation pairs); the host launches
+// ceil(L / (256 / (D/8))) blocks of 256 threads.
 __global__ void __launch_bounds__(256) chunk_prep_kernel(const ChunkPrepArgs a) {
   const int P = a.D >> 1;
-  const int rows = blockDim.x / P;
-  const int t = blockIdx.x * rows + threadIdx.x / P;
-  const int i = threadIdx.x % P;
+  const int Q = P >> 2;                       // four-pair chunks per row
+  const int rows = blockDim.x / Q;
+  const int t = blockIdx.x * rows + threadIdx.x / Q;
+  const int c = threadIdx.x % Q;
   if (t >= a.L) return;
   if (a.k_rem != nullptr) {
-    double sd, cd;
-    sincos(static_cast<double>(pos_remote(a.m, t) - t) * a.theta[i], &sd, &cd);
-    const float c = static_cast<float>(cd), s = static_cast<float>(sd);
-    for (int b = 0; b < a.B; ++b) {
-      for (int h = 0; h < a.Hkv; ++h) {
-        const size_t w = ((static_cast<size_t>(b) * a.L + t) * a.Hkv + h) * P + i;
-        const size_t r = ((static_cast<size_t>(b) * a.cache_rows + t) * a.Hkv + h) * P + i;
-        const uint32_t x = __ldg(a.k_cache + r);
+    float cs[4], sn[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      double sd, cd;
+      sincos(static_cast<double>(pos_remote(a.m, t) - t) * a.theta[4 * c + j], &sd, &cd);
+      cs[j] = static_cast<float>(cd);
+      sn[j] = static_cast<float>(sd);
+    }
+#pragma unroll 4
+    for (int bh = 0; bh < a.B * a.Hkv; ++bh) {
+      const int b = bh / a.Hkv, h = bh % a.Hkv;
+      const size_t w = ((static_cast<size_t>(b) * a.L + t) * a.Hkv + h) * P;
+      const size_t r = ((static_cast<size_t>(b) * a.cache_rows + t) * a.Hkv + h) * P;
+      const uint4 x = __ldg(reinterpret_cast<const uint4*>(a.k_cache + r) + c);
+      const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+      uint32_t y[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
         float y0, y1;
-        rot_pair(bf16lo(x), bf16hi(x), c, s, y0, y1);
-        a.k_rem[w] = pack_bf16x2(y0, y1);
+        rot_pair(bf16lo(xw[j]), bf16hi(xw[j]), cs[j], sn[j], y0, y1);
+        y[j] = pack_bf16x2(y0, y1);
       }
+      reinterpret_cast<uint4*>(a.k_rem + w)[c] = make_uint4(y[0], y[1], y[2], y[3]);
     }
   }
   if (t >= a.start && a.tab0 != nullptr) {
-    const size_t r = static_cast<size_t>(t - a.start) * P + i;
-    double sd, cd;
-    sincos(static_cast<double>(pos_primary(a.m, t)) * a.theta[i], &sd, &cd);
-    a.tab0[r] = make_float2(static_cast<float>(cd), static_cast<float>(sd));
-    if (a.tab1 != nullptr) {
-      sincos(static_cast<double>(pos_remote(a.m, t)) * a.theta[i], &sd, &cd);
-      a.tab1[r] = make_float2(static_cast<float>(cd), static_cast<float>(sd));
+    const size_t r = static_cast<size_t>(t - a.start) * P + 4 * c;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      double sd, cd;
+      sincos(static_cast<double>(pos_primary(a.m, t)) * a.theta[4 * c + j], &sd, &cd);
+      a.tab0[r + j] = make_float2(static_cast<float>(cd), static_cast<float>(sd));
+      if (a.tab1 != nullptr) {
+        sincos(static_cast<double>(pos_remote(a.m, t)) * a.theta[4 * c + j], &sd, &cd);
+        a.tab1[r + j] = make_float2(static_cast<float>(cd), static_cast<float>(sd));
+      }
     }
   }
 }

@@ -655,7 +655,7 @@ int ropeattn_prefill_chunk_cache(const void* q, const void* k_cache, const void*
     a.start = static_cast<int>(start);
     a.m = m;
     fill_theta(params, D, a.theta);
-    const int rows = 256 / (D / 2);
+    const int rows = 256 / (D / 8);   // four rotation pairs per thread
     chunk_prep_kernel<<<static_cast<unsigned>((L + rows - 1) / rows), 256, 0, st>>>(a);
     CUDA_TRY(cudaGetLastError(), "chunk_prep launch");
     pp.tab0 = a.tab0;
