@@ -143,7 +143,9 @@ struct PrefillSmem {
   static constexpr int kQBytes = kBM * D * 2;                       // one query tile
   static constexpr int kTileBytes = PrefillShape<D>::kBN * D * 2;   // one K or V tile
   static constexpr int kQ = 0;
-  static constexpr int kRing = kQ + PrefillShape<D>::kQT * kQBytes;
+  // at D = 256 the rotated query tile lives in TMEM and arrives through two
+  // ring slots, so the ring takes the whole space (six 32 KiB slots)
+  static constexpr int kRing = kQ + (D == 256 ? 0 : PrefillShape<D>::kQT * kQBytes);
   static constexpr int kBar = kRing + NSLOT * kTileBytes;
   // barriers: q_full, q_ready[2], q_free, ring_full[NSLOT], ring_empty[NSLOT],
   // s_full[2], s_free, p_full[2], o_done[2], o_free[2]
@@ -170,6 +172,9 @@ __global__ void __launch_bounds__(PrefillShape<D>::kThreads, 1)
   constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, false);
   constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, true);
   constexpr uint32_t kTmemCols = 512;
+  // D = 256: the rotated query tile is the A operand of QK^T from TMEM
+  // (128 lanes x 128 columns of bf16 pairs), staged through two ring slots
+  constexpr bool kQTmem = D == 256;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -245,7 +250,9 @@ __global__ void __launch_bounds__(PrefillShape<D>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tS = tmem;            // S, shared by the two tiles
-  const uint32_t tP = tmem + 128;      // P_a at 128 + 64 a
+  // P_a at 128 + 64 a; at D = 256: S [0,64), Q [64,192), P [192,224)
+  const uint32_t tP = tmem + (kQTmem ? 192 : 128);
+  const uint32_t tQ = tmem + 64;       // D = 256 only
   const uint32_t tO = tmem + 256;      // O_a at 256 + a D
 
   if (warp == SH::kWarpTMA) {
@@ -255,12 +262,26 @@ __global__ void __launch_bounds__(PrefillShape<D>::kThreads, 1)
       int pos = 0;
       bool ok = true;
       for (int pi = 0; pi < npass && ok; ++pi) {
-        // the query tiles of the previous pass must no longer be read
-        if (pi > 0 && !mbar_wait(q_free, (pi - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(q_full, kQT * L::kQBytes);
-        for (int a = 0; a < kQT; ++a)
-          for (int cb = 0; cb < kCB; ++cb)
-            tma_load_4d(sQ + a * L::kQBytes + cb * kBlockBytes, &tmQ, q_full, cb * 64, h, q0 + a * kBM, b);
+        if constexpr (kQTmem) {
+          // the query tile through the next two ring positions (even, so
+          // the two slots are adjacent): its 64-column blocks 0-1, then 2-3
+          for (int hq = 0; hq < 2 && ok; ++hq, ++pos) {
+            const int slot = pos % NSLOT;
+            if (!mbar_wait(ring_empty + slot, ((pos / NSLOT) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            mbar_arrive_expect_tx(ring_full + slot, L::kTileBytes);
+            for (int cb = 2 * hq; cb < 2 * hq + 2; ++cb)
+              tma_load_4d(sRing + slot * L::kTileBytes + (cb - 2 * hq) * kBlockBytes, &tmQ, ring_full + slot,
+                          cb * 64, h, q0, b);
+          }
+          if (!ok) break;
+        } else {
+          // the query tiles of the previous pass must no longer be read
+          if (pi > 0 && !mbar_wait(q_free, (pi - 1) & 1, abort_flag)) break;
+          mbar_arrive_expect_tx(q_full, kQT * L::kQBytes);
+          for (int a = 0; a < kQT; ++a)
+            for (int cb = 0; cb < kCB; ++cb)
+              tma_load_4d(sQ + a * L::kQBytes + cb * kBlockBytes, &tmQ, q_full, cb * 64, h, q0 + a * kBM, b);
+        }
         const CUtensorMap* tk = passes[pi].sel ? &tmK1 : &tmK0;
         for (int j = passes[pi].j_lo; j <= passes[pi].j_hi && ok; ++j) {
           for (int kv = 0; kv < 2; ++kv, ++pos) {
@@ -284,6 +305,13 @@ __global__ void __launch_bounds__(PrefillShape<D>::kThreads, 1)
         if (!mbar_wait(q_ready + 0, pi & 1, abort_flag) ||
             (kQT == 2 && !mbar_wait(q_ready + 1, pi & 1, abort_flag)))
           break;
+        if constexpr (kQTmem) {
+          // every softmax thread has read the query tile's two ring slots
+          // (and stored it in TMEM): hand the slots back to the producer
+          mbar_arrive(ring_empty + pos % NSLOT);
+          mbar_arrive(ring_empty + (pos + 1) % NSLOT);
+          pos += 2;
+        }
         const int T = passes[pi].j_hi - passes[pi].j_lo + 1;
         for (int i = 0; i < T && ok; ++i, pos += 2) {
           const int kslot = pos % NSLOT;
@@ -293,12 +321,22 @@ __global__ void __launch_bounds__(PrefillShape<D>::kThreads, 1)
             // S = Q_a K^T, once the previous S has been copied out
             if (nqk > 0 && !mbar_wait(s_free, (nqk - 1) & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t qaddr = smem_u32(sQ + a * L::kQBytes);
+            if constexpr (kQTmem) {
+              // A = the rotated query tile in TMEM (8 columns per 16 dimensions)
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t kin = (kk & 3) * 32;   // K step inside a 64-column swizzle block
-              umma_ss(tS, sdesc_sw128(qaddr + (kk >> 2) * kBlockBytes + kin, 16, 1024),
-                      sdesc_sw128(kaddr + (kk >> 2) * kKVBlockBytes + kin, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t kin = (kk & 3) * 32;   // K step inside a 64-column swizzle block
+                umma_ts(tS, tQ + kk * 8, sdesc_sw128(kaddr + (kk >> 2) * kKVBlockBytes + kin, 16, 1024), kIdescQK,
+                        kk > 0 ? 1u : 0u);
+              }
+            } else {
+              const uint32_t qaddr = smem_u32(sQ + a * L::kQBytes);
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t kin = (kk & 3) * 32;   // K step inside a 64-column swizzle block
+                umma_ss(tS, sdesc_sw128(qaddr + (kk >> 2) * kBlockBytes + kin, 16, 1024),
+                        sdesc_sw128(kaddr + (kk >> 2) * kKVBlockBytes + kin, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+              }
             }
             umma_commit(s_full + a);
             ++nqk;
@@ -317,6 +355,7 @@ __global__ void __launch_bounds__(PrefillShape<D>::kThreads, 1)
       int pos = 0, g = 0;
       bool ok = true;
       for (int pi = 0; pi < npass && ok; ++pi) {
+        if constexpr (kQTmem) pos += 2;   // the query tile's two ring positions
         const int T = passes[pi].j_hi - passes[pi].j_lo + 1;
         for (int i = 0; i < T && ok; ++i, ++g, pos += 2) {
           const int vpos = pos + 1, vslot = vpos % NSLOT;
@@ -361,12 +400,60 @@ __global__ void __launch_bounds__(PrefillShape<D>::kThreads, 1)
     float* orow = p.out + ((static_cast<size_t>(b) * p.S + (row_ok ? t : 0)) * p.Hq + h) * D;
     bool ok = true;
     int g = 0;
+    int qpos = 0;                            // D = 256: ring position of the pass's query tile
     for (int pi = 0; pi < npass && ok; ++pi) {
       const PassDesc ps = passes[pi];
       // ---- rotate this row of the staged query tile (Periodic RoPE §3.1
       // Eq. 2 at the pass's positions)
-      if (!wwait(q_full, pi & 1)) { ok = false; break; }
-      if (p.tab0 != nullptr) {
+      if constexpr (kQTmem) {
+        // the tile sits in two adjacent ring slots; the rotated row goes to
+        // TMEM lane `row` (column c = dimensions 2c, 2c+1), 32 columns per
+        // store, once the previous pass's QK^T has read the TMEM tile
+        const int qslot = qpos % NSLOT;
+        if (!wwait(ring_full + qslot, (qpos / NSLOT) & 1) ||
+            !wwait(ring_full + qslot + 1, ((qpos + 1) / NSLOT) & 1)) { ok = false; break; }
+        if (pi > 0 && !wwait(q_free, (pi - 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint8_t* sq = sRing + qslot * L::kTileBytes;
+        const float2* tab = ps.sel ? p.tab1 : p.tab0;
+        const float4* tr =
+            tab != nullptr ? reinterpret_cast<const float4*>(tab + static_cast<size_t>(row_ok ? t : 0) * (D / 2))
+                           : nullptr;
+        for (int c0 = 0; c0 < D / 8; c0 += 8) {
+          uint32_t w[32];
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc) {
+            const int c = c0 + cc;
+            const int off = (c >> 3) * kBlockBytes + row * 128 + (((c & 7) ^ (row & 7)) << 4);
+            const uint4 x = *reinterpret_cast<const uint4*>(sq + off);
+            const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) w[4 * cc + e] = xw[e];
+            if (tr != nullptr && row_ok) {
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const float4 cs = __ldg(tr + c * 2 + e);   // pairs 4c+2e, 4c+2e+1
+                float a0, a1;
+                rot_pair(bf16lo(xw[2 * e]), bf16hi(xw[2 * e]), cs.x, cs.y, a0, a1);
+                w[4 * cc + 2 * e] = pack_bf16x2(a0, a1);
+                rot_pair(bf16lo(xw[2 * e + 1]), bf16hi(xw[2 * e + 1]), cs.z, cs.w, a0, a1);
+                w[4 * cc + 2 * e + 1] = pack_bf16x2(a0, a1);
+              }
+            }
+          }
+          tmem_st32(tQ + lane_off + c0 * 4, w);
+        }
+        tmem_st_wait();
+        // this thread's reads of the two slots are done before the next TMA
+        // writes them: the QK issuer hands the slots back once all 128
+        // softmax threads have arrived here
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(q_ready + a);
+        qpos += 2 + 2 * (ps.j_hi - ps.j_lo + 1);
+      }
+      if (!kQTmem && !wwait(q_full, pi & 1)) { ok = false; break; }
+      if (!kQTmem && p.tab0 != nullptr) {
         const float2* tab = ps.sel ? p.tab1 : p.tab0;
         const float4* tr = reinterpret_cast<const float4*>(tab + static_cast<size_t>(row_ok ? t : 0) * (D / 2));
 #pragma unroll 4
@@ -390,8 +477,10 @@ __global__ void __launch_bounds__(PrefillShape<D>::kThreads, 1)
           }
         }
       }
-      fence_proxy_async_smem();
-      mbar_arrive(q_ready + a);
+      if constexpr (!kQTmem) {
+        fence_proxy_async_smem();
+        mbar_arrive(q_ready + a);
+      }
 
       // ---- key tiles of the pass
       float m = -INFINITY, l = 0.f;

@@ -297,7 +297,7 @@ int prefill_bn(int D) { return D == 256 ? PrefillShape<256>::kBN : PrefillShape<
 // One prefill attention launch for the head dimension.
 int launch_prefill_d(int D, const CUtensorMap& tq, const CUtensorMap& tk0, const CUtensorMap& tk1,
                      const CUtensorMap& tv, const PrefillParams& pp, int grid, cudaStream_t st) {
-  if (D == 256) return launch_prefill<256, 4>(tq, tk0, tk1, tv, pp, grid, st);
+  if (D == 256) return launch_prefill<256, 6>(tq, tk0, tk1, tv, pp, grid, st);
   if (D == 128) return launch_prefill<128, 4>(tq, tk0, tk1, tv, pp, grid, st);
   return launch_prefill<64, 8>(tq, tk0, tk1, tv, pp, grid, st);
 }
