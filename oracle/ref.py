@@ -55,6 +55,7 @@ __all__ = [
     "round_bf16", "rope_frequencies", "pair_index", "rotation_matrix", "rotate",
     "periodic_position", "endprompt_position", "group_size", "bifocal_group", "remote_position",
     "position_maps", "softmax_scale", "prefill", "prefill_three_call", "prefill_backward",
+    "prefill_backward_dq_rows",
     "decode", "cache_keys", "prefill_from_cache", "brute_prefill", "brute_decode", "to_f64",
 ]
 
@@ -384,6 +385,67 @@ def prefill_backward(q, k, v, dout, params, stage_bf16: bool = False):
                 dq[b, :, h] += scale * rot(dS @ kl, -p_loc)
                 dk[b, :, hk] += scale * rot(dS.T @ ql, -p_loc)
     return dq, dk, dv
+
+
+def prefill_backward_dq_rows(q, k, v, dout, params, rows, stage_bf16: bool = False, heads=None):
+    """dq of ``prefill_backward`` for the query rows ``rows`` only (and the
+    query heads ``heads``, default all), [B, len(rows), len(heads), D]: the
+    same chain rule, one block of rows at a time, so a row costs O(S D)
+    instead of the O(S^2) softmax of the whole prefill:
+      dq_t = scale * sum_s dS(t,s) R_a^T R_b k_s,
+      dS(t,s) = P(t,s) (dout_t . v_s - sum_s' P(t,s') dout_t . v_s'),
+    with P the row softmax of scale * score(t,s) over the allowed keys
+    (Periodic RoPE §3.1 Eq. 2, §3.2 Eq. 4; Jet-Long §3 Eq. 1, §3.1 Eq. 2-3),
+    split by the window into a local and a remote part for BIFOCAL.
+    Only the slices these rows and heads need are taken to float64."""
+    rows = np.asarray(rows, dtype=np.int64)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    grp = Hq // Hkv
+    heads = list(range(Hq)) if heads is None else list(heads)
+    scale = softmax_scale(D, params)
+    kind = int(params.kind)
+    freqs = _freqs(params, D)
+    pr = _pairing(params)
+    p_loc, p_rem, _G = position_maps(params, S)
+    t_all = np.arange(S)
+    ok = np.stack([_allowed(params, int(r), t_all) for r in rows])            # [R, S]
+    local = (rows[:, None] - t_all[None, :]) <= int(params.w0)
+    stage = round_bf16 if stage_bf16 else (lambda a: a)
+
+    def rot(x, pos):
+        return x if kind == NOPE else rotate(x, pos, freqs, pr)
+
+    def srot(x, pos):
+        return x if kind == NOPE else stage(rotate(x, pos, freqs, pr))
+
+    dq = np.zeros((B, len(rows), len(heads), D))
+    for b in range(B):
+        keys = {}
+        for j, h in enumerate(heads):
+            hk = h // grp
+            if hk not in keys:
+                kk = to_f64(k[b, :, hk])
+                keys[hk] = (srot(kk, p_loc), srot(kk, p_rem) if kind == BIFOCAL else None, to_f64(v[b, :, hk]))
+            kl, kr, vv = keys[hk]
+            qq = to_f64(q[b, rows, h])
+            ql = srot(qq, p_loc[rows])
+            sc = ql @ kl.T
+            if kind == BIFOCAL:
+                qr = srot(qq, p_rem[rows])
+                sc = np.where(local, sc, qr @ kr.T)
+            sc = np.where(ok, sc * scale, -np.inf)
+            m = sc.max(axis=1, keepdims=True)
+            e = np.where(ok, np.exp(sc - m), 0.0)
+            P = e / e.sum(axis=1, keepdims=True)
+            dP = to_f64(dout[b, rows, h]) @ vv.T
+            dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))
+            if kind == BIFOCAL:
+                dSl, dSr = np.where(local, dS, 0.0), np.where(local, 0.0, dS)
+                dq[b, :, j] = scale * (rot(dSl @ kl, -p_loc[rows]) + rot(dSr @ kr, -p_rem[rows]))
+            else:
+                dq[b, :, j] = scale * rot(dS @ kl, -p_loc[rows])
+    return dq
 
 
 # ----------------------------------------------------------------------------

@@ -702,3 +702,25 @@ def test_staged_bifocal_backward_is_close_to_unstaged():
     u = O.prefill_backward(q, k, v, dout, params, stage_bf16=False)
     d = max(np.abs(x - y).max() / max(1.0, np.abs(y).max()) for x, y in zip(a, u))
     assert 1e-8 < d < 0.05
+
+
+@pytest.mark.parametrize("params", [
+    MapParams(O.STANDARD, rope_base=1e4),
+    MapParams(O.ENDPROMPT, rope_base=5e5, interp=8.0, seg1_len=25, term_start=60000),
+    MapParams(O.PERIODIC, rope_base=1e4, window=9),
+    MapParams(O.NOPE),
+    MapParams(O.BIFOCAL, rope_base=1e6, w0=6, w_pretrained=12),
+    MapParams(O.BIFOCAL, rope_base=1e4, w0=3, fixed_group=3, pairing=1),
+], ids=["standard", "endprompt", "periodic", "nope", "bifocal", "bifocal_fixed_half"])
+@pytest.mark.parametrize("staged", [False, True])
+def test_backward_dq_rows_is_the_backward_on_those_rows(params, staged):
+    # the row-block dq (used at full size) against the whole-prefill backward
+    # that the finite-difference and closed-form pins above fix
+    q, k, v = make_qkv(2, 40, 4, 2, 16, seed=51)
+    g = torch.Generator("cpu").manual_seed(52)
+    dout = torch.randn((2, 40, 4, 16), generator=g).to(torch.bfloat16)
+    rows, heads = [0, 5, 17, 30, 39], [1, 3]
+    dq, _, _ = O.prefill_backward(q, k, v, dout, params, stage_bf16=staged)
+    dq_rows = O.prefill_backward_dq_rows(q, k, v, dout, params, rows, stage_bf16=staged, heads=heads)
+    ref = dq[:, rows][:, :, heads]
+    assert np.max(np.abs(dq_rows - ref)) <= 1e-12 * max(1.0, np.max(np.abs(ref)))
