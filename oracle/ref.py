@@ -55,7 +55,7 @@ __all__ = [
     "round_bf16", "rope_frequencies", "pair_index", "rotation_matrix", "rotate",
     "periodic_position", "endprompt_position", "group_size", "bifocal_group", "remote_position",
     "position_maps", "softmax_scale", "prefill", "prefill_three_call", "prefill_backward",
-    "prefill_backward_dq_rows",
+    "prefill_backward_dq_rows", "prefill_backward_tail",
     "decode", "cache_keys", "prefill_from_cache", "brute_prefill", "brute_decode", "to_f64",
 ]
 
@@ -387,22 +387,17 @@ def prefill_backward(q, k, v, dout, params, stage_bf16: bool = False):
     return dq, dk, dv
 
 
-def prefill_backward_dq_rows(q, k, v, dout, params, rows, stage_bf16: bool = False, heads=None):
-    """dq of ``prefill_backward`` for the query rows ``rows`` only (and the
-    query heads ``heads``, default all), [B, len(rows), len(heads), D]: the
-    same chain rule, one block of rows at a time, so a row costs O(S D)
-    instead of the O(S^2) softmax of the whole prefill:
-      dq_t = scale * sum_s dS(t,s) R_a^T R_b k_s,
-      dS(t,s) = P(t,s) (dout_t . v_s - sum_s' P(t,s') dout_t . v_s'),
-    with P the row softmax of scale * score(t,s) over the allowed keys
-    (Periodic RoPE §3.1 Eq. 2, §3.2 Eq. 4; Jet-Long §3 Eq. 1, §3.1 Eq. 2-3),
-    split by the window into a local and a remote part for BIFOCAL.
-    Only the slices these rows and heads need are taken to float64."""
+def _backward_rows(q, k, v, dout, params, rows, stage_bf16, heads):
+    """The chain rule of ``prefill_backward`` restricted to the query rows
+    ``rows`` and the query heads ``heads``: yields, per (batch b, head h),
+    the row softmax P and dS of those rows over all S keys with the operands
+    the sums need. Only the slices these rows and heads touch are taken to
+    float64, so a row costs O(S D) instead of the O(S^2) of the whole
+    prefill."""
     rows = np.asarray(rows, dtype=np.int64)
     B, S, Hq, D = q.shape
     Hkv = k.shape[2]
     grp = Hq // Hkv
-    heads = list(range(Hq)) if heads is None else list(heads)
     scale = softmax_scale(D, params)
     kind = int(params.kind)
     freqs = _freqs(params, D)
@@ -413,13 +408,9 @@ def prefill_backward_dq_rows(q, k, v, dout, params, rows, stage_bf16: bool = Fal
     local = (rows[:, None] - t_all[None, :]) <= int(params.w0)
     stage = round_bf16 if stage_bf16 else (lambda a: a)
 
-    def rot(x, pos):
-        return x if kind == NOPE else rotate(x, pos, freqs, pr)
-
     def srot(x, pos):
         return x if kind == NOPE else stage(rotate(x, pos, freqs, pr))
 
-    dq = np.zeros((B, len(rows), len(heads), D))
     for b in range(B):
         keys = {}
         for j, h in enumerate(heads):
@@ -430,22 +421,91 @@ def prefill_backward_dq_rows(q, k, v, dout, params, rows, stage_bf16: bool = Fal
             kl, kr, vv = keys[hk]
             qq = to_f64(q[b, rows, h])
             ql = srot(qq, p_loc[rows])
+            qr = srot(qq, p_rem[rows]) if kind == BIFOCAL else None
             sc = ql @ kl.T
             if kind == BIFOCAL:
-                qr = srot(qq, p_rem[rows])
                 sc = np.where(local, sc, qr @ kr.T)
             sc = np.where(ok, sc * scale, -np.inf)
             m = sc.max(axis=1, keepdims=True)
             e = np.where(ok, np.exp(sc - m), 0.0)
             P = e / e.sum(axis=1, keepdims=True)
-            dP = to_f64(dout[b, rows, h]) @ vv.T
+            do = to_f64(dout[b, rows, h])
+            dP = do @ vv.T
             dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))
-            if kind == BIFOCAL:
-                dSl, dSr = np.where(local, dS, 0.0), np.where(local, 0.0, dS)
-                dq[b, :, j] = scale * (rot(dSl @ kl, -p_loc[rows]) + rot(dSr @ kr, -p_rem[rows]))
-            else:
-                dq[b, :, j] = scale * rot(dS @ kl, -p_loc[rows])
+            yield dict(b=b, j=j, h=h, hk=hk, P=P, dS=dS, do=do, ql=ql, qr=qr, kl=kl, kr=kr, local=local,
+                       scale=scale, kind=kind, freqs=freqs, pr=pr, p_loc=p_loc, p_rem=p_rem)
+
+
+def _unrot(c, x, pos):
+    return x if c["kind"] == NOPE else rotate(x, pos, c["freqs"], c["pr"])
+
+
+def prefill_backward_dq_rows(q, k, v, dout, params, rows, stage_bf16: bool = False, heads=None):
+    """dq of ``prefill_backward`` for the query rows ``rows`` only (and the
+    query heads ``heads``, default all), [B, len(rows), len(heads), D]: the
+    same chain rule, one block of rows at a time,
+      dq_t = scale * sum_s dS(t,s) R_a^T R_b k_s,
+      dS(t,s) = P(t,s) (dout_t . v_s - sum_s' P(t,s') dout_t . v_s'),
+    with P the row softmax of scale * score(t,s) over the allowed keys
+    (Periodic RoPE §3.1 Eq. 2, §3.2 Eq. 4; Jet-Long §3 Eq. 1, §3.1 Eq. 2-3),
+    split by the window into a local and a remote part for BIFOCAL."""
+    B, S, Hq, D = q.shape
+    heads = list(range(Hq)) if heads is None else list(heads)
+    rows = np.asarray(rows, dtype=np.int64)
+    dq = np.zeros((B, len(rows), len(heads), D))
+    for c in _backward_rows(q, k, v, dout, params, rows, stage_bf16, heads):
+        dS, scale = c["dS"], c["scale"]
+        if c["kind"] == BIFOCAL:
+            dSl, dSr = np.where(c["local"], dS, 0.0), np.where(c["local"], 0.0, dS)
+            g = _unrot(c, dSl @ c["kl"], -c["p_loc"][rows]) + _unrot(c, dSr @ c["kr"], -c["p_rem"][rows])
+        else:
+            g = _unrot(c, dS @ c["kl"], -c["p_loc"][rows])
+        dq[c["b"], :, c["j"]] = scale * g
     return dq
+
+
+def prefill_backward_tail(q, k, v, dout, params, n: int, stage_bf16: bool = False, heads=None):
+    """(dq, dk, dv) of ``prefill_backward`` on the last ``n`` positions: dq of
+    the query rows [S-n, S) for the query heads ``heads`` ([B, n, len(heads),
+    D]) and dk, dv of the keys [S-n, S) for the KV heads those query heads
+    belong to ([B, n, len(kv heads), D], kv heads in increasing order).
+    Attention is causal for every kind, so a key s receives dk and dv only
+    from the rows t >= s; for the tail keys those rows are the tail rows,
+    and the sums
+      dv_s = sum_t P(t,s) dout_t,   dk_s = scale * sum_t dS(t,s) R_b^T R_a q_t
+    over them are complete. ``heads`` must hold whole GQA groups (dk and dv
+    of a KV head collect all the heads of its group)."""
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    grp = Hq // Hkv
+    heads = list(range(Hq)) if heads is None else list(heads)
+    kvh = sorted({h // grp for h in heads})
+    for hk in kvh:
+        if not set(range(hk * grp, (hk + 1) * grp)) <= set(heads):
+            raise ValueError(f"heads must hold the whole GQA group of kv head {hk}")
+    n = int(n)
+    if not 0 <= n <= S:
+        raise ValueError("n must lie in [0, S]")
+    rows = np.arange(S - n, S, dtype=np.int64)
+    dq = np.zeros((B, n, len(heads), D))
+    dk = np.zeros((B, n, len(kvh), D))
+    dv = np.zeros((B, n, len(kvh), D))
+    if n == 0:
+        return dq, dk, dv
+    for c in _backward_rows(q, k, v, dout, params, rows, stage_bf16, heads):
+        b, x, scale = c["b"], kvh.index(c["hk"]), c["scale"]
+        P, dS = c["P"][:, rows], c["dS"]
+        dv[b, :, x] += P.T @ c["do"]
+        if c["kind"] == BIFOCAL:
+            dSl, dSr = np.where(c["local"], dS, 0.0), np.where(c["local"], 0.0, dS)
+            dq[b, :, c["j"]] = scale * (_unrot(c, dSl @ c["kl"], -c["p_loc"][rows])
+                                        + _unrot(c, dSr @ c["kr"], -c["p_rem"][rows]))
+            dk[b, :, x] += scale * (_unrot(c, dSl[:, rows].T @ c["ql"], -c["p_loc"][rows])
+                                    + _unrot(c, dSr[:, rows].T @ c["qr"], -c["p_rem"][rows]))
+        else:
+            dq[b, :, c["j"]] = scale * _unrot(c, dS @ c["kl"], -c["p_loc"][rows])
+            dk[b, :, x] += scale * _unrot(c, dS[:, rows].T @ c["ql"], -c["p_loc"][rows])
+    return dq, dk, dv
 
 
 # ----------------------------------------------------------------------------

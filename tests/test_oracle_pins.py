@@ -724,3 +724,34 @@ def test_backward_dq_rows_is_the_backward_on_those_rows(params, staged):
     dq_rows = O.prefill_backward_dq_rows(q, k, v, dout, params, rows, stage_bf16=staged, heads=heads)
     ref = dq[:, rows][:, :, heads]
     assert np.max(np.abs(dq_rows - ref)) <= 1e-12 * max(1.0, np.max(np.abs(ref)))
+
+
+@pytest.mark.parametrize("params", [
+    MapParams(O.STANDARD, rope_base=1e4),
+    MapParams(O.ENDPROMPT, rope_base=5e5, interp=8.0, seg1_len=25, term_start=60000),
+    MapParams(O.PERIODIC, rope_base=1e4, window=9),
+    MapParams(O.NOPE),
+    MapParams(O.BIFOCAL, rope_base=1e6, w0=6, w_pretrained=12),
+    MapParams(O.BIFOCAL, rope_base=1e4, w0=3, fixed_group=3, pairing=1),
+], ids=["standard", "endprompt", "periodic", "nope", "bifocal", "bifocal_fixed_half"])
+@pytest.mark.parametrize("staged", [False, True])
+def test_backward_tail_is_the_backward_on_the_last_positions(params, staged):
+    # causal attention: the last n keys get dk, dv only from the last n rows,
+    # so the tail function's sums are complete and equal the whole-prefill
+    # backward there (n = 0, a ragged n and the whole sequence)
+    q, k, v = make_qkv(2, 40, 4, 2, 16, seed=53)
+    g = torch.Generator("cpu").manual_seed(54)
+    dout = torch.randn((2, 40, 4, 16), generator=g).to(torch.bfloat16)
+    dq, dk, dv = O.prefill_backward(q, k, v, dout, params, stage_bf16=staged)
+    heads = [2, 3]                                    # the GQA group of kv head 1
+    for n in (0, 7, 40):
+        tq, tk, tv = O.prefill_backward_tail(q, k, v, dout, params, n, stage_bf16=staged, heads=heads)
+        assert tq.shape == (2, n, 2, 16) and tk.shape == tv.shape == (2, n, 1, 16)
+        for got, ref in ((tq, dq[:, 40 - n:][:, :, heads]), (tk, dk[:, 40 - n:, 1:2]), (tv, dv[:, 40 - n:, 1:2])):
+            assert np.max(np.abs(got - ref), initial=0.0) <= 1e-12 * max(1.0, np.max(np.abs(ref), initial=0.0))
+
+
+def test_backward_tail_needs_whole_groups():
+    q, k, v = make_qkv(1, 10, 4, 2, 16, seed=55)
+    with pytest.raises(ValueError):
+        O.prefill_backward_tail(q, k, v, q, MapParams(O.NOPE), 3, heads=[0, 2, 3])
