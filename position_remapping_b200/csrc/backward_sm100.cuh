@@ -36,8 +36,9 @@
 // half of the 64 columns of a score tile and half of the accumulator columns
 // in the epilogue; TMEM lane = row), 8 TMA producer, 9 and 10 issue the two
 // score-side MMAs (S and dP), 11 issues the gradient MMAs. TMEM (512
-// columns): S[2] at [0,64) and [64,128), dP[2] at [128,256), then the
-// accumulators (kernel A: dV and dK, D columns each; kernel B: dQ). The bf16
+// columns): kernel A S[2] at [0,64) and [64,128), dP[2] at [128,256), then
+// dV and dK, D columns each; kernel B three sets, S[3] at [0,192), dP[3] at
+// [192,384), then dQ (a third set fits beside one accumulator). The bf16
 // P and dS of a warpgroup's 32 columns are packed into the first 16 of those
 // columns, where only that warpgroup reads the fp32 scores.
 #pragma once
@@ -539,8 +540,11 @@ struct BwdQSmem {
   static constexpr int kRing = 2 * kQTile;                 // [slot]{K tile, V tile}
   static constexpr int kSlotBytes = 2 * kKTile;
   static constexpr int kBar = kRing + kSlots * kSlotBytes;
-  // q_full, q_free, ring_full[S], ring_empty[S], s_full[2], dp_full[2], p_full[2], sd_free[2], dq_free
-  static constexpr int kNumBars = 3 + 2 * kSlots + 8;
+  // S/dP buffer sets in TMEM: three (S 3 x 64, dP 3 x 64 and dQ D columns fit
+  // in 512), so the chain S -> dS -> dQ MMA of one set spans three tiles
+  static constexpr int kBufs = 3;
+  // q_full, q_free, dq_free, ring_full[S], ring_empty[S], s_full[B], dp_full[B], p_full[B], sd_free[B]
+  static constexpr int kNumBars = 3 + 2 * kSlots + 4 * kBufs;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kTotal = kMisc + 16;
   static constexpr int kAlloc = kTotal + 1024;
@@ -555,7 +559,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                   const BwdParams p) {
   using L = BwdQSmem<D>;
   constexpr int NS = L::kSlots;
+  constexpr int NB = L::kBufs;
   constexpr int kCB = D / 64;
+  static_assert(2 * NB * kBwdN + D <= 512, "TMEM columns");
   constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBwdN, false);   // queries x 64 keys
   constexpr uint32_t kIdescG = idesc_bf16_f32(kBM, D, true);        // queries x D, B MN-major
 
@@ -568,9 +574,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* ring_full = bars + 3;
   uint64_t* ring_empty = ring_full + NS;
   uint64_t* s_full = ring_empty + NS;
-  uint64_t* dp_full = s_full + 2;
-  uint64_t* p_full = dp_full + 2;
-  uint64_t* sd_free = p_full + 2;
+  uint64_t* dp_full = s_full + NB;
+  uint64_t* p_full = dp_full + NB;
+  uint64_t* sd_free = p_full + NB;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
@@ -614,7 +620,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(ring_full + i, 1);
       mbar_init(ring_empty + i, 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < NB; ++a) {
       mbar_init(s_full + a, 1);
       mbar_init(dp_full + a, 1);
       mbar_init(p_full + a, 2 * kBM);
@@ -631,7 +637,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tDP = tmem + 128, tDQ = tmem + 256;
+  const uint32_t tS = tmem, tDP = tmem + NB * kBwdN, tDQ = tmem + 2 * NB * kBwdN;
 
   if (warp == kBwdWarpTMA) {
     // ------------------------------------------------------------------ TMA
@@ -673,9 +679,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (!mbar_wait(q_full, pi & 1, abort_flag)) break;
         const int T = passes[pi].j_hi - passes[pi].j_lo + 1;
         for (int step = 0; step < T; ++step, ++g) {
-          const int slot = g % NS, buf = g & 1;
+          const int slot = g % NS, buf = g % NB;
           if (!mbar_wait(ring_full + slot, (g / NS) & 1, abort_flag)) { ok = false; break; }
-          if (g >= 2 && !mbar_wait(sd_free + buf, ((g >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+          if (g >= NB && !mbar_wait(sd_free + buf, ((g / NB) - 1) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t baddr = smem_u32(smem + L::kRing + slot * L::kSlotBytes + (is_s ? 0 : L::kKTile));
 #pragma unroll
@@ -696,8 +702,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int pi = 0; pi < npass && ok; ++pi) {
         const int T = passes[pi].j_hi - passes[pi].j_lo + 1;
         for (int step = 0; step < T; ++step, ++g) {
-          const int slot = g % NS, buf = g & 1;
-          if (!mbar_wait(p_full + buf, (g >> 1) & 1, abort_flag)) { ok = false; break; }
+          const int slot = g % NS, buf = g % NB;
+          if (!mbar_wait(p_full + buf, (g / NB) & 1, abort_flag)) { ok = false; break; }
           if (step == 0 && pi > 0 && !mbar_wait(dq_free, (pi - 1) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t kaddr = smem_u32(smem + L::kRing + slot * L::kSlotBytes);
@@ -733,9 +739,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const BwdKVPass ps = passes[pi];
       const int T = ps.j_hi - ps.j_lo + 1;
       for (int step = 0; step < T; ++step, ++g) {
-        const int buf = g & 1;
+        const int buf = g % NB;
         const int kv0 = (ps.j_lo + step) * kBwdN;
-        if (!wwait(s_full + buf, (g >> 1) & 1) || !wwait(dp_full + buf, (g >> 1) & 1)) { ok = false; break; }
+        if (!wwait(s_full + buf, (g / NB) & 1) || !wwait(dp_full + buf, (g / NB) & 1)) { ok = false; break; }
         tc_fence_after();
         uint32_t sv[32], dv[32];
         tmem_ld32(tS + buf * kBwdN + hw * 32 + lane_off, sv);
@@ -763,7 +769,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!ok) break;
       // ---- pass epilogue: dQ of this map, turned back and scaled; this
       // warpgroup's half of the columns
-      if (!wwait(sd_free + ((g - 1) & 1), ((g - 1) >> 1) & 1)) { ok = false; break; }
+      if (!wwait(sd_free + ((g - 1) % NB), ((g - 1) / NB) & 1)) { ok = false; break; }
       tc_fence_after();
       float gq[D / 2];
       const float2* tab = p.tab0 == nullptr ? nullptr
