@@ -243,8 +243,9 @@ struct BwdKVSmem {
   static constexpr int kSlotBytes = 2 * kQTile;
   static constexpr int kLD = kRing + kSlots * kSlotBytes;  // [slot]{lse2[64], delta[64]}
   static constexpr int kBar = kLD + kSlots * 2 * kBwdN * 4;
-  // kv_full, ring_full[S], ring_empty[S], s_full[2], dp_full[2], p_full[2], sd_free[2], dk_free
-  static constexpr int kNumBars = 2 + 2 * kSlots + 8;
+  // kv_full, ring_full[S], ring_empty[S], s_full[2], dp_full[2], p_full[2], sd_free[2], dk_free,
+  // s_free[2]
+  static constexpr int kNumBars = 2 + 2 * kSlots + 10;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kTotal = kMisc + 16;
   static constexpr int kAlloc = kTotal + 1024;
@@ -280,6 +281,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* p_full = dp_full + 2;
   uint64_t* sd_free = p_full + 2;
   uint64_t* dk_free = sd_free + 2;
+  uint64_t* s_free = dk_free + 1;   // the dV MMAs of the buffer's step are done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
@@ -323,6 +325,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(dp_full + a, 1);
       mbar_init(p_full + a, 2 * kBM);
       mbar_init(sd_free + a, 1);
+      mbar_init(s_free + a, 1);
     }
     mbar_init(dk_free, 2 * kBM);
     *abort_flag = 0;
@@ -387,8 +390,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int step = 0; step < grp * T; ++step, ++g) {
           const int slot = g % NS, buf = g & 1;
           if (!mbar_wait(ring_full + slot, (g / NS) & 1, abort_flag)) { ok = false; break; }
-          // the buffer's P^T / dS^T of step g - 2 have been read by its gradient MMAs
-          if (g >= 2 && !mbar_wait(sd_free + buf, ((g >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+          // the buffer's P^T (S^T side) or dS^T (dP^T side) of step g - 2 has
+          // been read by its dV or dK MMAs; S^T is queued behind the dK MMAs
+          if (g >= 2 && !mbar_wait((is_s ? s_free : sd_free) + buf, ((g >> 1) - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const uint32_t baddr = smem_u32(smem + L::kRing + slot * L::kSlotBytes + (is_s ? 0 : L::kQTile));
 #pragma unroll
@@ -421,6 +428,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             umma_ts(tDV, tS + buf * kBwdN + bwd_pcol(kk), sdesc_sw128(oaddr + kk * 2048, kBwdN * 128, 1024),
                     kIdescG, (g > 0 || kk > 0) ? 1u : 0u);
           }
+          umma_commit(s_free + buf);
 #pragma unroll
           for (int kk = 0; kk < kBwdN / 16; ++kk) {
             umma_ts(tDK, tDP + buf * kBwdN + bwd_pcol(kk), sdesc_sw128(qaddr + kk * 2048, kBwdN * 128, 1024),
