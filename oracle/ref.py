@@ -533,7 +533,7 @@ def cache_keys(k, params, start: int = 0):
     return out
 
 
-def prefill_from_cache(q, k_cache, v_cache, params, start: int, stage_bf16: bool = True):
+def prefill_from_cache(q, k_cache, v_cache, params, start: int, stage_bf16: bool = True, rows=None, heads=None):
     """Rows start..L-1 of a prefill of length L = k_cache.shape[1] whose keys
     come from a decode cache (Eq. 4: k_cache[s] = RoPE(x_s, p(s))) instead of
     raw keys: q [B,count,Hq,D] holds the unrotated queries of tokens
@@ -542,11 +542,17 @@ def prefill_from_cache(q, k_cache, v_cache, params, start: int, stage_bf16: bool
     rotation by Delta s = f(s) - s (Eq. 5-6, as in decode) against the query
     rotated to f(t). ``stage_bf16`` rounds the rotated queries and the
     corrected remote keys to bf16 (the cache itself is taken as given).
-    Returns out [B,count,Hq,D], lse [B,Hq,count]."""
-    q, kc, vc = to_f64(q), to_f64(k_cache), to_f64(v_cache)
+    ``rows`` (token indices in [start, L)) and ``heads`` (query heads)
+    restrict the result to those rows and heads, for checks at lengths where
+    every row is out of reach; only the slices they need are taken to
+    float64. Returns out [B,R,H,D], lse [B,H,R] (R rows, H heads; by default
+    every row start..L-1 and every head)."""
     B, count, Hq, D = q.shape
-    L, Hkv = kc.shape[1], kc.shape[2]
+    L, Hkv = k_cache.shape[1], k_cache.shape[2]
     assert count == L - int(start)
+    rows = np.arange(int(start), L) if rows is None else np.asarray(rows, dtype=np.int64)
+    assert rows.size == 0 or (rows.min() >= int(start) and rows.max() < L)
+    heads = list(range(Hq)) if heads is None else list(heads)
     grp = Hq // Hkv
     scale = softmax_scale(D, params)
     kind = int(params.kind)
@@ -555,19 +561,21 @@ def prefill_from_cache(q, k_cache, v_cache, params, start: int, stage_bf16: bool
     p_loc, p_rem, G = position_maps(params, L)
     stage = round_bf16 if stage_bf16 else (lambda a: a)
     keys = np.arange(L)
-    rows = np.arange(int(start), L)
-    out = np.zeros((B, count, Hq, D))
-    lse = np.zeros((B, Hq, count))
+    out = np.zeros((B, rows.size, len(heads), D))
+    lse = np.zeros((B, len(heads), rows.size))
     for b in range(B):
-        for hk in range(Hkv):
-            kl = kc[b, :, hk]
+        for hk in sorted({h // grp for h in heads}):
+            kl = to_f64(k_cache[b, :, hk])
+            vv = to_f64(v_cache[b, :, hk])
             kr = stage(rotate(kl, p_rem - keys, freqs, pr)) if kind == BIFOCAL else None   # Eq. 6, keys
-            for h in range(hk * grp, (hk + 1) * grp):
-                for c0 in range(0, count, 64):
+            for j, h in enumerate(heads):
+                if h // grp != hk:
+                    continue
+                for c0 in range(0, rows.size, 64):
                     rr = rows[c0:c0 + 64]
                     nk = int(rr.max()) + 1
                     ok = np.stack([_allowed(params, int(t), keys[:nk]) for t in rr])
-                    qq = q[b, rr - int(start), h, :]
+                    qq = to_f64(q[b, rr - int(start), h, :])
                     ql = qq if kind == NOPE else stage(rotate(qq, p_loc[rr], freqs, pr))
                     sc = (ql @ kl[:nk].T) * scale
                     if kind == BIFOCAL:
@@ -575,9 +583,9 @@ def prefill_from_cache(q, k_cache, v_cache, params, start: int, stage_bf16: bool
                         sr = (qr @ kr[:nk].T) * scale
                         local = (rr[:, None] - keys[None, :nk]) <= int(params.w0)
                         sc = np.where(local, sc, sr)
-                    o, l = _softmax_rows(sc, ok, vc[b, :nk, hk, :])
-                    out[b, c0:c0 + 64, h, :] = o
-                    lse[b, h, c0:c0 + 64] = l
+                    o, l = _softmax_rows(sc, ok, vv[:nk])
+                    out[b, c0:c0 + 64, j, :] = o
+                    lse[b, j, c0:c0 + 64] = l
     return out, lse
 
 

@@ -477,6 +477,15 @@ def test_prefill_from_cache_equals_prefill_rows(kind):
         a = O.prefill_from_cache(qn[:, start:], cache, vn, params, start, stage_bf16=False)
         b = O.prefill(qn, kn, vn, params, rows=list(range(start, 27)), stage_bf16=False)
         assert np.allclose(a[0], b[0], atol=1e-12) and np.allclose(a[1], b[1], atol=1e-12)
+        # the row and head selection (used at full size) picks the same values
+        rows, heads = [r for r in (start, 20, 26) if r >= start], [3, 0]
+        for staged in (False, True):
+            full = O.prefill_from_cache(qn[:, start:], cache, vn, params, start, stage_bf16=staged)
+            sel = O.prefill_from_cache(q[:, start:], cache, v, params, start, stage_bf16=staged, rows=rows,
+                                       heads=heads)
+            idx = [r - start for r in rows]
+            assert np.allclose(sel[0], full[0][:, idx][:, :, heads], rtol=0, atol=1e-12)
+            assert np.allclose(sel[1], full[1][:, heads][:, :, idx], rtol=0, atol=1e-12)
 
 
 def test_fixed_group_positions_and_brute_force():
