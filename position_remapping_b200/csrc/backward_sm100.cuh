@@ -37,8 +37,9 @@
 // in the epilogue; TMEM lane = row), 8 TMA producer, 9 and 10 issue the two
 // score-side MMAs (S and dP), 11 issues the gradient MMAs. TMEM (512
 // columns): kernel A S[2] at [0,64) and [64,128), dP[2] at [128,256), then
-// dV and dK, D columns each; kernel B three sets, S[3] at [0,192), dP[3] at
-// [192,384), then dQ (a third set fits beside one accumulator). The bf16
+// dV and dK, D columns each (three sets at D = 64, where they fit); kernel B
+// three sets, S[3] at [0,192), dP[3] at [192,384), then dQ (a third set fits
+// beside one accumulator). The bf16
 // P and dS of a warpgroup's 32 columns are packed into the first 16 of those
 // columns, where only that warpgroup reads the fp32 scores.
 #pragma once
@@ -243,9 +244,12 @@ struct BwdKVSmem {
   static constexpr int kSlotBytes = 2 * kQTile;
   static constexpr int kLD = kRing + kSlots * kSlotBytes;  // [slot]{lse2[64], delta[64]}
   static constexpr int kBar = kLD + kSlots * 2 * kBwdN * 4;
-  // kv_full, ring_full[S], ring_empty[S], s_full[2], dp_full[2], p_full[2], sd_free[2], dk_free,
-  // s_free[2]
-  static constexpr int kNumBars = 2 + 2 * kSlots + 10;
+  // S^T/dP^T buffer sets in TMEM: three where they fit beside dV and dK
+  // (D = 64: 3 x 64 + 3 x 64 + 2 x 64 = 512 columns), else two
+  static constexpr int kBufs = 2 * 3 * kBwdN + 2 * D <= 512 ? 3 : 2;
+  // kv_full, ring_full[S], ring_empty[S], s_full[B], dp_full[B], p_full[B], sd_free[B], dk_free,
+  // s_free[B]
+  static constexpr int kNumBars = 2 + 2 * kSlots + 5 * kBufs + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kTotal = kMisc + 16;
   static constexpr int kAlloc = kTotal + 1024;
@@ -266,6 +270,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     const BwdParams p) {
   using L = BwdKVSmem<D>;
   constexpr int NS = L::kSlots;
+  constexpr int NB = L::kBufs;
+  static_assert(2 * NB * kBwdN + 2 * D <= 512, "TMEM columns");
   constexpr int kCB = D / 64;
   constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBwdN, false);   // keys x 64 queries
   constexpr uint32_t kIdescG = idesc_bf16_f32(kBM, D, true);        // keys x D, B MN-major
@@ -277,10 +283,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* ring_full = bars + 1;
   uint64_t* ring_empty = ring_full + NS;
   uint64_t* s_full = ring_empty + NS;
-  uint64_t* dp_full = s_full + 2;
-  uint64_t* p_full = dp_full + 2;
-  uint64_t* sd_free = p_full + 2;
-  uint64_t* dk_free = sd_free + 2;
+  uint64_t* dp_full = s_full + NB;
+  uint64_t* p_full = dp_full + NB;
+  uint64_t* sd_free = p_full + NB;
+  uint64_t* dk_free = sd_free + NB;
   uint64_t* s_free = dk_free + 1;   // the dV MMAs of the buffer's step are done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
@@ -320,7 +326,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(ring_full + i, 1);
       mbar_init(ring_empty + i, 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < NB; ++a) {
       mbar_init(s_full + a, 1);
       mbar_init(dp_full + a, 1);
       mbar_init(p_full + a, 2 * kBM);
@@ -339,7 +345,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tDP = tmem + 128, tDV = tmem + 256, tDK = tmem + 256 + D;
+  const uint32_t tS = tmem, tDP = tmem + NB * kBwdN, tDV = tmem + 2 * NB * kBwdN, tDK = tDV + D;
 
   if (warp == kBwdWarpTMA) {
     // ------------------------------------------------------------------ TMA
@@ -388,11 +394,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t aaddr = smem_u32(smem + (is_s ? (passes[pi].sel ? L::kK1 : L::kK0) : L::kV));
         const int T = passes[pi].j_hi - passes[pi].j_lo + 1;
         for (int step = 0; step < grp * T; ++step, ++g) {
-          const int slot = g % NS, buf = g & 1;
+          const int slot = g % NS, buf = g % NB;
           if (!mbar_wait(ring_full + slot, (g / NS) & 1, abort_flag)) { ok = false; break; }
-          // the buffer's P^T (S^T side) or dS^T (dP^T side) of step g - 2 has
+          // the buffer's P^T (S^T side) or dS^T (dP^T side) of step g - NB has
           // been read by its dV or dK MMAs; S^T is queued behind the dK MMAs
-          if (g >= 2 && !mbar_wait((is_s ? s_free : sd_free) + buf, ((g >> 1) - 1) & 1, abort_flag)) {
+          if (g >= NB && !mbar_wait((is_s ? s_free : sd_free) + buf, ((g / NB) - 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
@@ -416,8 +422,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int pi = 0; pi < npass && ok; ++pi) {
         const int T = passes[pi].j_hi - passes[pi].j_lo + 1;
         for (int step = 0; step < grp * T; ++step, ++g) {
-          const int slot = g % NS, buf = g & 1;
-          if (!mbar_wait(p_full + buf, (g >> 1) & 1, abort_flag)) { ok = false; break; }
+          const int slot = g % NS, buf = g % NB;
+          if (!mbar_wait(p_full + buf, (g / NB) & 1, abort_flag)) { ok = false; break; }
           // the previous pass's dK has been read out (parked) before it is reset
           if (step == 0 && pi > 0 && !mbar_wait(dk_free, (pi - 1) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
@@ -456,10 +462,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const BwdKVPass ps = passes[pi];
       const int T = ps.j_hi - ps.j_lo + 1;
       for (int step = 0; step < grp * T; ++step, ++g) {
-        const int slot = g % NS, buf = g & 1;
+        const int slot = g % NS, buf = g % NB;
         const int j = ps.j_lo + step % T;
-        if (!wwait(ring_full + slot, (g / NS) & 1) || !wwait(s_full + buf, (g >> 1) & 1) ||
-            !wwait(dp_full + buf, (g >> 1) & 1)) {
+        if (!wwait(ring_full + slot, (g / NS) & 1) || !wwait(s_full + buf, (g / NB) & 1) ||
+            !wwait(dp_full + buf, (g / NB) & 1)) {
           ok = false;
           break;
         }
@@ -494,7 +500,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!ok) break;
       // ---- pass epilogue: dK of this map, turned back and scaled; this
       // warpgroup's half of the columns
-      if (!wwait(sd_free + ((g - 1) & 1), ((g - 1) >> 1) & 1)) { ok = false; break; }
+      if (!wwait(sd_free + ((g - 1) % NB), ((g - 1) / NB) & 1)) { ok = false; break; }
       tc_fence_after();
       float gk[D / 2];
       const float2* tab = p.tab0 == nullptr ? nullptr
@@ -508,7 +514,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
     // ---- dV (every pass and head), after the last gradient MMA
-    if (ok && g > 0 && wwait(sd_free + ((g - 1) & 1), ((g - 1) >> 1) & 1)) {
+    if (ok && g > 0 && wwait(sd_free + ((g - 1) % NB), ((g - 1) / NB) & 1)) {
       tc_fence_after();
       float gv[D / 2];
       grad_half_from_tmem<D>(tDV + lane_off, 1.0f, nullptr, hw * (D / 2), gv);
