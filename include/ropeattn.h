@@ -195,7 +195,9 @@ int ropeattn_prefill_attend(const void* q, const void* k, const void* v, float* 
 
 /* Workspace bytes of ropeattn_prefill_backward: per position map the rotated
  * queries and keys (bf16) and the angle table, plus the log-sum-exp in log2
- * units and Delta (fp32, rows padded to a multiple of 64). */
+ * units and Delta (fp32, rows padded to a multiple of 64). 0 for arguments
+ * the backward rejects (head_dim other than 64 and 128 among them) and for
+ * an empty problem. */
 size_t ropeattn_prefill_backward_workspace_size(const ropeattn_params* params, int64_t B, int64_t S,
                                                 int32_t Hq, int32_t Hkv, int32_t D);
 

@@ -1071,7 +1071,9 @@ extern "C" size_t ropeattn_prefill_backward_workspace_size(const ropeattn_params
                                                            int32_t Hq, int32_t Hkv, int32_t D) {
   PosMap m;
   int eff;
-  if (check_shapes(B, S, Hq, Hkv, D) || check_params(params, S, D, &m, &eff) || B == 0 || S == 0) return 0;
+  if (check_shapes(B, S, Hq, Hkv, D) || (D != 64 && D != 128) || check_params(params, S, D, &m, &eff) || B == 0 ||
+      S == 0)
+    return 0;
   return bwd_layout(eff, B, S, Hq, Hkv, D).total;
 }
 

@@ -98,6 +98,14 @@ def test_host_argument_checks(ra):
     assert lib.ropeattn_prefill_three_call_workspace_size(bif, 1, 4096, 2, 1, 256) > \
         lib.ropeattn_prefill_workspace_size(bif, 1, 4096, 2, 1, 256) > 0
     assert lib.ropeattn_decode_workspace_size(1, 1000, 2, 1, 256) > 0
+    # the backward offers head_dim 64 and 128 only: no workspace size and a
+    # rejection before any device work for 256
+    std = ctypes.byref(cp(_p(kind=STANDARD)))
+    assert lib.ropeattn_prefill_backward_workspace_size(std, 1, 4096, 2, 1, 128) > 0
+    assert lib.ropeattn_prefill_backward_workspace_size(std, 1, 4096, 2, 1, 256) == 0
+    assert lib.ropeattn_prefill_backward(nullp, nullp, nullp, nullp, nullp, nullp, nullp, nullp, nullp, 1, 4096, 2, 1,
+                                         256, std, nullp, 0, nullp) == ra.ERR_INVALID_ARG
+    assert "64 and 128" in lib.ropeattn_last_error().decode()
     assert lib.ropeattn_decode(nullp, nullp, nullp, nullp, nullp, 1, 1000, 32, 1, 256,
                                ctypes.byref(cp(_p(kind=STANDARD))), nullp, 0, nullp) == ra.ERR_INVALID_ARG  # GQA 32
     assert "16" in lib.ropeattn_last_error().decode()
